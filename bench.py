@@ -1,0 +1,477 @@
+#!/usr/bin/env python
+"""Benchmark of the routed MoE FFN layer on B200 (one JSON line on stdout, rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one moe_forward of the whole layer (router -> top-k -> bucketing -> experts ->
+combine with the shared expert) over one batch of synthetic tokens.  Workloads (seed 0,
+synthetic inputs of the pages' model shapes; no datasets or trained weights):
+
+  glm_decode   (default) GLM-5.2-like layer, T=1: d=6144, E=256, top-8 sigmoid router with
+               selection bias, x2.5 scaling, f=2048 int4 experts (+1 shared), ~4.8 GB resident
+  glm_union2   the same layer, T=2 (batch-union)
+  glm_union32  the same layer, T=32 (batch-union)
+  glm_prefill  the same layer, T=2048, bf16 output
+  granite      Granite-1B-a400m-like decode layer: T=1, d=1024, E=32, top-8 softmax, f=512 bf16
+  tiny         T=4, d=256, E=8, top-2 softmax, f=128 int4
+
+Timing: CUDA events on the launching stream around every step; L2 is flushed (a 512 MiB
+write) between steps, outside the events.  Multi-GPU: one process per GPU, each a data-parallel
+replica with its own token stream; value = all ranks' tokens / max over ranks of device time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synthetic as syn  # noqa: E402
+
+METRIC = "MoE-layer tokens/s"
+WORKLOADS = {
+    "glm_decode": "GLM-5.2-like MoE layer decode, T=1, d=6144, E=256, top-8 sigmoid+bias x2.5, f=2048 int4 + 1 shared",
+    "glm_union2": "GLM-5.2-like MoE layer batch-union decode, T=2",
+    "glm_union32": "GLM-5.2-like MoE layer batch-union decode, T=32",
+    "glm_prefill": "GLM-5.2-like MoE layer prefill, T=2048, bf16 out",
+    "granite": "Granite-1B-a400m-like MoE layer decode, T=1, d=1024, E=32, top-8 softmax, f=512 bf16",
+    "tiny": "tiny MoE layer, T=4, d=256, E=8, top-2 softmax, f=128 int4",
+}
+DEFAULT_STEPS = {"glm_decode": 400, "glm_union2": 300, "glm_union32": 100, "glm_prefill": 30, "granite": 2000,
+                 "tiny": 200}
+FLUSH_BYTES = 512 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="glm_decode", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+    if a.steps is None:
+        a.steps = DEFAULT_STEPS[a.workload]
+    a.warmup = max(a.warmup, 3)
+    return a
+
+
+def expert_bytes(cfg, f=None) -> int:
+    f = cfg.f if f is None else f
+    if cfg.wkind == syn.W_INT4:
+        return 2 * f * (cfg.d // 2 + 4) + cfg.d * (f // 2 + 4)
+    return 2 * f * cfg.d * 2 + cfg.d * f * 2
+
+
+# ------------------------------------------------------------------------------------------
+# device-side layer and inputs
+# ------------------------------------------------------------------------------------------
+
+def build_device_layer(cfg, seed, max_tokens, device):
+    import torch
+
+    import quantized_expert_ffn_02_b200 as qe
+
+    E, d, f = cfg.E, cfg.d, cfg.f
+    int4 = cfg.wkind == syn.W_INT4
+    W = {}
+
+    def mat(name, rows, cols):
+        return syn.torch_normal_fp32(seed, name, rows * cols, syn.WEIGHT_STD, device).view(rows, cols)
+
+    def alloc(prefix, n, f_):
+        if int4:
+            W[prefix + "gate_up"] = torch.empty((n, 2 * f_, d // 2), dtype=torch.uint8, device=device)
+            W[prefix + "gate_up_scale"] = torch.empty((n, 2 * f_), dtype=torch.float32, device=device)
+            W[prefix + "down"] = torch.empty((n, d, f_ // 2), dtype=torch.uint8, device=device)
+            W[prefix + "down_scale"] = torch.empty((n, d), dtype=torch.float32, device=device)
+        else:
+            W[prefix + "gate_up"] = torch.empty((n, 2 * f_, d), dtype=torch.int16, device=device)
+            W[prefix + "down"] = torch.empty((n, d, f_), dtype=torch.int16, device=device)
+
+    def fill(prefix, i, e, f_):
+        for which, rows, cols in (("gate_up", 2 * f_, d), ("down", d, f_)):
+            w = mat(syn.expert_tensor_name(e, which), rows, cols)
+            if int4:
+                qe.moe_pack_int4(w, W[prefix + which][i], W[prefix + which + "_scale"][i])
+            else:
+                W[prefix + which][i].copy_(w.to(torch.bfloat16).view(torch.int16))
+
+    alloc("", E, f)
+    for e in range(E):
+        fill("", e, e, f)
+    if cfg.n_shared:
+        alloc("shared_", 1, cfg.f_shared)
+        fill("shared_", 0, "shared", cfg.f_shared)
+        for key in list(W):
+            if key.startswith("shared_"):
+                W[key] = W[key][0]
+    W["router_w"] = torch.from_numpy(syn.gen_router_w(cfg, seed)).to(device)
+    b = syn.gen_router_bias(cfg, seed)
+    W["router_bias"] = None if b is None else torch.from_numpy(b).to(device)
+    torch.cuda.synchronize()
+    layer = qe.MoELayer(d, f, E, cfg.k, max_tokens, cfg.router, cfg.wkind, W, n_shared=cfg.n_shared,
+                        f_shared=cfg.f_shared, routed_scaling_factor=cfg.scaling, out_bf16=cfg.out_bf16)
+    return layer, W
+
+
+def make_batches(cfg, T, n, seed, token_offset, device):
+    """n batches of T tokens: token stream "x" from `token_offset` on (bf16 bits as int16)."""
+    import torch
+    out = []
+    for i in range(n):
+        v = syn.torch_normal_fp32(seed, "x", T * cfg.d, 1.0, device, offset=(token_offset + i * T) * cfg.d)
+        out.append(v.to(torch.bfloat16).view(torch.int16).view(T, cfg.d))
+    return out
+
+
+# ------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------
+
+class Clocks:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 8:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        load = sorted(sm)[len(sm) // 2:] if sm else []
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------------------
+# oracle CPU baseline (host cores): the plain fp64 oracle as it stands
+# ------------------------------------------------------------------------------------------
+
+def oracle_sample_layer(cfg, seed, x_bits):
+    """Oracle layer holding the experts that the sample's tokens route to (host-drawn)."""
+    import oracle
+    router = oracle.Layer(cfg.d, cfg.f, cfg.E, cfg.k, cfg.router, cfg.scaling, cfg.wkind,
+                          syn.gen_router_w(cfg, seed), syn.gen_router_bias(cfg, seed), f_shared=cfg.f_shared or cfg.f)
+    need = sorted(set(router.route(x_bits)["idx"].reshape(-1).tolist()))
+
+    def host_expert(e):
+        out = {}
+        for which in ("gate_up", "down"):
+            w = syn.gen_expert_fp32(cfg, e, which, seed)
+            if cfg.wkind == syn.W_BF16:
+                out[which] = syn.fp32_to_bf16_bits(w)
+            else:
+                out[which], out[which + "_scale"] = oracle.pack_int4(w)
+        return out
+
+    experts = {e: host_expert(e) for e in need}
+    shared = host_expert("shared") if cfg.n_shared else None
+    return oracle.Layer(cfg.d, cfg.f, cfg.E, cfg.k, cfg.router, cfg.scaling, cfg.wkind, router.router_w,
+                        router.router_bias, experts=experts, shared=shared, f_shared=cfg.f_shared or cfg.f)
+
+
+def oracle_sample_tokens(cfg, name):
+    """Tokens of one oracle sample call: a single token for decode, a slice for the larger batches."""
+    return {"glm_union2": 2, "glm_union32": 2, "glm_prefill": 2}.get(name, cfg.T)
+
+
+def time_oracle(cfg, name, seed, budget_s, min_calls=1, max_calls=None):
+    import oracle
+    n_tok = oracle_sample_tokens(cfg, name)
+    x = syn.gen_x(cfg, seed, T=n_tok)
+    L = oracle_sample_layer(cfg, seed, x)
+    calls, t0 = 0, time.perf_counter()
+    while True:
+        L.forward(x)
+        calls += 1
+        el = time.perf_counter() - t0
+        if calls >= min_calls and (el >= budget_s or (max_calls and calls >= max_calls)):
+            break
+    return {"value": calls * n_tok / el, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{calls} oracle calls of {n_tok} token(s) of the {name} workload ({el:.1f} s on host cores)"}
+
+
+# ------------------------------------------------------------------------------------------
+# roofline helpers
+# ------------------------------------------------------------------------------------------
+
+def kernel_bytes(cfg, T, n_unique):
+    """Algorithmic HBM bytes per launch of the expert kernels for a batch with n_unique routed experts."""
+    S = 1 if cfg.n_shared else 0
+    slots = T * cfg.k + T * S
+    fmax = max(cfg.f, cfg.f_shared if S else 0)
+    q = cfg.wkind == syn.W_INT4
+    gu_rows = n_unique * 2 * cfg.f + S * 2 * cfg.f_shared
+    dn_rows = (n_unique + S) * cfg.d
+    gu = gu_rows * ((cfg.d // 2 + 4) if q else cfg.d * 2) + T * cfg.d * 2 + slots * fmax * 2
+    f_of = lambda ff: (ff // 2 + 4) if q else ff * 2  # noqa: E731
+    dn = n_unique * cfg.d * f_of(cfg.f) + S * cfg.d * f_of(cfg.f_shared) + slots * fmax * 2 + slots * cfg.d * 4
+    return {"gateup": gu, "down": dn}
+
+
+def source_sha(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel):
+    """dram bytes per launch from a committed ncu capture, if the kernel source is unchanged since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path)).get(kernel)
+    if not rec:
+        return None
+    try:
+        if source_sha(rec["sources"]) != rec["source_sha"]:
+            return None
+    except OSError:
+        return None
+    return rec.get("bytes_per_launch")
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return p.get("hbm_gbs", 6650.0), p.get("bf16_tflops", 1590.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------------------------------------
+# arms
+# ------------------------------------------------------------------------------------------
+
+def run_reference(a, rank, world):
+    """The oracle on host cores: each step one bounded oracle call of the workload."""
+    if rank != 0:
+        return
+    cfg = syn.CONFIGS[a.workload]
+    import oracle
+    n_tok = oracle_sample_tokens(cfg, a.workload)
+    x = syn.gen_x(cfg, a.seed, T=n_tok)
+    L = oracle_sample_layer(cfg, a.seed, x)
+    for _ in range(a.warmup):
+        L.forward(x)
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        L.forward(x)
+    el = time.perf_counter() - t0
+    value = a.steps * n_tok / el
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference", "n_gpus": a.gpus,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * el / a.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": a.workload, "desc": WORKLOADS[a.workload], "tokens_per_step": n_tok,
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": f"{a.steps} timed oracle calls of {n_tok} token(s) of {a.workload}"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(a, rank, world, local_rank):
+    import torch
+
+    import quantized_expert_ffn_02_b200 as qe
+
+    cfg = syn.CONFIGS[a.workload]
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    T = cfg.T
+    layer, W = build_device_layer(cfg, a.seed, T, dev)
+    # every rank is an independent replica with its own tokens
+    n_batches = a.warmup + a.steps if T <= 32 else 4
+    token_base = rank * 1_000_000
+    xs = make_batches(cfg, T, n_batches, a.seed, token_base, dev)
+    out = torch.empty((T, cfg.d), dtype=torch.int16 if cfg.out_bf16 else torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    # census of unique experts per batch (outside timing) for the algorithmic byte counts
+    uniq = []
+    idx = torch.empty((T, cfg.k), dtype=torch.int32, device=dev)
+    wts = torch.empty((T, cfg.k), dtype=torch.float32, device=dev)
+    for x in xs:
+        layer.route(x, idx, wts)
+        uniq.append(len(torch.unique(idx).tolist()))
+    torch.cuda.synchronize()
+
+    def bx(i):
+        return xs[i % len(xs)]
+
+    for i in range(a.warmup):
+        layer.forward(bx(i), out)
+    torch.cuda.synchronize()
+    if layer.last_error() != qe.MOE_OK:
+        raise RuntimeError("device status after warm-up: " + qe.status_str(layer.last_error()))
+    launches_per_step = layer.last_launches()
+
+    def timed_pass(profile: bool):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+        layer.profile(profile)
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(a.steps):
+            flush.zero_()
+            evs[i][0].record(stream)
+            layer.forward(bx(a.warmup + i), out)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        layer.profile(False)
+        return sum(s.elapsed_time(e) for s, e in evs)
+
+    clocks = Clocks(local_rank)
+    clocks.start()
+    total_ms = timed_pass(False)
+    clk = clocks.stop()
+    prof_ms = timed_pass(True)
+    prof = layer.profile_read()
+    if layer.last_error() != qe.MOE_OK:
+        raise RuntimeError("device status after timing: " + qe.status_str(layer.last_error()))
+    if dist:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = world * a.steps * T / (total_ms / 1e3)
+
+    # end to end: host buffers through the C ABI, copies inside the timed region
+    xh = [bx(a.warmup + i).cpu().pin_memory() for i in range(min(a.steps, len(xs)))]
+    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e2e_steps = a.steps
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(e2e_steps):
+        layer.forward_host(xh[i % len(xh)], oh)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = t0.elapsed_time(t1)
+    if dist:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": world * e2e_steps * T / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": T * cfg.d * 2, "d2h_bytes_per_step": T * cfg.d * out.element_size()}
+
+    # roofline of the dominant kernel (device time measured by the library's event pairs)
+    hbm, tf, peak_kind = measured_peaks()
+    dom = max(prof, key=lambda k: prof[k][0]) if prof else None
+    roof = None
+    if dom:
+        ms, n = prof[dom]
+        per_launch_ms = ms / n
+        timed_uniq = [uniq[(a.warmup + i) % len(xs)] for i in range(a.steps)]
+        bytes_per = statistics.mean(kernel_bytes(cfg, T, u)[dom] for u in timed_uniq) if dom in ("gateup", "down") \
+            else None
+        if bytes_per:
+            achieved = bytes_per / (per_launch_ms / 1e3) / 1e9
+            roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                    "frac": achieved / hbm, "traffic": traffic_for(dom), "peak_kind": f"{peak_kind} (copy)",
+                    "algorithmic_bytes_per_launch": bytes_per, "ms_per_launch": per_launch_ms}
+    step_bytes = statistics.mean(uniq[(a.warmup + i) % len(xs)] for i in range(a.steps)) * expert_bytes(cfg) + \
+        (expert_bytes(cfg, cfg.f_shared) if cfg.n_shared else 0) + cfg.E * cfg.d * 4
+    ms_per_step = total_ms / a.steps
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4xbf16->f32" if cfg.wkind == syn.W_INT4 else "bf16->f32", "data": "synthetic",
+        "config": {"workload": a.workload, "desc": WORKLOADS[a.workload], "tokens_per_step": T,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed between steps (512 MiB write, outside the step events)",
+                   "weights": "seed 0, drawn on the device by the counter-based generator"},
+        "roofline": roof,
+        "step_hbm": {"gbs": step_bytes / (ms_per_step / 1e3) / 1e9, "frac": step_bytes / (ms_per_step / 1e3) / 1e9 / hbm,
+                     "bytes_per_step": step_bytes, "unique_experts_mean": statistics.mean(uniq)},
+        "kernels": {k: {"ms_per_launch": v[0] / v[1], "launches": v[1]} for k, v in prof.items()},
+        "profiled_ms_per_step": prof_ms / a.steps,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * a.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        line["cpu_baseline"] = time_oracle(cfg, a.workload, a.seed, a.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    layer.close()
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    a = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if a.impl == "reference":
+        run_reference(a, rank, world)
+    else:
+        run_ours(a, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

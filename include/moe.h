@@ -1,0 +1,201 @@
+/*
+ * moe.h -- C ABI of libmoe.so: the forward pass of a routed Mixture-of-Experts FFN layer on
+ * one NVIDIA B200 (sm_100a), for decode (a few tokens) and prefill (thousands of tokens).
+ *
+ * The layer (as the colibri README and the iliria page describe it, sections "The idea" and
+ * "What's implemented", and the Glacial page, section "What works"):
+ *
+ *   1. router: logits[t][e] = sum_i x[t][i] * Wr[e][i]; then either
+ *        softmax top-k (Granite style): the k largest logits, weights = softmax over those k;
+ *        sigmoid + selection bias (DeepSeek-V3 style, "noaux_tc", routed_scaling_factor):
+ *        key = sigmoid(logit) + bias[e] picks the k experts, the weights are
+ *        routed_scaling_factor * sigmoid / (sum of the chosen sigmoids) -- the bias is used
+ *        for selection only;
+ *      equal keys go to the lower expert index; the k outputs of a token are in rank order.
+ *   2. batch-union dispatch: every chosen expert's weights are read once and applied to every
+ *      token routed to it ("Batch-union MoE", colibri README).
+ *   3. SwiGLU experts: g = Wg x, u = Wu x, h = silu(g) * u, y = Wd h, over packed int4 weights
+ *      with one fp32 scale per output row dequantised on use ("Quantization kernels ... packed
+ *      int4 ... per-row scales ... dequant-on-use", colibri README), or over bf16 weights.
+ *   4. combine: out[t] = sum over the chosen experts (ascending expert index) of
+ *      weight * y, plus the shared expert with weight 1 ("shared expert", colibri README).
+ *
+ * Conventions used by every entry point:
+ *   - Pointers marked "device" must point to memory of the CUDA device that was current when
+ *     the layer was created (or, for moe_pack_int4, the current device); "host" means CPU
+ *     memory (pageable or pinned).
+ *   - bf16 data are passed as uint16_t bit patterns.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default stream).  Only
+ *     the calls documented as synchronous wait for the device.
+ *   - No C++ exception or CUDA error escapes: every failure is a moe_status.  Argument errors
+ *     are returned before anything is enqueued.  Errors found by the device while running
+ *     (a bounded wait that ran out, a value out of range) are latched in the layer's device
+ *     status word and returned by moe_last_error().
+ *   - The library never allocates on the hot path: moe_route / moe_forward use the workspace
+ *     that moe_layer_create allocated for `max_tokens` tokens.
+ */
+#ifndef QEFFN_MOE_H
+#define QEFFN_MOE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct moe_layer moe_layer;          /* opaque */
+typedef struct CUstream_st *moe_stream;      /* the same type as cudaStream_t */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,   /* a NULL pointer, a size out of range, a misaligned pointer */
+    MOE_ERR_CUDA = 2,          /* a CUDA runtime call failed (launch, copy, allocation flags) */
+    MOE_ERR_OOM = 3,           /* workspace allocation failed */
+    MOE_ERR_TIMEOUT = 4,       /* a bounded device-side wait gave up */
+    MOE_ERR_RANGE = 5,         /* non-finite weights given to the packer; an fp16 overflow of h */
+    MOE_ERR_UNSUPPORTED = 6    /* a shape this build has no kernel for */
+} moe_status;
+
+enum { MOE_ROUTER_SOFTMAX_TOPK = 0, MOE_ROUTER_SIGMOID_BIAS = 1 };
+enum { MOE_W_INT4_ROWSCALE = 0, MOE_W_BF16 = 1 };
+
+typedef struct {
+    int32_t d;                   /* hidden size; even, and a multiple of 64 */
+    int32_t f;                   /* routed expert intermediate size; a multiple of 64 */
+    int32_t n_experts;           /* E, 1..1024 */
+    int32_t top_k;               /* k, 1..min(E, 32) */
+    int32_t n_shared;            /* 0 or 1 */
+    int32_t f_shared;            /* shared expert intermediate size (multiple of 64); ignored if n_shared == 0 */
+    int32_t max_tokens;          /* largest T that moe_route / moe_forward accept (>= 1) */
+    int32_t router;              /* MOE_ROUTER_* */
+    float routed_scaling_factor; /* multiplies the renormalised weights (1.0 for the softmax router) */
+    int32_t wkind;               /* MOE_W_* */
+    int32_t out_bf16;            /* 0: moe_forward writes fp32 [T][d]; 1: bf16 [T][d] */
+} moe_config;
+
+/*
+ * Expert weights, all device pointers, all borrowed: the caller keeps them alive and
+ * unchanged for the life of the layer.  Row-major throughout; one expert's data are
+ * contiguous.  The fused gate/up matrix holds the f gate rows first, then the f up rows (the
+ * split-at-the-row-boundary convention of the open-1b-verify page, "Tensor mapping").
+ *
+ *   int4 (MOE_W_INT4_ROWSCALE): the output of moe_pack_int4 --
+ *     gate_up        [E][2f][d/2] bytes     gate_up_scale [E][2f] fp32
+ *     down           [E][d][f/2]  bytes     down_scale    [E][d]  fp32
+ *   bf16 (MOE_W_BF16): gate_up [E][2f][d], down [E][d][f]; the scale pointers are ignored.
+ *   shared_*: the same for the single shared expert (with f_shared in place of f), or NULL
+ *   when n_shared == 0.
+ *   router_w [E][d] fp32; router_bias [E] fp32 for the sigmoid router (NULL means zeros).
+ * Every pointer must be 16-byte aligned.
+ */
+typedef struct {
+    const float *router_w;
+    const float *router_bias;
+    const void *gate_up;
+    const float *gate_up_scale;
+    const void *down;
+    const float *down_scale;
+    const void *shared_gate_up;
+    const float *shared_gate_up_scale;
+    const void *shared_down;
+    const float *shared_down_scale;
+} moe_weights;
+
+/*
+ * moe_pack_int4 -- quantise an fp32 matrix to the packed int4 container (colibri README,
+ * "What's implemented": packed int4 with per-row scales, validated bit-identical to the int8
+ * container).  For each row: scale = fp32(max|w| / 7); q = clamp(round-half-even(fp32(w /
+ * scale)), -8, 7); a row of zeros has scale 0 and codes 0.  Byte j of a row holds column 2j in
+ * its low nibble and column 2j+1 in its high nibble, each a 4-bit two's-complement code.
+ *
+ *   w       device, [rows][cols] fp32
+ *   packed  device, [rows][cols/2] bytes (written)
+ *   scales  device, [rows] fp32 (written)
+ *   rows >= 0; cols even and > 0.
+ * Synchronous: waits for `stream`, because it reports non-finite input (MOE_ERR_RANGE; such
+ * elements are written as code 0) -- it is a set-up call, not part of the forward pass.
+ */
+moe_status moe_pack_int4(const float *w, int64_t rows, int64_t cols, uint8_t *packed, float *scales,
+                         moe_stream stream);
+
+/*
+ * moe_layer_create -- validate the configuration, borrow the weights, and allocate the
+ * workspace for cfg->max_tokens tokens on the current CUDA device.  *out is set only on
+ * success.  Errors: MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_OOM, MOE_ERR_CUDA.
+ */
+moe_status moe_layer_create(const moe_config *cfg, const moe_weights *w, moe_layer **out);
+
+/*
+ * moe_route -- router and top-k only (step 1 above).
+ *   x    device, [T][d] bf16
+ *   idx  device, [T][k] int32 (written): chosen experts in rank order
+ *   w    device, [T][k] fp32 (written): their gate weights (computed in fp64, rounded once)
+ *   0 <= T <= max_tokens.  Asynchronous.  The logits are accumulated in fp64.
+ */
+moe_status moe_route(moe_layer *layer, const uint16_t *x, int32_t T, int32_t *idx, float *w,
+                     moe_stream stream);
+
+/*
+ * moe_forward -- the whole layer, steps 1 to 4.
+ *   x    device, [T][d] bf16
+ *   out  device, [T][d] fp32, or bf16 when cfg->out_bf16 (written)
+ *   0 <= T <= max_tokens.  Asynchronous and host-sync free (it can be captured in a CUDA
+ *   graph).  Calls on one layer must not overlap on the device (they share its workspace).
+ */
+moe_status moe_forward(moe_layer *layer, const uint16_t *x, int32_t T, void *out, moe_stream stream);
+
+/*
+ * moe_forward_host -- moe_forward on host buffers: copies x host->device, runs the layer,
+ * copies out device->host, and waits for `stream`.  x_host [T][d] bf16; out_host [T][d] fp32
+ * or bf16.  Synchronous.  Uses a staging area inside the workspace; pinned host buffers make
+ * the copies asynchronous with respect to other streams.
+ */
+moe_status moe_forward_host(moe_layer *layer, const uint16_t *x_host, int32_t T, void *out_host,
+                            moe_stream stream);
+
+/*
+ * moe_last_error -- wait for the layer's most recent stream, then return (and clear) the
+ * device status word: MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_RANGE; MOE_ERR_CUDA if the wait
+ * itself failed.  Synchronous.
+ */
+moe_status moe_last_error(moe_layer *layer);
+
+/* moe_layer_destroy -- free the workspace (after waiting for the layer's last stream).  NULL is
+ * ignored.  The borrowed weights are not touched. */
+void moe_layer_destroy(moe_layer *layer);
+
+/* Bytes of device workspace the layer holds. */
+int64_t moe_layer_workspace_bytes(const moe_layer *layer);
+
+/* Number of kernel launches the most recent moe_forward / moe_route enqueued (host bookkeeping). */
+int32_t moe_layer_last_launches(const moe_layer *layer);
+
+/* Static text for a status code. */
+const char *moe_status_str(moe_status status);
+
+/*
+ * Per-kernel timing.  While enabled, every kernel launch of the layer is bracketed by a pair of
+ * CUDA events recorded on the launching stream; moe_profile_read waits for the layer's last
+ * stream and returns (and resets) the summed device time and the launch count of one kernel.
+ * Off by default; turning it on adds two event records per launch.
+ */
+enum {
+    MOE_KERNEL_ROUTER_LOGITS = 0,   /* router GEMV, fp64 accumulation */
+    MOE_KERNEL_TOPK = 1,            /* top-k selection and gate weights */
+    MOE_KERNEL_BUCKET = 2,          /* histogram, scan, scatter, unique list */
+    MOE_KERNEL_GATEUP = 3,          /* decode: gate/up rows + SiLU */
+    MOE_KERNEL_DOWN = 4,            /* decode: down rows */
+    MOE_KERNEL_COMBINE = 5,         /* weighted combine with the shared expert */
+    MOE_KERNEL_GATHER = 6,          /* prefill: x rows gathered per expert */
+    MOE_KERNEL_GEMM_GATEUP = 7,     /* prefill: tcgen05 grouped GEMM gate/up + SiLU */
+    MOE_KERNEL_GEMM_DOWN = 8,       /* prefill: tcgen05 grouped GEMM down */
+    MOE_KERNEL_COUNT = 9
+};
+moe_status moe_profile_enable(moe_layer *layer, int32_t on);
+moe_status moe_profile_read(moe_layer *layer, int32_t kernel, double *total_ms, int64_t *launches);
+const char *moe_kernel_name(int32_t kernel);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QEFFN_MOE_H */

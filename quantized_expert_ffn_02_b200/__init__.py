@@ -1,0 +1,223 @@
+"""Thin Python binding of libmoe.so (the routed MoE FFN layer for B200).
+
+Argument marshalling only: every step of the layer runs in the CUDA library.  Functions
+carry the C ABI's names (``include/moe.h``); tensors are torch CUDA tensors (device memory
+and streams come from PyTorch), passed to the library as raw pointers.  If the shared
+library is missing the import fails: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_CUDA, MOE_ERR_OOM, MOE_ERR_TIMEOUT, MOE_ERR_RANGE, MOE_ERR_UNSUPPORTED = range(7)
+MOE_ROUTER_SOFTMAX_TOPK, MOE_ROUTER_SIGMOID_BIAS = 0, 1
+MOE_W_INT4_ROWSCALE, MOE_W_BF16 = 0, 1
+
+# Every symbol that include/moe.h declares.
+EXPORTS = (
+    "moe_pack_int4", "moe_layer_create", "moe_route", "moe_forward", "moe_forward_host", "moe_last_error",
+    "moe_layer_destroy", "moe_layer_workspace_bytes", "moe_layer_last_launches", "moe_status_str",
+    "moe_profile_enable", "moe_profile_read", "moe_kernel_name",
+)
+KERNELS = ("router_logits", "topk", "bucket", "gateup", "down", "combine", "gather", "gemm_gateup", "gemm_down")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_str(status)} ({status})")
+
+
+class moe_config(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("f", ctypes.c_int32), ("n_experts", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("n_shared", ctypes.c_int32), ("f_shared", ctypes.c_int32),
+                ("max_tokens", ctypes.c_int32), ("router", ctypes.c_int32),
+                ("routed_scaling_factor", ctypes.c_float), ("wkind", ctypes.c_int32), ("out_bf16", ctypes.c_int32)]
+
+
+class moe_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "router_w", "router_bias", "gate_up", "gate_up_scale", "down", "down_scale",
+        "shared_gate_up", "shared_gate_up_scale", "shared_down", "shared_down_scale")]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libmoe.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is missing: build it with `python -m quantized_expert_ffn_02_b200.build`")
+        L = ctypes.CDLL(path)
+        P, I32, I64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+        L.moe_pack_int4.argtypes = [P, I64, I64, P, P, P]
+        L.moe_layer_create.argtypes = [ctypes.POINTER(moe_config), ctypes.POINTER(moe_weights), ctypes.POINTER(P)]
+        L.moe_route.argtypes = [P, P, I32, P, P, P]
+        L.moe_forward.argtypes = [P, P, I32, P, P]
+        L.moe_forward_host.argtypes = [P, P, I32, P, P]
+        L.moe_last_error.argtypes = [P]
+        L.moe_layer_destroy.argtypes = [P]
+        L.moe_layer_destroy.restype = None
+        L.moe_layer_workspace_bytes.argtypes = [P]
+        L.moe_layer_workspace_bytes.restype = I64
+        L.moe_layer_last_launches.argtypes = [P]
+        L.moe_layer_last_launches.restype = I32
+        L.moe_status_str.argtypes = [ctypes.c_int]
+        L.moe_status_str.restype = ctypes.c_char_p
+        L.moe_profile_enable.argtypes = [P, I32]
+        L.moe_profile_read.argtypes = [P, I32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(I64)]
+        L.moe_kernel_name.argtypes = [I32]
+        L.moe_kernel_name.restype = ctypes.c_char_p
+        for n in ("moe_pack_int4", "moe_layer_create", "moe_route", "moe_forward", "moe_forward_host",
+                  "moe_last_error", "moe_profile_enable", "moe_profile_read"):
+            getattr(L, n).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_str(status: int) -> str:
+    return load().moe_status_str(int(status)).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != MOE_OK:
+        raise MoeError(rc, what)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+# ------------------------------------------------------------------------------------------
+# entry points (same names as the C ABI)
+# ------------------------------------------------------------------------------------------
+
+def moe_pack_int4(w, packed, scales, stream=None):
+    """w fp32 [rows][cols] (CUDA) -> packed uint8 [rows][cols/2], scales fp32 [rows] (written)."""
+    rows, cols = w.shape
+    _check(load().moe_pack_int4(_ptr(w), rows, cols, _ptr(packed), _ptr(scales), _stream(stream)),
+           "moe_pack_int4")
+
+
+def moe_layer_create(cfg: moe_config, weights: moe_weights) -> int:
+    h = ctypes.c_void_p()
+    _check(load().moe_layer_create(ctypes.byref(cfg), ctypes.byref(weights), ctypes.byref(h)), "moe_layer_create")
+    return h.value
+
+
+def moe_route(layer: int, x, T: int, idx, w, stream=None):
+    _check(load().moe_route(layer, _ptr(x), T, _ptr(idx), _ptr(w), _stream(stream)), "moe_route")
+
+
+def moe_forward(layer: int, x, T: int, out, stream=None):
+    _check(load().moe_forward(layer, _ptr(x), T, _ptr(out), _stream(stream)), "moe_forward")
+
+
+def moe_forward_host(layer: int, x_host, T: int, out_host, stream=None):
+    """x_host / out_host are CPU tensors (pinned for asynchronous copies)."""
+    _check(load().moe_forward_host(layer, _ptr(x_host), T, _ptr(out_host), _stream(stream)), "moe_forward_host")
+
+
+def moe_last_error(layer: int) -> int:
+    return int(load().moe_last_error(layer))
+
+
+def moe_layer_destroy(layer: int):
+    load().moe_layer_destroy(layer)
+
+
+def moe_layer_workspace_bytes(layer: int) -> int:
+    return int(load().moe_layer_workspace_bytes(layer))
+
+
+def moe_layer_last_launches(layer: int) -> int:
+    return int(load().moe_layer_last_launches(layer))
+
+
+def moe_profile_enable(layer: int, on: bool):
+    _check(load().moe_profile_enable(layer, 1 if on else 0), "moe_profile_enable")
+
+
+def moe_profile_read(layer: int, kernel: int):
+    """(summed device milliseconds, launches) of one kernel since the last read; resets them."""
+    ms, n = ctypes.c_double(), ctypes.c_int64()
+    _check(load().moe_profile_read(layer, kernel, ctypes.byref(ms), ctypes.byref(n)), "moe_profile_read")
+    return ms.value, n.value
+
+
+def moe_kernel_name(kernel: int) -> str:
+    return load().moe_kernel_name(kernel).decode()
+
+
+# ------------------------------------------------------------------------------------------
+# convenience owner of a layer handle
+# ------------------------------------------------------------------------------------------
+
+class MoELayer:
+    """Owns a moe_layer handle and keeps the borrowed weight tensors alive.
+
+    ``weights`` maps the moe_weights field names to CUDA tensors (or None)."""
+
+    def __init__(self, d, f, n_experts, top_k, max_tokens, router, wkind, weights: dict, n_shared=0, f_shared=0,
+                 routed_scaling_factor=1.0, out_bf16=False):
+        self.cfg = moe_config(d=d, f=f, n_experts=n_experts, top_k=top_k, n_shared=n_shared, f_shared=f_shared,
+                              max_tokens=max_tokens, router=router, routed_scaling_factor=routed_scaling_factor,
+                              wkind=wkind, out_bf16=1 if out_bf16 else 0)
+        self._tensors = dict(weights)
+        self.w = moe_weights(**{k: _ptr(v) for k, v in weights.items()})
+        self.handle = moe_layer_create(self.cfg, self.w)
+
+    def route(self, x, idx, w, stream=None):
+        moe_route(self.handle, x, x.shape[0], idx, w, stream)
+
+    def forward(self, x, out, stream=None):
+        moe_forward(self.handle, x, x.shape[0], out, stream)
+
+    def forward_host(self, x_host, out_host, stream=None):
+        moe_forward_host(self.handle, x_host, x_host.shape[0], out_host, stream)
+
+    def last_error(self) -> int:
+        return moe_last_error(self.handle)
+
+    def workspace_bytes(self) -> int:
+        return moe_layer_workspace_bytes(self.handle)
+
+    def last_launches(self) -> int:
+        return moe_layer_last_launches(self.handle)
+
+    def profile(self, on: bool):
+        moe_profile_enable(self.handle, on)
+
+    def profile_read(self) -> dict:
+        """{kernel name: (ms, launches)} for the kernels that ran since the last read."""
+        out = {}
+        for kid, name in enumerate(KERNELS):
+            ms, n = moe_profile_read(self.handle, kid)
+            if n:
+                out[name] = (ms, n)
+        return out
+
+    def close(self):
+        if self.handle:
+            moe_layer_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,147 @@
+// internal.cuh -- device helpers and the launch interface shared by the kernels of libmoe.so.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace qe {
+
+constexpr int kWarp = 32;
+
+// ---------------------------------------------------------------------------------------
+// Status word: the first error a kernel meets is latched (later ones are dropped).
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ void latch_status(int* status, int code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+// ---------------------------------------------------------------------------------------
+// 16-bit lanes of a 32-bit register and mixed-precision FMA (f32 += bf16*bf16 / f16*f16).
+// The product of two 16-bit floats is exact in the fused operation; only the sum rounds.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ void halves(uint32_t v, unsigned short& lo, unsigned short& hi) {
+    asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(v));
+}
+__device__ __forceinline__ float fma_bf16(unsigned short a, unsigned short b, float c) {
+    float d;
+    asm("fma.rn.f32.bf16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float fma_f16(unsigned short a, unsigned short b, float c) {
+    float d;
+    asm("fma.rn.f32.f16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(c));
+    return d;
+}
+// (a & b) | (~b & ... ) -- the 3-input function  b ? (a ^ c) : c, one LOP3.
+// With b = 0x000F000F it keeps the low nibble of each 16-bit half, flips the bits where c
+// has a 1 inside that nibble, and copies c elsewhere.
+__device__ __forceinline__ uint32_t lop_sel_xor(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Streaming 16-byte load (read once: do not keep in L1).
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+// Read-only 16-byte load that may stay in L1 (activations reused by many warps).
+__device__ __forceinline__ uint4 ld_ro16(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(unsigned short b) {
+    return __uint_as_float(((uint32_t)b) << 16);
+}
+
+}  // namespace qe
+
+// ---------------------------------------------------------------------------------------
+// Launch interface (host functions defined next to their kernels).
+// ---------------------------------------------------------------------------------------
+namespace qe {
+
+struct Workspace {
+    double* logits;        // [maxT][E]
+    int32_t* idx;          // [maxT][k]   rank order
+    float* wts;            // [maxT][k]
+    int32_t* asc;          // [maxT][k]   ranks of a token's experts in ascending expert order
+    double* xsum;          // [maxT]      sum of x over the hidden dimension
+    int32_t* cnt;          // [E]
+    int32_t* off;          // [E + 1]
+    int32_t* perm;         // [maxT * k]  routed slot -> entry (t * k + rank)
+    int32_t* slot_of;      // [maxT * k]  entry -> routed slot
+    int32_t* ulist;        // [E]         unique chosen experts, ascending
+    int32_t* n_unique;     // [1]
+    uint16_t* h;           // [slots][fmax] fp16 bits: SwiGLU activations
+    float* Y;              // [slots][d]   per-slot expert outputs (before the gate weight)
+    int32_t* status;       // [1]
+};
+
+struct LayerDims {
+    int d, f, E, k, S, f_shared, router, wkind, out_bf16;
+    float scaling;
+};
+
+// Optional per-kernel event timing (defined in layer.cu).  `prof` may be null.
+struct Profiler;
+void prof_mark(Profiler* prof, int kernel, bool begin, cudaStream_t s);
+
+// What every launch function needs: the stream, the launch counter, the profiler.
+struct Launch {
+    cudaStream_t s;
+    int* launches;
+    Profiler* prof;
+};
+
+// Per-device, per-layer set-up (shared-memory opt-ins); called by moe_layer_create.
+cudaError_t prepare_router(const LayerDims& L);
+cudaError_t prepare_bucket(const LayerDims& L);
+cudaError_t prepare_decode(const LayerDims& L);
+
+cudaError_t launch_pack_int4(const float* w, int64_t rows, int64_t cols, uint8_t* packed, float* scales,
+                             int* status, cudaStream_t s);
+cudaError_t launch_router(const LayerDims& L, const float* router_w, const float* router_bias,
+                          const uint16_t* x, int T, double* logits, double* xsum, int32_t* idx, float* wts,
+                          int32_t* asc, const Launch& ctx);
+cudaError_t launch_bucket(const LayerDims& L, int T, const Workspace& ws, const Launch& ctx);
+cudaError_t launch_decode_experts(const LayerDims& L, const moe_weights& W, const uint16_t* x, int T,
+                                  const Workspace& ws, int num_sms, const Launch& ctx);
+cudaError_t launch_combine(const LayerDims& L, int T, const Workspace& ws, void* out, const Launch& ctx);
+
+// Launch bookkeeping shared by the launch functions: profiler marks and the launch count.
+#define QE_LAUNCH(ctx, kernel_id, ...)                       \
+    do {                                                     \
+        prof_mark((ctx).prof, (kernel_id), true, (ctx).s);   \
+        __VA_ARGS__;                                         \
+        cudaError_t qe_err_ = cudaGetLastError();            \
+        prof_mark((ctx).prof, (kernel_id), false, (ctx).s);  \
+        if (qe_err_ != cudaSuccess) return qe_err_;          \
+        ++*(ctx).launches;                                   \
+    } while (0)
+
+}  // namespace qe

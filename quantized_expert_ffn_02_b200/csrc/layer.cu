@@ -1,0 +1,334 @@
+// layer.cu -- the C ABI of libmoe.so: argument checks, workspace, launch sequencing, status.
+//
+// moe_forward enqueues (all on the caller's stream, no host synchronisation):
+//   router logits + top-k (K2) -> bucketing (K3) -> gate/up + SiLU (K4) -> down (K4)
+//   -> combine with the shared expert (K6)
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "internal.cuh"
+
+namespace qe {
+
+// Event pairs around launches, summed on demand.  Events are created lazily and reused.
+struct Profiler {
+    bool on = false;
+    struct Pair { cudaEvent_t a, b; int kernel; };
+    std::vector<Pair> pending;
+    std::vector<cudaEvent_t> pool;
+    cudaEvent_t open_ev = nullptr;
+    double total_ms[MOE_KERNEL_COUNT] = {};
+    int64_t count[MOE_KERNEL_COUNT] = {};
+
+    cudaEvent_t get() {
+        if (!pool.empty()) {
+            cudaEvent_t e = pool.back();
+            pool.pop_back();
+            return e;
+        }
+        cudaEvent_t e = nullptr;
+        cudaEventCreate(&e);
+        return e;
+    }
+    void collect() {
+        for (Pair& p : pending) {
+            float ms = 0.f;
+            if (cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) {
+                total_ms[p.kernel] += ms;
+                count[p.kernel] += 1;
+            }
+            pool.push_back(p.a);
+            pool.push_back(p.b);
+        }
+        pending.clear();
+    }
+    ~Profiler() {
+        for (Pair& p : pending) { cudaEventDestroy(p.a); cudaEventDestroy(p.b); }
+        for (cudaEvent_t e : pool) cudaEventDestroy(e);
+        if (open_ev) cudaEventDestroy(open_ev);
+    }
+};
+
+void prof_mark(Profiler* p, int kernel, bool begin, cudaStream_t s) {
+    if (!p || !p->on) return;
+    cudaEvent_t e = p->get();
+    if (!e) return;
+    cudaEventRecord(e, s);
+    if (begin) {
+        p->open_ev = e;
+    } else if (p->open_ev) {
+        p->pending.push_back(Profiler::Pair{p->open_ev, e, kernel});
+        p->open_ev = nullptr;
+    }
+}
+
+}  // namespace qe
+
+struct moe_layer {
+    moe_config cfg;
+    moe_weights w;
+    qe::LayerDims dims;
+    qe::Workspace ws;
+    int device;
+    int num_sms;
+    void* ws_base;
+    size_t ws_bytes;
+    uint16_t* x_stage;     // [maxT][d] staging for moe_forward_host
+    void* out_stage;       // [maxT][d] fp32 staging
+    cudaStream_t last_stream;
+    int last_launches;
+    qe::Profiler prof;
+};
+
+namespace {
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+moe_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return MOE_OK;
+    if (e == cudaErrorMemoryAllocation) return MOE_ERR_OOM;
+    return MOE_ERR_CUDA;
+}
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Carves the workspace out of one allocation.  With base == nullptr it only measures.
+size_t carve(const moe_config& c, char* base, qe::Workspace* ws, uint16_t** x_stage, void** out_stage) {
+    const size_t T = (size_t)c.max_tokens, E = (size_t)c.n_experts, k = (size_t)c.top_k;
+    const size_t S = c.n_shared > 0 ? 1 : 0;
+    const size_t fmax = S && c.f_shared > c.f ? (size_t)c.f_shared : (size_t)c.f;
+    const size_t slots = T * k + T * S;
+    size_t o = 0;
+    auto take = [&](size_t bytes) -> char* {
+        char* p = base ? base + o : nullptr;
+        o = round_up(o + bytes, 256);
+        return p;
+    };
+    qe::Workspace w{};
+    w.logits = (double*)take(sizeof(double) * T * E);
+    w.idx = (int32_t*)take(sizeof(int32_t) * T * k);
+    w.wts = (float*)take(sizeof(float) * T * k);
+    w.asc = (int32_t*)take(sizeof(int32_t) * T * k);
+    w.xsum = (double*)take(sizeof(double) * T);
+    w.cnt = (int32_t*)take(sizeof(int32_t) * E);
+    w.off = (int32_t*)take(sizeof(int32_t) * (E + 1));
+    w.perm = (int32_t*)take(sizeof(int32_t) * T * k);
+    w.slot_of = (int32_t*)take(sizeof(int32_t) * T * k);
+    w.ulist = (int32_t*)take(sizeof(int32_t) * E);
+    w.n_unique = (int32_t*)take(sizeof(int32_t));
+    w.h = (uint16_t*)take(sizeof(uint16_t) * slots * fmax);
+    w.Y = (float*)take(sizeof(float) * slots * (size_t)c.d);
+    w.status = (int32_t*)take(sizeof(int32_t));
+    uint16_t* xs = (uint16_t*)take(sizeof(uint16_t) * T * (size_t)c.d);
+    void* os = (void*)take(sizeof(float) * T * (size_t)c.d);
+    if (ws) *ws = w;
+    if (x_stage) *x_stage = xs;
+    if (out_stage) *out_stage = os;
+    return o;
+}
+
+moe_status check_config(const moe_config* c, const moe_weights* w) {
+    if (!c || !w) return MOE_ERR_INVALID_ARG;
+    if (c->d <= 0 || c->d % 64 || c->f <= 0 || c->f % 64) return MOE_ERR_INVALID_ARG;
+    if (c->n_experts < 1 || c->n_experts > 1024) return MOE_ERR_INVALID_ARG;
+    if (c->top_k < 1 || c->top_k > c->n_experts || c->top_k > 32) return MOE_ERR_INVALID_ARG;
+    if (c->n_shared < 0 || c->n_shared > 1) return MOE_ERR_INVALID_ARG;
+    if (c->n_shared && (c->f_shared <= 0 || c->f_shared % 64)) return MOE_ERR_INVALID_ARG;
+    if (c->max_tokens < 1) return MOE_ERR_INVALID_ARG;
+    if (c->router != MOE_ROUTER_SOFTMAX_TOPK && c->router != MOE_ROUTER_SIGMOID_BIAS) return MOE_ERR_INVALID_ARG;
+    if (c->wkind != MOE_W_INT4_ROWSCALE && c->wkind != MOE_W_BF16) return MOE_ERR_INVALID_ARG;
+    if (!(c->routed_scaling_factor == c->routed_scaling_factor)) return MOE_ERR_INVALID_ARG;
+    if (c->d > 14336) return MOE_ERR_UNSUPPORTED;     // router x tile must fit in shared memory
+    if ((size_t)c->max_tokens * (size_t)(c->top_k + 1) > (size_t)INT32_MAX / 2) return MOE_ERR_UNSUPPORTED;
+    const bool q = c->wkind == MOE_W_INT4_ROWSCALE;
+    if (!w->router_w || !w->gate_up || !w->down) return MOE_ERR_INVALID_ARG;
+    if (q && (!w->gate_up_scale || !w->down_scale)) return MOE_ERR_INVALID_ARG;
+    if (c->n_shared && (!w->shared_gate_up || !w->shared_down)) return MOE_ERR_INVALID_ARG;
+    if (c->n_shared && q && (!w->shared_gate_up_scale || !w->shared_down_scale)) return MOE_ERR_INVALID_ARG;
+    const void* ptrs[] = {w->router_w, w->router_bias, w->gate_up, w->gate_up_scale, w->down, w->down_scale,
+                          w->shared_gate_up, w->shared_gate_up_scale, w->shared_down, w->shared_down_scale};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_str(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_CUDA: return "CUDA runtime error";
+        case MOE_ERR_OOM: return "out of device memory";
+        case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+        case MOE_ERR_RANGE: return "value out of range";
+        case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    }
+    return "unknown status";
+}
+
+moe_status moe_pack_int4(const float* w, int64_t rows, int64_t cols, uint8_t* packed, float* scales,
+                         moe_stream stream) {
+    if (rows < 0 || cols <= 0 || (cols & 1)) return MOE_ERR_INVALID_ARG;
+    if (rows == 0) return MOE_OK;
+    if (!w || !packed || !scales) return MOE_ERR_INVALID_ARG;
+    if (((uintptr_t)w & 3) || ((uintptr_t)scales & 3)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    int* status = nullptr;
+    cudaError_t e = cudaMallocAsync((void**)&status, sizeof(int), s);
+    if (e != cudaSuccess) return from_cuda(e);
+    e = cudaMemsetAsync(status, 0, sizeof(int), s);
+    if (e == cudaSuccess) e = qe::launch_pack_int4(w, rows, cols, packed, scales, status, s);
+    int host_status = 0;
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&host_status, status, sizeof(int), cudaMemcpyDeviceToHost, s);
+    cudaError_t e2 = cudaFreeAsync(status, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = e2;
+    if (e != cudaSuccess) return from_cuda(e);
+    return host_status ? (moe_status)host_status : MOE_OK;
+}
+
+moe_status moe_layer_create(const moe_config* cfg, const moe_weights* w, moe_layer** out) {
+    if (!out) return MOE_ERR_INVALID_ARG;
+    moe_status st = check_config(cfg, w);
+    if (st != MOE_OK) return st;
+    moe_layer* L = new (std::nothrow) moe_layer();
+    if (!L) return MOE_ERR_OOM;
+    L->cfg = *cfg;
+    L->w = *w;
+    if (cfg->router != MOE_ROUTER_SIGMOID_BIAS) L->w.router_bias = nullptr;
+    L->dims = qe::LayerDims{cfg->d, cfg->f, cfg->n_experts, cfg->top_k, cfg->n_shared > 0 ? 1 : 0,
+                            cfg->n_shared > 0 ? cfg->f_shared : 0, cfg->router, cfg->wkind, cfg->out_bf16 ? 1 : 0,
+                            cfg->routed_scaling_factor};
+    cudaError_t e = cudaGetDevice(&L->device);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&L->num_sms, cudaDevAttrMultiProcessorCount, L->device);
+    if (e == cudaSuccess) e = qe::prepare_router(L->dims);
+    if (e == cudaSuccess) e = qe::prepare_bucket(L->dims);
+    if (e == cudaSuccess) e = qe::prepare_decode(L->dims);
+    if (e != cudaSuccess) {
+        delete L;
+        return e == cudaErrorInvalidValue ? MOE_ERR_UNSUPPORTED : from_cuda(e);
+    }
+    L->ws_bytes = carve(*cfg, nullptr, nullptr, nullptr, nullptr);
+    e = cudaMalloc(&L->ws_base, L->ws_bytes);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        delete L;
+        return MOE_ERR_OOM;
+    }
+    carve(*cfg, (char*)L->ws_base, &L->ws, &L->x_stage, &L->out_stage);
+    e = cudaMemset(L->ws_base, 0, L->ws_bytes);
+    if (e != cudaSuccess) {
+        cudaFree(L->ws_base);
+        delete L;
+        return from_cuda(e);
+    }
+    L->last_stream = nullptr;
+    *out = L;
+    return MOE_OK;
+}
+
+moe_status moe_route(moe_layer* L, const uint16_t* x, int32_t T, int32_t* idx, float* w, moe_stream stream) {
+    if (!L || T < 0 || T > L->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !idx || !w || !aligned16(x) || ((uintptr_t)idx & 3) || ((uintptr_t)w & 3)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    int launches = 0;
+    const qe::Launch ctx{s, &launches, &L->prof};
+    cudaError_t e = qe::launch_router(L->dims, L->w.router_w, L->w.router_bias, x, T, L->ws.logits, L->ws.xsum, idx, w,
+                                      nullptr, ctx);
+    L->last_stream = s;
+    L->last_launches = launches;
+    return from_cuda(e);
+}
+
+moe_status moe_forward(moe_layer* L, const uint16_t* x, int32_t T, void* out, moe_stream stream) {
+    if (!L || T < 0 || T > L->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !out || !aligned16(x) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    int launches = 0;
+    const qe::Launch ctx{s, &launches, &L->prof};
+    const qe::Workspace& ws = L->ws;
+    cudaError_t e = qe::launch_router(L->dims, L->w.router_w, L->w.router_bias, x, T, ws.logits, ws.xsum, ws.idx,
+                                      ws.wts, ws.asc, ctx);
+    if (e == cudaSuccess) e = qe::launch_bucket(L->dims, T, ws, ctx);
+    if (e == cudaSuccess) e = qe::launch_decode_experts(L->dims, L->w, x, T, ws, L->num_sms, ctx);
+    if (e == cudaSuccess) e = qe::launch_combine(L->dims, T, ws, out, ctx);
+    L->last_stream = s;
+    L->last_launches = launches;
+    return from_cuda(e);
+}
+
+moe_status moe_forward_host(moe_layer* L, const uint16_t* x_host, int32_t T, void* out_host, moe_stream stream) {
+    if (!L || T < 0 || T > L->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t xbytes = sizeof(uint16_t) * (size_t)T * L->cfg.d;
+    const size_t obytes = (L->cfg.out_bf16 ? 2 : 4) * (size_t)T * L->cfg.d;
+    cudaError_t e = cudaMemcpyAsync(L->x_stage, x_host, xbytes, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    moe_status st = moe_forward(L, L->x_stage, T, L->out_stage, stream);
+    if (st != MOE_OK) return st;
+    e = cudaMemcpyAsync(out_host, L->out_stage, obytes, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    return from_cuda(e);
+}
+
+moe_status moe_last_error(moe_layer* L) {
+    if (!L) return MOE_ERR_INVALID_ARG;
+    cudaError_t e = L->last_stream ? cudaStreamSynchronize(L->last_stream) : cudaDeviceSynchronize();
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    int st = 0;
+    e = cudaMemcpy(&st, L->ws.status, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (st != 0) {
+        e = cudaMemset(L->ws.status, 0, sizeof(int));
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    return (moe_status)st;
+}
+
+void moe_layer_destroy(moe_layer* L) {
+    if (!L) return;
+    if (L->last_stream) cudaStreamSynchronize(L->last_stream);
+    else cudaDeviceSynchronize();
+    cudaFree(L->ws_base);
+    delete L;
+}
+
+int64_t moe_layer_workspace_bytes(const moe_layer* L) { return L ? (int64_t)L->ws_bytes : 0; }
+
+int32_t moe_layer_last_launches(const moe_layer* L) { return L ? L->last_launches : 0; }
+
+moe_status moe_profile_enable(moe_layer* L, int32_t on) {
+    if (!L) return MOE_ERR_INVALID_ARG;
+    L->prof.on = on != 0;
+    return MOE_OK;
+}
+
+moe_status moe_profile_read(moe_layer* L, int32_t kernel, double* total_ms, int64_t* launches) {
+    if (!L || kernel < 0 || kernel >= MOE_KERNEL_COUNT || !total_ms || !launches) return MOE_ERR_INVALID_ARG;
+    cudaError_t e = L->last_stream ? cudaStreamSynchronize(L->last_stream) : cudaDeviceSynchronize();
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    L->prof.collect();
+    *total_ms = L->prof.total_ms[kernel];
+    *launches = L->prof.count[kernel];
+    L->prof.total_ms[kernel] = 0.0;
+    L->prof.count[kernel] = 0;
+    return MOE_OK;
+}
+
+const char* moe_kernel_name(int32_t kernel) {
+    static const char* names[MOE_KERNEL_COUNT] = {"router_logits", "topk", "bucket", "gateup", "down", "combine",
+                                                  "gather", "gemm_gateup", "gemm_down"};
+    return (kernel >= 0 && kernel < MOE_KERNEL_COUNT) ? names[kernel] : "unknown";
+}
+
+}  // extern "C"

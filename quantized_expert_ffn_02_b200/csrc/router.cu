@@ -1,0 +1,184 @@
+// router.cu -- K2: router logits (fp64 accumulation) and top-k selection.
+//
+// Softmax top-k (Glacial, "What works": the Granite MoE layer) and the DeepSeek-V3-style
+// sigmoid router with a selection-only bias and routed_scaling_factor (colibri README and
+// iliria page, "What's implemented": noaux_tc).  Logits are accumulated in fp64: every
+// product bf16 * fp32 is exact in fp64, so the only rounding is in the sums and the top-k
+// boundary is decided at fp64 resolution.  Equal keys go to the lower expert index.
+#include "internal.cuh"
+
+namespace qe {
+namespace {
+
+constexpr int kRouterWarps = 8;      // experts per block
+constexpr int kRouterTokens = 8;     // tokens per block (x tile in shared memory)
+
+// grid = (ceil(E / 8), ceil(T / 8)); one warp per expert row, 8 tokens per block.
+// The block's x tile [8][d] bf16 sits in dynamic shared memory.  Blocks with
+// blockIdx.x == 0 also write sum_i x[t][i] (fp64) for their tokens.
+__global__ void __launch_bounds__(kRouterWarps * kWarp)
+router_logits_kernel(const float* __restrict__ wr, const uint16_t* __restrict__ x, int T, int d, int E,
+                     double* __restrict__ logits, double* __restrict__ xsum) {
+    extern __shared__ __align__(16) uint16_t xs[];      // [kRouterTokens][d]
+    const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
+    const int t0 = blockIdx.y * kRouterTokens;
+    const int nt = min(kRouterTokens, T - t0);
+    // stage x (16-byte copies; d % 64 == 0 so rows are 16-byte multiples)
+    const int row16 = d / 8;
+    for (int i = threadIdx.x; i < nt * row16; i += blockDim.x) {
+        const int tt = i / row16, c = i % row16;
+        reinterpret_cast<uint4*>(xs + (size_t)tt * d)[c] =
+            ld_ro16(reinterpret_cast<const uint4*>(x + (size_t)(t0 + tt) * d) + c);
+    }
+    __syncthreads();
+    if (blockIdx.x == 0 && warp < nt) {
+        double acc = 0.0;
+        for (int i = lane; i < d; i += kWarp) acc += (double)bf16_bits_to_f32(xs[(size_t)warp * d + i]);
+        acc = warp_sum_d(acc);
+        if (lane == 0) xsum[t0 + warp] = acc;
+    }
+    const int e = blockIdx.x * kRouterWarps + warp;
+    if (e >= E) return;
+    double acc[kRouterTokens];
+#pragma unroll
+    for (int tt = 0; tt < kRouterTokens; ++tt) acc[tt] = 0.0;
+    const float4* wrow = reinterpret_cast<const float4*>(wr + (size_t)e * d);
+    for (int c = lane; c < d / 4; c += kWarp) {
+        const float4 wv = __ldg(wrow + c);
+#pragma unroll
+        for (int tt = 0; tt < kRouterTokens; ++tt) {
+            if (tt < nt) {
+                const uint2 xv = *reinterpret_cast<const uint2*>(xs + (size_t)tt * d + 4 * c);
+                acc[tt] = fma((double)__uint_as_float(xv.x << 16), (double)wv.x, acc[tt]);
+                acc[tt] = fma((double)__uint_as_float(xv.x & 0xffff0000u), (double)wv.y, acc[tt]);
+                acc[tt] = fma((double)__uint_as_float(xv.y << 16), (double)wv.z, acc[tt]);
+                acc[tt] = fma((double)__uint_as_float(xv.y & 0xffff0000u), (double)wv.w, acc[tt]);
+            }
+        }
+    }
+#pragma unroll
+    for (int tt = 0; tt < kRouterTokens; ++tt) {
+        if (tt < nt) {
+            const double v = warp_sum_d(acc[tt]);
+            if (lane == 0) logits[(size_t)(t0 + tt) * E + e] = v;
+        }
+    }
+}
+
+struct KeyIdx {
+    double key;
+    int idx;
+};
+__device__ __forceinline__ bool beats(double ka, int ia, double kb, int ib) {
+    return ka > kb || (ka == kb && ia < ib);
+}
+
+// One warp per token: keys, k rounds of warp arg-max, gate weights.
+// Writes idx[t][r] / w[t][r] in rank order and asc[t][p] = the rank whose expert is the
+// p-th smallest of the token's k experts.
+template <int MAXPER>
+__global__ void __launch_bounds__(256)
+topk_kernel(const double* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k, int router,
+            float scaling, int32_t* __restrict__ idx_out, float* __restrict__ w_out, int32_t* __restrict__ asc_out) {
+    const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
+    const int t = blockIdx.x * (blockDim.x / kWarp) + warp;
+    if (t >= T) return;
+    const double* lg = logits + (size_t)t * E;
+    double key[MAXPER];
+    uint32_t taken = 0;
+#pragma unroll
+    for (int m = 0; m < MAXPER; ++m) {
+        const int e = lane + kWarp * m;
+        double kv = -INFINITY;
+        if (e < E) {
+            const double l = lg[e];
+            if (router == MOE_ROUTER_SIGMOID_BIAS)
+                kv = 1.0 / (1.0 + exp(-l)) + (bias ? (double)bias[e] : 0.0);
+            else
+                kv = l;
+            if (isnan(kv)) kv = -INFINITY;     // keeps every pick a valid expert index
+        } else {
+            taken |= 1u << m;
+        }
+        key[m] = kv;
+    }
+    int my_e = -1;          // lane r < k ends up holding the rank-r expert
+    for (int r = 0; r < k; ++r) {
+        double bk = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int m = 0; m < MAXPER; ++m) {
+            const int e = lane + kWarp * m;
+            if (!(taken >> m & 1u) && beats(key[m], e, bk, bi)) { bk = key[m]; bi = e; }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const double ok = __shfl_xor_sync(0xffffffffu, bk, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (beats(ok, oi, bk, bi)) { bk = ok; bi = oi; }
+        }
+        if ((bi % kWarp) == lane) taken |= 1u << (bi / kWarp);
+        if (lane == r) my_e = bi;
+    }
+    // gate weights over the chosen k (fp64, rounded once to fp32)
+    const bool mine = lane < k;
+    const double l = mine ? lg[my_e] : 0.0;
+    double num, den;
+    if (router == MOE_ROUTER_SIGMOID_BIAS) {
+        num = mine ? 1.0 / (1.0 + exp(-l)) : 0.0;
+        den = warp_sum_d(num);
+    } else {
+        double m = mine ? l : -INFINITY;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+        num = mine ? exp(l - m) : 0.0;
+        den = warp_sum_d(num);
+    }
+    // position of this rank in ascending expert order
+    int pos = 0;
+    for (int r2 = 0; r2 < k; ++r2) {
+        const int e2 = __shfl_sync(0xffffffffu, my_e, r2);
+        if (mine && e2 < my_e) ++pos;
+    }
+    if (mine) {
+        idx_out[(size_t)t * k + lane] = my_e;
+        w_out[(size_t)t * k + lane] = (float)((double)scaling * num / den);
+        if (asc_out) asc_out[(size_t)t * k + pos] = lane;
+    }
+}
+
+}  // namespace
+
+// The opt-in is set to the whole 227 KB once per device, so that layers of different widths
+// can coexist; each launch still asks only for its own tile.
+cudaError_t prepare_router(const LayerDims& L) {
+    const size_t smem = (size_t)kRouterTokens * L.d * sizeof(uint16_t);
+    if (smem > 227 * 1024) return cudaErrorInvalidValue;
+    return cudaFuncSetAttribute(router_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+}
+
+cudaError_t launch_router(const LayerDims& L, const float* router_w, const float* router_bias,
+                          const uint16_t* x, int T, double* logits, double* xsum, int32_t* idx, float* wts,
+                          int32_t* asc, const Launch& ctx) {
+    if (T == 0) return cudaSuccess;
+    const cudaStream_t s = ctx.s;
+    const size_t smem = (size_t)kRouterTokens * L.d * sizeof(uint16_t);
+    dim3 grid((L.E + kRouterWarps - 1) / kRouterWarps, (T + kRouterTokens - 1) / kRouterTokens);
+    QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,
+              (router_logits_kernel<<<grid, kRouterWarps * kWarp, smem, s>>>(router_w, x, T, L.d, L.E, logits, xsum)));
+    const int tpb = 8;
+    const unsigned g = (unsigned)((T + tpb - 1) / tpb);
+    const float* bias = L.router == MOE_ROUTER_SIGMOID_BIAS ? router_bias : nullptr;
+    if (L.E <= 32)
+        QE_LAUNCH(ctx, MOE_KERNEL_TOPK, (topk_kernel<1><<<g, tpb * kWarp, 0, s>>>(logits, bias, T, L.E, L.k, L.router,
+                                                                                    L.scaling, idx, wts, asc)));
+    else if (L.E <= 256)
+        QE_LAUNCH(ctx, MOE_KERNEL_TOPK, (topk_kernel<8><<<g, tpb * kWarp, 0, s>>>(logits, bias, T, L.E, L.k, L.router,
+                                                                                    L.scaling, idx, wts, asc)));
+    else
+        QE_LAUNCH(ctx, MOE_KERNEL_TOPK, (topk_kernel<32><<<g, tpb * kWarp, 0, s>>>(logits, bias, T, L.E, L.k, L.router,
+                                                                                     L.scaling, idx, wts, asc)));
+    return cudaSuccess;
+}
+
+}  // namespace qe

@@ -37,7 +37,9 @@ host with numpy.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
+import os
 from typing import Dict, Optional
 
 import numpy as np
@@ -82,8 +84,34 @@ def uniform(seed: int, name: str, offset: int, n: int) -> np.ndarray:
     return ((z >> np.uint64(11)).astype(np.float64) + 0.5) * _TWO_M53
 
 
+_THREADS = max(1, min(16, os.cpu_count() or 1))
+_CHUNK = 1 << 21
+
+
 def normal(seed: int, name: str, offset: int, n: int) -> np.ndarray:
-    """Standard normals, elements ``[offset, offset + n)`` of stream ``name`` (float64)."""
+    """Standard normals, elements ``[offset, offset + n)`` of stream ``name`` (float64).
+
+    Large draws are split into even-aligned pieces drawn on a thread pool (numpy releases the
+    GIL); the generator is counter based, so the pieces are exactly the serial draw."""
+    if n > 2 * _CHUNK and _THREADS > 1:
+        out = np.empty(n, dtype=np.float64)
+        first = min(n, (_CHUNK - (offset % 2)))
+        bounds = [(0, first)]
+        while bounds[-1][1] < n:
+            a = bounds[-1][1]
+            bounds.append((a, min(n, a + _CHUNK)))
+
+        def work(ab):
+            a, b = ab
+            out[a:b] = _normal_serial(seed, name, offset + a, b - a)
+
+        with concurrent.futures.ThreadPoolExecutor(_THREADS) as ex:
+            list(ex.map(work, bounds))
+        return out
+    return _normal_serial(seed, name, offset, n)
+
+
+def _normal_serial(seed: int, name: str, offset: int, n: int) -> np.ndarray:
     if n == 0:
         return np.zeros(0, dtype=np.float64)
     j0 = offset // 2
