@@ -191,6 +191,29 @@ enum {
     MOE_KERNEL_GEMM_DOWN = 8,       /* prefill: tcgen05 grouped GEMM down */
     MOE_KERNEL_COUNT = 9
 };
+/*
+ * moe_route_noalloc -- the routing step of moe_route, for callers that must not allocate device
+ * memory and so cannot create a layer: code running while a CUDA graph is captured (an
+ * allocation call breaks the capture), engines that serve every device byte from their own
+ * preallocated arena, and real-time loops that allow no allocation after start-up.  The pages
+ * have no counterpart: this is a deployment convenience of this library.
+ *
+ *   cfg       only d, n_experts, top_k, router and routed_scaling_factor are read
+ *   router_w  device, [E][d] fp32;  router_bias  device, [E] fp32 or NULL (sigmoid router)
+ *   x         device, [T][d] bf16;  idx [T][k] int32 and w [T][k] fp32 are written (device)
+ * The only scratch is a fixed 1 MiB array inside libmoe.so's device image, present on every GPU
+ * that loads the library until the process exits.  A call needs T*E*8 (rounded up to 256) +
+ * T*8 bytes of it; a larger request returns MOE_ERR_UNSUPPORTED (E = 256 allows T <= 510).
+ * The first call on each device looks up that array's device address and sets the router
+ * kernel's shared-memory limit (neither allocates); make that first call before any stream
+ * capture.  Every call on a device shares the array and the array keeps the last call's
+ * contents (each call overwrites all it reads); calls that overlap on the GPU -- on different
+ * streams, or from different host threads -- race on it.  Asynchronous; no allocation, no
+ * synchronisation.
+ */
+moe_status moe_route_noalloc(const moe_config *cfg, const float *router_w, const float *router_bias,
+                             const uint16_t *x, int32_t T, int32_t *idx, float *w, moe_stream stream);
+
 moe_status moe_profile_enable(moe_layer *layer, int32_t on);
 moe_status moe_profile_read(moe_layer *layer, int32_t kernel, double *total_ms, int64_t *launches);
 const char *moe_kernel_name(int32_t kernel);

@@ -22,7 +22,7 @@ MOE_W_INT4_ROWSCALE, MOE_W_BF16 = 0, 1
 EXPORTS = (
     "moe_pack_int4", "moe_layer_create", "moe_route", "moe_forward", "moe_forward_host", "moe_last_error",
     "moe_layer_destroy", "moe_layer_workspace_bytes", "moe_layer_last_launches", "moe_status_str",
-    "moe_profile_enable", "moe_profile_read", "moe_kernel_name",
+    "moe_profile_enable", "moe_profile_read", "moe_kernel_name", "moe_route_noalloc",
 )
 KERNELS = ("router_logits", "topk", "bucket", "gateup", "down", "combine", "gather", "gemm_gateup", "gemm_down")
 
@@ -75,8 +75,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         L.moe_profile_read.argtypes = [P, I32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(I64)]
         L.moe_kernel_name.argtypes = [I32]
         L.moe_kernel_name.restype = ctypes.c_char_p
+        L.moe_route_noalloc.argtypes = [ctypes.POINTER(moe_config), P, P, P, I32, P, P, P]
         for n in ("moe_pack_int4", "moe_layer_create", "moe_route", "moe_forward", "moe_forward_host",
-                  "moe_last_error", "moe_profile_enable", "moe_profile_read"):
+                  "moe_last_error", "moe_profile_enable", "moe_profile_read", "moe_route_noalloc"):
             getattr(L, n).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -161,6 +162,12 @@ def moe_profile_read(layer: int, kernel: int):
 
 def moe_kernel_name(kernel: int) -> str:
     return load().moe_kernel_name(kernel).decode()
+
+
+def moe_route_noalloc(cfg: moe_config, router_w, router_bias, x, T: int, idx, w, stream=None):
+    """Routing without any device allocation (for callers that may not allocate; see moe.h)."""
+    _check(load().moe_route_noalloc(ctypes.byref(cfg), _ptr(router_w), _ptr(router_bias), _ptr(x), T, _ptr(idx),
+                                    _ptr(w), _stream(stream)), "moe_route_noalloc")
 
 
 # ------------------------------------------------------------------------------------------

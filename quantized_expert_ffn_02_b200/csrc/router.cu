@@ -182,3 +182,82 @@ cudaError_t launch_router(const LayerDims& L, const float* router_w, const float
 }
 
 }  // namespace qe
+
+// ---------------------------------------------------------------------------------------
+// Routing for callers that cannot allocate device memory.
+//
+// Some callers of this library may not allocate on the device at all: code that runs while a
+// CUDA graph is being captured (where an allocation call breaks the capture), engines that
+// hand out every byte of device memory from their own preallocated arena, or real-time loops
+// that forbid an allocation (and its implicit synchronisation) after start-up.  They can still
+// route tokens with moe_route_noalloc: its only scratch (the fp64 logits and the per-token sum
+// of x) lives in a fixed array inside this library's device image, which every GPU that loads
+// the library holds until the process exits.
+// ---------------------------------------------------------------------------------------
+#include <mutex>
+
+namespace qe {
+namespace {
+
+constexpr size_t kRouteScratchBytes = (size_t)1 << 20;       // 1 MiB per device
+constexpr int kMaxDevices = 64;
+
+// The scratch itself.  In host code this name is only a stand-in for the device object:
+// kernels must be given the address that cudaGetSymbolAddress returns.
+static __device__ __align__(256) unsigned char g_route_scratch[kRouteScratchBytes];
+
+std::mutex g_route_scratch_mu;
+void* g_route_scratch_dev[kMaxDevices] = {};
+
+// Set-up, once per device, with that device current: look up the array's device address and
+// opt the router kernel into its shared memory.  Neither call allocates.
+moe_status route_scratch_for_current_device(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_route_scratch_mu);
+    if (!g_route_scratch_dev[dev]) {
+        void* p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
+        if (e != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+        e = cudaFuncSetAttribute(router_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        g_route_scratch_dev[dev] = p;
+    }
+    *out = g_route_scratch_dev[dev];
+    return MOE_OK;
+}
+
+}  // namespace
+}  // namespace qe
+
+extern "C" moe_status moe_route_noalloc(const moe_config* cfg, const float* router_w, const float* router_bias,
+                                        const uint16_t* x, int32_t T, int32_t* idx, float* w, moe_stream stream) {
+    if (!cfg || T < 0) return MOE_ERR_INVALID_ARG;
+    if (cfg->d <= 0 || cfg->d % 64 || cfg->d > 14336) return MOE_ERR_INVALID_ARG;
+    if (cfg->n_experts < 1 || cfg->n_experts > 1024) return MOE_ERR_INVALID_ARG;
+    if (cfg->top_k < 1 || cfg->top_k > cfg->n_experts || cfg->top_k > 32) return MOE_ERR_INVALID_ARG;
+    if (cfg->router != MOE_ROUTER_SOFTMAX_TOPK && cfg->router != MOE_ROUTER_SIGMOID_BIAS) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!router_w || !x || !idx || !w) return MOE_ERR_INVALID_ARG;
+    if (((uintptr_t)router_w & 15) || ((uintptr_t)x & 15) || ((uintptr_t)idx & 3) || ((uintptr_t)w & 3))
+        return MOE_ERR_INVALID_ARG;
+    // logits [T][E] fp64, then the sums of x [T] fp64, each part 256-byte aligned
+    const size_t logits_bytes = ((size_t)T * cfg->n_experts * sizeof(double) + 255) & ~(size_t)255;
+    const size_t need = logits_bytes + (size_t)T * sizeof(double);
+    if (need > qe::kRouteScratchBytes) return MOE_ERR_UNSUPPORTED;
+    void* scratch = nullptr;
+    moe_status st = qe::route_scratch_for_current_device(&scratch);
+    if (st != MOE_OK) return st;
+    // Every byte the kernels read from the scratch is written earlier in the same call, so
+    // nothing has to be cleared between calls.
+    double* logits = static_cast<double*>(scratch);
+    double* xsum = reinterpret_cast<double*>(static_cast<unsigned char*>(scratch) + logits_bytes);
+    const qe::LayerDims L{cfg->d, cfg->f, cfg->n_experts, cfg->top_k, 0, 0, cfg->router, cfg->wkind, 0,
+                          cfg->routed_scaling_factor};
+    int launches = 0;
+    const qe::Launch ctx{(cudaStream_t)stream, &launches, nullptr};
+    const float* bias = cfg->router == MOE_ROUTER_SIGMOID_BIAS ? router_bias : nullptr;
+    cudaError_t e = qe::launch_router(L, router_w, bias, x, T, logits, xsum, idx, w, nullptr, ctx);
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
