@@ -164,6 +164,20 @@ moe_status moe_last_error(moe_layer *layer);
  * ignored.  The borrowed weights are not touched. */
 void moe_layer_destroy(moe_layer *layer);
 
+/*
+ * Layer options.
+ *   MOE_OPT_PREFILL_MIN_TOKENS  batches with T >= value run the experts as tcgen05 grouped GEMMs
+ *                               (when the shape allows: int4 weights, d, f and f_shared multiples
+ *                               of 128); smaller batches use the HBM-streaming decode kernels.
+ *                               Default 128; value >= 1.  Both paths give the same results within
+ *                               the layer's tolerance.
+ *   MOE_OPT_PREFILL_AVAILABLE   (read only) 1 if this layer has the grouped-GEMM path.
+ * Setting an option is host-only and takes effect at the next moe_forward.
+ */
+enum { MOE_OPT_PREFILL_MIN_TOKENS = 0, MOE_OPT_PREFILL_AVAILABLE = 1 };
+moe_status moe_layer_set_option(moe_layer *layer, int32_t option, int64_t value);
+moe_status moe_layer_get_option(const moe_layer *layer, int32_t option, int64_t *value);
+
 /* Bytes of device workspace the layer holds. */
 int64_t moe_layer_workspace_bytes(const moe_layer *layer);
 

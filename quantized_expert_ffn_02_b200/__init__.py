@@ -23,7 +23,9 @@ EXPORTS = (
     "moe_pack_int4", "moe_layer_create", "moe_route", "moe_forward", "moe_forward_host", "moe_last_error",
     "moe_layer_destroy", "moe_layer_workspace_bytes", "moe_layer_last_launches", "moe_status_str",
     "moe_profile_enable", "moe_profile_read", "moe_kernel_name", "moe_route_noalloc",
+    "moe_layer_set_option", "moe_layer_get_option",
 )
+MOE_OPT_PREFILL_MIN_TOKENS, MOE_OPT_PREFILL_AVAILABLE = 0, 1
 KERNELS = ("router_logits", "topk", "bucket", "gateup", "down", "combine", "gather", "gemm_gateup", "gemm_down")
 
 
@@ -76,8 +78,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         L.moe_kernel_name.argtypes = [I32]
         L.moe_kernel_name.restype = ctypes.c_char_p
         L.moe_route_noalloc.argtypes = [ctypes.POINTER(moe_config), P, P, P, I32, P, P, P]
+        L.moe_layer_set_option.argtypes = [P, I32, I64]
+        L.moe_layer_get_option.argtypes = [P, I32, ctypes.POINTER(I64)]
         for n in ("moe_pack_int4", "moe_layer_create", "moe_route", "moe_forward", "moe_forward_host",
-                  "moe_last_error", "moe_profile_enable", "moe_profile_read", "moe_route_noalloc"):
+                  "moe_last_error", "moe_profile_enable", "moe_profile_read", "moe_route_noalloc",
+                  "moe_layer_set_option", "moe_layer_get_option"):
             getattr(L, n).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -164,6 +169,16 @@ def moe_kernel_name(kernel: int) -> str:
     return load().moe_kernel_name(kernel).decode()
 
 
+def moe_layer_set_option(layer: int, option: int, value: int):
+    _check(load().moe_layer_set_option(layer, option, int(value)), "moe_layer_set_option")
+
+
+def moe_layer_get_option(layer: int, option: int) -> int:
+    v = ctypes.c_int64()
+    _check(load().moe_layer_get_option(layer, option, ctypes.byref(v)), "moe_layer_get_option")
+    return v.value
+
+
 def moe_route_noalloc(cfg: moe_config, router_w, router_bias, x, T: int, idx, w, stream=None):
     """Routing without any device allocation (for callers that may not allocate; see moe.h)."""
     _check(load().moe_route_noalloc(ctypes.byref(cfg), _ptr(router_w), _ptr(router_bias), _ptr(x), T, _ptr(idx),
@@ -205,6 +220,13 @@ class MoELayer:
 
     def last_launches(self) -> int:
         return moe_layer_last_launches(self.handle)
+
+    def set_prefill_min_tokens(self, n: int):
+        moe_layer_set_option(self.handle, MOE_OPT_PREFILL_MIN_TOKENS, n)
+
+    @property
+    def has_gemm_path(self) -> bool:
+        return moe_layer_get_option(self.handle, MOE_OPT_PREFILL_AVAILABLE) == 1
 
     def profile(self, on: bool):
         moe_profile_enable(self.handle, on)

@@ -100,6 +100,10 @@ struct Workspace {
     uint16_t* h;           // [slots][fmax] fp16 bits: SwiGLU activations
     float* Y;              // [slots][d]   per-slot expert outputs (before the gate weight)
     int32_t* status;       // [1]
+    // grouped-GEMM (prefill) path
+    uint16_t* xg;          // [slots][d] bf16: x gathered per slot, K order permuted in groups of 8
+    int32_t* groups;       // [max_groups][4]: (expert or -1, first slot, tokens, unused)
+    int32_t* n_groups;     // [2]: routed groups, shared groups
 };
 
 struct LayerDims {
@@ -132,6 +136,16 @@ cudaError_t launch_bucket(const LayerDims& L, int T, const Workspace& ws, const 
 cudaError_t launch_decode_experts(const LayerDims& L, const moe_weights& W, const uint16_t* x, int T,
                                   const Workspace& ws, int num_sms, const Launch& ctx);
 cudaError_t launch_combine(const LayerDims& L, int T, const Workspace& ws, void* out, const Launch& ctx);
+
+// Grouped-GEMM path (prefill.cu).  A plan holds the layer's TMA tensor maps.
+struct PrefillPlan;
+bool prefill_supported(const LayerDims& L);
+size_t prefill_max_groups(const LayerDims& L, int max_tokens);
+cudaError_t prepare_prefill(const LayerDims& L);
+PrefillPlan* prefill_plan_create(const LayerDims& L, const moe_weights& W, const Workspace& ws, int max_tokens);
+void prefill_plan_destroy(PrefillPlan* p);
+cudaError_t launch_prefill_experts(const LayerDims& L, const PrefillPlan* p, const moe_weights& W, const uint16_t* x,
+                                   int T, const Workspace& ws, int num_sms, const Launch& ctx);
 
 // Launch bookkeeping shared by the launch functions: profiler marks and the launch count.
 #define QE_LAUNCH(ctx, kernel_id, ...)                       \

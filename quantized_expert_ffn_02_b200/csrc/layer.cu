@@ -81,6 +81,8 @@ struct moe_layer {
     cudaStream_t last_stream;
     int last_launches;
     qe::Profiler prof;
+    qe::PrefillPlan* plan = nullptr;     // TMA maps of the grouped-GEMM path (null if unsupported)
+    int64_t prefill_min_tokens = 128;    // batches at least this large take the grouped-GEMM path
 };
 
 namespace {
@@ -96,7 +98,9 @@ moe_status from_cuda(cudaError_t e) {
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Carves the workspace out of one allocation.  With base == nullptr it only measures.
-size_t carve(const moe_config& c, char* base, qe::Workspace* ws, uint16_t** x_stage, void** out_stage) {
+// max_groups > 0 adds the grouped-GEMM path's buffers.
+size_t carve(const moe_config& c, size_t max_groups, char* base, qe::Workspace* ws, uint16_t** x_stage,
+             void** out_stage) {
     const size_t T = (size_t)c.max_tokens, E = (size_t)c.n_experts, k = (size_t)c.top_k;
     const size_t S = c.n_shared > 0 ? 1 : 0;
     const size_t fmax = S && c.f_shared > c.f ? (size_t)c.f_shared : (size_t)c.f;
@@ -122,6 +126,11 @@ size_t carve(const moe_config& c, char* base, qe::Workspace* ws, uint16_t** x_st
     w.h = (uint16_t*)take(sizeof(uint16_t) * slots * fmax);
     w.Y = (float*)take(sizeof(float) * slots * (size_t)c.d);
     w.status = (int32_t*)take(sizeof(int32_t));
+    if (max_groups) {
+        w.xg = (uint16_t*)take(sizeof(uint16_t) * slots * (size_t)c.d);
+        w.groups = (int32_t*)take(sizeof(int32_t) * 4 * max_groups);
+        w.n_groups = (int32_t*)take(sizeof(int32_t) * 2);
+    }
     uint16_t* xs = (uint16_t*)take(sizeof(uint16_t) * T * (size_t)c.d);
     void* os = (void*)take(sizeof(float) * T * (size_t)c.d);
     if (ws) *ws = w;
@@ -210,23 +219,34 @@ moe_status moe_layer_create(const moe_config* cfg, const moe_weights* w, moe_lay
     if (e == cudaSuccess) e = qe::prepare_router(L->dims);
     if (e == cudaSuccess) e = qe::prepare_bucket(L->dims);
     if (e == cudaSuccess) e = qe::prepare_decode(L->dims);
+    const bool gemm = qe::prefill_supported(L->dims);
+    if (e == cudaSuccess && gemm) e = qe::prepare_prefill(L->dims);
     if (e != cudaSuccess) {
         delete L;
         return e == cudaErrorInvalidValue ? MOE_ERR_UNSUPPORTED : from_cuda(e);
     }
-    L->ws_bytes = carve(*cfg, nullptr, nullptr, nullptr, nullptr);
+    const size_t max_groups = gemm ? qe::prefill_max_groups(L->dims, cfg->max_tokens) : 0;
+    L->ws_bytes = carve(*cfg, max_groups, nullptr, nullptr, nullptr, nullptr);
     e = cudaMalloc(&L->ws_base, L->ws_bytes);
     if (e != cudaSuccess) {
         cudaGetLastError();
         delete L;
         return MOE_ERR_OOM;
     }
-    carve(*cfg, (char*)L->ws_base, &L->ws, &L->x_stage, &L->out_stage);
+    carve(*cfg, max_groups, (char*)L->ws_base, &L->ws, &L->x_stage, &L->out_stage);
     e = cudaMemset(L->ws_base, 0, L->ws_bytes);
     if (e != cudaSuccess) {
         cudaFree(L->ws_base);
         delete L;
         return from_cuda(e);
+    }
+    if (gemm) {
+        L->plan = qe::prefill_plan_create(L->dims, L->w, L->ws, cfg->max_tokens);
+        if (!L->plan) {
+            cudaFree(L->ws_base);
+            delete L;
+            return MOE_ERR_CUDA;
+        }
     }
     L->last_stream = nullptr;
     *out = L;
@@ -258,7 +278,12 @@ moe_status moe_forward(moe_layer* L, const uint16_t* x, int32_t T, void* out, mo
     cudaError_t e = qe::launch_router(L->dims, L->w.router_w, L->w.router_bias, x, T, ws.logits, ws.xsum, ws.idx,
                                       ws.wts, ws.asc, ctx);
     if (e == cudaSuccess) e = qe::launch_bucket(L->dims, T, ws, ctx);
-    if (e == cudaSuccess) e = qe::launch_decode_experts(L->dims, L->w, x, T, ws, L->num_sms, ctx);
+    if (e == cudaSuccess) {
+        if (L->plan && T >= L->prefill_min_tokens)
+            e = qe::launch_prefill_experts(L->dims, L->plan, L->w, x, T, ws, L->num_sms, ctx);
+        else
+            e = qe::launch_decode_experts(L->dims, L->w, x, T, ws, L->num_sms, ctx);
+    }
     if (e == cudaSuccess) e = qe::launch_combine(L->dims, T, ws, out, ctx);
     L->last_stream = s;
     L->last_launches = launches;
@@ -300,7 +325,29 @@ void moe_layer_destroy(moe_layer* L) {
     if (L->last_stream) cudaStreamSynchronize(L->last_stream);
     else cudaDeviceSynchronize();
     cudaFree(L->ws_base);
+    qe::prefill_plan_destroy(L->plan);
     delete L;
+}
+
+moe_status moe_layer_set_option(moe_layer* L, int32_t option, int64_t value) {
+    if (!L) return MOE_ERR_INVALID_ARG;
+    switch (option) {
+        case MOE_OPT_PREFILL_MIN_TOKENS:
+            if (value < 1) return MOE_ERR_INVALID_ARG;
+            L->prefill_min_tokens = value;
+            return MOE_OK;
+        default:
+            return MOE_ERR_INVALID_ARG;
+    }
+}
+
+moe_status moe_layer_get_option(const moe_layer* L, int32_t option, int64_t* value) {
+    if (!L || !value) return MOE_ERR_INVALID_ARG;
+    switch (option) {
+        case MOE_OPT_PREFILL_MIN_TOKENS: *value = L->prefill_min_tokens; return MOE_OK;
+        case MOE_OPT_PREFILL_AVAILABLE: *value = L->plan ? 1 : 0; return MOE_OK;
+        default: return MOE_ERR_INVALID_ARG;
+    }
 }
 
 int64_t moe_layer_workspace_bytes(const moe_layer* L) { return L ? (int64_t)L->ws_bytes : 0; }
