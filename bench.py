@@ -63,6 +63,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override E (smaller device footprint for profiler captures; same per-token work)")
     a = ap.parse_args()
     if a.steps is None:
         a.steps = DEFAULT_STEPS[a.workload]
@@ -246,18 +248,24 @@ def time_oracle(cfg, name, seed, budget_s, min_calls=1, max_calls=None):
 # roofline helpers
 # ------------------------------------------------------------------------------------------
 
-def kernel_bytes(cfg, T, n_unique):
-    """Algorithmic HBM bytes per launch of the expert kernels for a batch with n_unique routed experts."""
+def kernel_work(cfg, T, n_unique):
+    """Algorithmic work per launch of the expert kernels for a batch with n_unique routed experts:
+    {kernel: ("hbm", bytes) | ("tensor", flops)}.  Bytes count the weight rows and scales read
+    once, the activations read and the intermediate written; flops count 2 per multiply-add of
+    the expert FFN (padding columns of a GEMM tile are not counted)."""
     S = 1 if cfg.n_shared else 0
     slots = T * cfg.k + T * S
     fmax = max(cfg.f, cfg.f_shared if S else 0)
     q = cfg.wkind == syn.W_INT4
     gu_rows = n_unique * 2 * cfg.f + S * 2 * cfg.f_shared
-    dn_rows = (n_unique + S) * cfg.d
     gu = gu_rows * ((cfg.d // 2 + 4) if q else cfg.d * 2) + T * cfg.d * 2 + slots * fmax * 2
     f_of = lambda ff: (ff // 2 + 4) if q else ff * 2  # noqa: E731
-    dn = n_unique * cfg.d * f_of(cfg.f) + S * cfg.d * f_of(cfg.f_shared) + slots * fmax * 2 + slots * cfg.d * 4
-    return {"gateup": gu, "down": dn}
+    dn_w = n_unique * cfg.d * f_of(cfg.f) + S * cfg.d * f_of(cfg.f_shared) + slots * fmax * 2
+    # the single-token kernel adds the slots itself and writes the output; the others write y per slot
+    dn = dn_w + (T * cfg.d * 4 if T == 1 else slots * cfg.d * 4)
+    mac = T * cfg.k * cfg.d * cfg.f + T * S * cfg.d * cfg.f_shared
+    return {"gateup": ("hbm", gu), "down": ("hbm", dn), "gemm_gateup": ("tensor", 4 * mac),
+            "gemm_down": ("tensor", 2 * mac)}
 
 
 def source_sha(paths):
@@ -326,9 +334,13 @@ def run_reference(a, rank, world):
 def run_ours(a, rank, world, local_rank):
     import torch
 
+    import dataclasses
+
     import quantized_expert_ffn_02_b200 as qe
 
     cfg = syn.CONFIGS[a.workload]
+    if a.experts:
+        cfg = dataclasses.replace(cfg, E=a.experts)
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     dist = None
@@ -425,13 +437,22 @@ def run_ours(a, rank, world, local_rank):
         ms, n = prof[dom]
         per_launch_ms = ms / n
         timed_uniq = [uniq[(a.warmup + i) % len(xs)] for i in range(a.steps)]
-        bytes_per = statistics.mean(kernel_bytes(cfg, T, u)[dom] for u in timed_uniq) if dom in ("gateup", "down") \
-            else None
-        if bytes_per:
-            achieved = bytes_per / (per_launch_ms / 1e3) / 1e9
-            roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                    "frac": achieved / hbm, "traffic": traffic_for(dom), "peak_kind": f"{peak_kind} (copy)",
-                    "algorithmic_bytes_per_launch": bytes_per, "ms_per_launch": per_launch_ms}
+        works = [kernel_work(cfg, T, u).get(dom) for u in timed_uniq]
+        if works[0] is not None:
+            kind = works[0][0]
+            amount = statistics.mean(w[1] for w in works)
+            if kind == "hbm":
+                achieved = amount / (per_launch_ms / 1e3) / 1e9
+                roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                        "frac": achieved / hbm, "traffic": traffic_for(dom),
+                        "peak_kind": f"{peak_kind} copy bandwidth",
+                        "algorithmic_bytes_per_launch": amount, "ms_per_launch": per_launch_ms}
+            else:
+                achieved = amount / (per_launch_ms / 1e3) / 1e12
+                roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": tf, "unit": "TFLOP/s",
+                        "frac": achieved / tf, "traffic": traffic_for(dom),
+                        "peak_kind": f"{peak_kind} bf16 dense (burst)",
+                        "algorithmic_flops_per_launch": amount, "ms_per_launch": per_launch_ms}
     step_bytes = statistics.mean(uniq[(a.warmup + i) % len(xs)] for i in range(a.steps)) * expert_bytes(cfg) + \
         (expert_bytes(cfg, cfg.f_shared) if cfg.n_shared else 0) + cfg.E * cfg.d * 4
     ms_per_step = total_ms / a.steps

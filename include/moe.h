@@ -174,9 +174,33 @@ void moe_layer_destroy(moe_layer *layer);
  *   MOE_OPT_PREFILL_AVAILABLE   (read only) 1 if this layer has the grouped-GEMM path.
  * Setting an option is host-only and takes effect at the next moe_forward.
  */
-enum { MOE_OPT_PREFILL_MIN_TOKENS = 0, MOE_OPT_PREFILL_AVAILABLE = 1 };
+/*   MOE_OPT_SINGLE_TOKEN_KERNELS 1 (default): a T = 1 batch uses the dedicated single-token
+ *                               kernels when the shape allows (int4, d and f multiples of 1024,
+ *                               f_shared == f, k + shared <= 10); 0: the general decode kernels.
+ */
+/*   MOE_OPT_PROGRAMMATIC_LAUNCH  1 (default): chained kernels of the single-token path start
+ *                               early with programmatic dependent launch and wait on the device
+ *                               for their inputs; 0: ordinary stream order.  Same results.
+ */
+enum { MOE_OPT_PREFILL_MIN_TOKENS = 0, MOE_OPT_PREFILL_AVAILABLE = 1, MOE_OPT_SINGLE_TOKEN_KERNELS = 2,
+       MOE_OPT_PROGRAMMATIC_LAUNCH = 3 };
 moe_status moe_layer_set_option(moe_layer *layer, int32_t option, int64_t value);
 moe_status moe_layer_get_option(const moe_layer *layer, int32_t option, int64_t *value);
+
+/*
+ * moe_layer_debug_read -- copy one intermediate of the most recent moe_forward to host memory
+ * (waits for the layer's last stream).  For tests and debugging; the contents depend on which
+ * kernels ran (see each item).  `bytes` is the size of `dst`; at most the item's size is copied.
+ *   MOE_DEBUG_H      h = silu(g) * u, fp16 [slots][fmax] (slot = routed slot, then T*k + t for the
+ *                    shared expert; K order of the grouped-GEMM path is permuted in groups of 8)
+ *   MOE_DEBUG_Y      y per slot, fp32 [slots][d] (not written by the single-token kernels)
+ *   MOE_DEBUG_IDX / MOE_DEBUG_W / MOE_DEBUG_ASC   int32 / fp32 / int32 [T][k]
+ *   MOE_DEBUG_ULIST  int32 [E] unique chosen experts, ascending;  MOE_DEBUG_CNT int32 [E]
+ *   MOE_DEBUG_XSUM   fp64 [T]
+ */
+enum { MOE_DEBUG_H = 0, MOE_DEBUG_Y = 1, MOE_DEBUG_IDX = 2, MOE_DEBUG_W = 3, MOE_DEBUG_ASC = 4,
+       MOE_DEBUG_ULIST = 5, MOE_DEBUG_CNT = 6, MOE_DEBUG_XSUM = 7 };
+moe_status moe_layer_debug_read(moe_layer *layer, int32_t item, void *dst, int64_t bytes);
 
 /* Bytes of device workspace the layer holds. */
 int64_t moe_layer_workspace_bytes(const moe_layer *layer);

@@ -23,9 +23,10 @@ EXPORTS = (
     "moe_pack_int4", "moe_layer_create", "moe_route", "moe_forward", "moe_forward_host", "moe_last_error",
     "moe_layer_destroy", "moe_layer_workspace_bytes", "moe_layer_last_launches", "moe_status_str",
     "moe_profile_enable", "moe_profile_read", "moe_kernel_name", "moe_route_noalloc",
-    "moe_layer_set_option", "moe_layer_get_option",
+    "moe_layer_set_option", "moe_layer_get_option", "moe_layer_debug_read",
 )
-MOE_OPT_PREFILL_MIN_TOKENS, MOE_OPT_PREFILL_AVAILABLE = 0, 1
+MOE_OPT_PREFILL_MIN_TOKENS, MOE_OPT_PREFILL_AVAILABLE, MOE_OPT_SINGLE_TOKEN_KERNELS, MOE_OPT_PROGRAMMATIC_LAUNCH = 0, 1, 2, 3
+DEBUG_ITEMS = {"h": 0, "y": 1, "idx": 2, "w": 3, "asc": 4, "ulist": 5, "cnt": 6, "xsum": 7}
 KERNELS = ("router_logits", "topk", "bucket", "gateup", "down", "combine", "gather", "gemm_gateup", "gemm_down")
 
 
@@ -80,9 +81,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         L.moe_route_noalloc.argtypes = [ctypes.POINTER(moe_config), P, P, P, I32, P, P, P]
         L.moe_layer_set_option.argtypes = [P, I32, I64]
         L.moe_layer_get_option.argtypes = [P, I32, ctypes.POINTER(I64)]
+        L.moe_layer_debug_read.argtypes = [P, I32, P, I64]
         for n in ("moe_pack_int4", "moe_layer_create", "moe_route", "moe_forward", "moe_forward_host",
                   "moe_last_error", "moe_profile_enable", "moe_profile_read", "moe_route_noalloc",
-                  "moe_layer_set_option", "moe_layer_get_option"):
+                  "moe_layer_set_option", "moe_layer_get_option", "moe_layer_debug_read"):
             getattr(L, n).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -179,6 +181,12 @@ def moe_layer_get_option(layer: int, option: int) -> int:
     return v.value
 
 
+def moe_layer_debug_read(layer: int, item: str, dst) -> None:
+    """Copy an intermediate of the last forward into the numpy array ``dst`` (see moe.h)."""
+    _check(load().moe_layer_debug_read(layer, DEBUG_ITEMS[item], dst.ctypes.data, dst.nbytes),
+           "moe_layer_debug_read")
+
+
 def moe_route_noalloc(cfg: moe_config, router_w, router_bias, x, T: int, idx, w, stream=None):
     """Routing without any device allocation (for callers that may not allocate; see moe.h)."""
     _check(load().moe_route_noalloc(ctypes.byref(cfg), _ptr(router_w), _ptr(router_bias), _ptr(x), T, _ptr(idx),
@@ -220,6 +228,12 @@ class MoELayer:
 
     def last_launches(self) -> int:
         return moe_layer_last_launches(self.handle)
+
+    def set_single_token_kernels(self, on: bool):
+        moe_layer_set_option(self.handle, MOE_OPT_SINGLE_TOKEN_KERNELS, 1 if on else 0)
+
+    def debug_read(self, item: str, dst):
+        moe_layer_debug_read(self.handle, item, dst)
 
     def set_prefill_min_tokens(self, n: int):
         moe_layer_set_option(self.handle, MOE_OPT_PREFILL_MIN_TOKENS, n)

@@ -387,7 +387,6 @@ cudaError_t launch_experts_t(const LayerDims& L, const moe_weights& W, const uin
 
 }  // namespace
 
-cudaError_t prepare_decode(const LayerDims&) { return cudaSuccess; }
 
 cudaError_t launch_decode_experts(const LayerDims& L, const moe_weights& W, const uint16_t* x, int T,
                                   const Workspace& ws, int num_sms, const Launch& ctx) {

@@ -1,0 +1,485 @@
+// decode1.cu -- K4/K6 for a single token (T = 1) with int4 experts: the decode step of the layer.
+//
+// One token touches k routed experts plus the shared one; every weight byte is read once, so
+// the step is bound by HBM.  Two kernels, chained with programmatic dependent launch (PDL):
+//
+//   gateup_t1   persistent, one CTA per SM.  Each lane keeps its share of the token's activations
+//               in registers for the whole kernel (d/32 values, pre-paired to match the nibble
+//               pairs).  Each warp streams its row pairs (a gate row and the matching up row) into
+//               its own ring of shared-memory stages with TMA bulk copies, so the bytes in flight
+//               do not cost registers; it reduces each pair with warp shuffles and writes h.  The
+//               shared expert's rows need no routing and come first: they run while the router
+//               kernel is still finishing, and `griddepcontrol.wait` is reached only before the
+//               first routed row is fetched.
+//   down_t1     one CTA per block of output rows, two warps per slot (routed experts in
+//               ascending index, then the shared expert).  A warp keeps its slot's h in registers
+//               and streams its rows through its own TMA ring; the weight copies start before
+//               `griddepcontrol.wait` (they do not depend on h).  The CTA then adds the slots in
+//               order with their gate weights (the combine), so y never goes through global memory.
+//
+// Dequantisation as in decode.cu: bf16 (136 + s) with the offset removed per row through the
+// sum of x (computed here in fp64 from the registers); fp16 s exactly for the down rows.
+//
+// Data written by a kernel that may still run while this one runs (the router's tables, h) are
+// read through L2 with ld.global.cg: the non-coherent path may return stale lines.
+//
+// Every wait on an mbarrier is bounded (about 2 s).  A warp that gives up latches
+// MOE_ERR_TIMEOUT, waits (bounded again) for the copies it issued, and skips its remaining work.
+#include "internal.cuh"
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+namespace qe {
+namespace {
+
+constexpr uint32_t kNib = 0x000F000Fu;
+constexpr uint32_t kBf16Magic = 0x43084308u;
+constexpr uint32_t kF16Magic = 0x64086408u;
+constexpr int kGuStages = 3;          // row pairs in flight per warp (gate/up)
+constexpr int kGuMaxWarps = 12;
+constexpr int kDnSlotWarps = 2;       // warps per slot (down)
+constexpr int kDnRows = 4;            // rows per stage (down)
+constexpr int kDnStages = 3;
+constexpr int kDnMaxSlots = 10;       // k + 1
+constexpr int kDnRowsMax = 64;        // output rows per CTA at most
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr size_t kSmemLimit = 227 * 1024;
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void bar_init(uint32_t bar, uint32_t n) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(n));
+}
+__device__ __forceinline__ void bar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool bar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t now_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Bounded wait (every lane of the warp calls it; the result is made uniform by the caller).
+__device__ bool bar_wait(uint32_t bar, uint32_t parity) {
+    if (bar_try(bar, parity)) return true;
+    const uint64_t t0 = now_ns();
+    while (!bar_try(bar, parity))
+        if (now_ns() - t0 > kWaitLimitNs) return false;
+    return true;
+}
+// Bulk copy global -> shared, completion counted on `bar`.  16-byte aligned, size % 16 == 0.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ uint4 lds16(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+
+// 8 bf16 of columns 8m..8m+7 -> four registers holding (col i, col i+4), i = 0..3
+__device__ __forceinline__ void pair_cols(const uint4 v, uint32_t* p) {
+    p[0] = __byte_perm(v.x, v.z, 0x5410);
+    p[1] = __byte_perm(v.x, v.z, 0x7632);
+    p[2] = __byte_perm(v.y, v.w, 0x5410);
+    p[3] = __byte_perm(v.y, v.w, 0x7632);
+}
+
+// acc += sum over the 8 codes of word w of (136 + s) * x (x pairs matching the nibble pairs)
+__device__ __forceinline__ float dot_word_bf16(uint32_t w, const uint32_t* xp, float acc) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t p = lop_sel_xor(w >> (4 * i), kNib, kBf16Magic);
+        unsigned short wl, wh, xl, xh;
+        halves(p, wl, wh);
+        halves(xp[i], xl, xh);
+        acc = fma_bf16(wl, xl, acc);
+        acc = fma_bf16(wh, xh, acc);
+    }
+    return acc;
+}
+
+// acc += sum over the 8 codes of word w of s * h (h pairs matching the nibble pairs)
+__device__ __forceinline__ float dot_word_f16(uint32_t w, const uint32_t* hp, float acc) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t p = hsub2_u32(lop_sel_xor(w >> (4 * i), kNib, kF16Magic), kF16Magic);
+        unsigned short wl, wh, hl, hh;
+        halves(p, wl, wh);
+        halves(hp[i], hl, hh);
+        acc = fma_f16(wl, hl, acc);
+        acc = fma_f16(wh, hh, acc);
+    }
+    return acc;
+}
+
+// ---------------------------------------------------------------------------------------
+// gate/up + SiLU, T = 1.  NCH = d / 1024 chunks of 32 columns per lane.
+// Row pairs: [0, f_sh) of the shared expert (slot k), then u * f + r of routed expert ulist[u]
+// (slot u: with one token the routed slots are the unique experts in ascending order).
+// Warp gw takes tasks gw, gw + nw, ... (nw warps in the grid).
+// ---------------------------------------------------------------------------------------
+struct GuTask {
+    const uint8_t* gate;     // gate row (the up row is fe rows further)
+    const float* sc;         // scale of the gate row (the up row's is fe further)
+    int r, fe, slot;
+};
+
+template <int NCH>
+__global__ void __launch_bounds__(kGuMaxWarps * kWarp, 1)
+gateup_t1_kernel(const uint8_t* __restrict__ gate_up, const float* __restrict__ gu_scale,
+                 const uint8_t* __restrict__ sh_gate_up, const float* __restrict__ sh_gu_scale,
+                 const uint16_t* __restrict__ x, int k, int d, int f, int f_sh, int S, const int32_t* ulist,
+                 uint16_t* __restrict__ h, int fmax, int* status) {
+    extern __shared__ __align__(128) uint8_t smem[];          // [warps][kGuStages][2 * rowbytes]
+    __shared__ __align__(8) uint64_t bars[kGuMaxWarps][kGuStages];
+    const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
+    const int nwarps_cta = blockDim.x / kWarp;
+    const int gw = blockIdx.x * nwarps_cta + warp;
+    const int nw = gridDim.x * nwarps_cta;
+    const uint32_t rowbytes = (uint32_t)d / 2;
+    const int n_shared_tasks = S ? f_sh : 0;
+    const int n_tasks = n_shared_tasks + k * f;
+    const int my_tasks = gw < n_tasks ? (n_tasks - gw + nw - 1) / nw : 0;
+    const uint32_t ring = saddr(smem) + (uint32_t)warp * kGuStages * 2 * rowbytes;
+    if (lane == 0) {
+        for (int s = 0; s < kGuStages; ++s) bar_init(saddr(&bars[warp][s]), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+
+    bool routed_ready = false;          // lane 0 only: the router kernel has finished
+    auto task = [&](int i) {
+        GuTask tk;
+        const int t = gw + i * nw;
+        if (t < n_shared_tasks) {
+            tk.gate = sh_gate_up + (size_t)t * rowbytes;
+            tk.sc = sh_gu_scale + t;
+            tk.r = t;
+            tk.fe = f_sh;
+            tk.slot = k;
+        } else {
+            if (!routed_ready) {
+                pdl_wait();
+                pdl_trigger();          // the down kernel may now read the routing
+                routed_ready = true;
+            }
+            const int t2 = t - n_shared_tasks;
+            const int u = t2 / f, r = t2 % f;
+            const int e = __ldcg(ulist + u);
+            tk.gate = gate_up + ((size_t)e * 2 * f + r) * rowbytes;
+            tk.sc = gu_scale + (size_t)e * 2 * f + r;
+            tk.r = r;
+            tk.fe = f;
+            tk.slot = u;
+        }
+        return tk;
+    };
+    // lane 0 issues task i into stage i % kGuStages
+    auto issue = [&](int i) {
+        const GuTask tk = task(i);
+        const uint32_t bar = saddr(&bars[warp][i % kGuStages]);
+        const uint32_t dst = ring + (uint32_t)(i % kGuStages) * 2 * rowbytes;
+        bar_expect_tx(bar, 2 * rowbytes);
+        bulk_g2s(dst, tk.gate, rowbytes, bar);
+        bulk_g2s(dst + rowbytes, tk.gate + (size_t)tk.fe * rowbytes, rowbytes, bar);
+    };
+    int issued = 0;
+    if (lane == 0)      // prologue: shared-expert rows only (they need no routing)
+        while (issued < my_tasks && issued < kGuStages && gw + issued * nw < n_shared_tasks) issue(issued++);
+
+    // the token's activations: lane owns chunks lane + 32 j
+    uint32_t xr[NCH][16];
+    double xs = 0.0;
+#pragma unroll
+    for (int j = 0; j < NCH; ++j) {
+        const int c = lane + kWarp * j;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const uint4 v = ld_ro16(x + (size_t)c * 32 + 8 * m);
+            pair_cols(v, &xr[j][4 * m]);
+            const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                xs += (double)__uint_as_float(ws[q] << 16) + (double)__uint_as_float(ws[q] & 0xffff0000u);
+        }
+    }
+    xs = warp_sum_d(xs);
+    const float off136 = 136.0f * (float)xs;
+
+    bool ok = true;
+    int i = 0;
+    for (; i < my_tasks; ++i) {
+        if (lane == 0 && issued == i) issue(issued++);         // a routed first task: fetch it now
+        const int s = i % kGuStages;
+        ok = bar_wait(saddr(&bars[warp][s]), (uint32_t)(i / kGuStages) & 1u);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        const uint32_t st = ring + (uint32_t)s * 2 * rowbytes;
+        float ag = 0.0f, au = 0.0f;
+#pragma unroll
+        for (int j = 0; j < NCH; ++j) {
+            const uint32_t off = (uint32_t)(lane + kWarp * j) * 16;
+            const uint4 G = lds16(st + off), U = lds16(st + rowbytes + off);
+            ag = dot_word_bf16(G.x, &xr[j][0], ag);
+            au = dot_word_bf16(U.x, &xr[j][0], au);
+            ag = dot_word_bf16(G.y, &xr[j][4], ag);
+            au = dot_word_bf16(U.y, &xr[j][4], au);
+            ag = dot_word_bf16(G.z, &xr[j][8], ag);
+            au = dot_word_bf16(U.z, &xr[j][8], au);
+            ag = dot_word_bf16(G.w, &xr[j][12], ag);
+            au = dot_word_bf16(U.w, &xr[j][12], au);
+        }
+        __syncwarp();                                          // stage s is free again
+        if (lane == 0)
+            while (issued < my_tasks && issued < i + 1 + kGuStages) issue(issued++);
+        ag = warp_sum(ag);
+        au = warp_sum(au);
+        if (lane == 0) {
+            const GuTask tk = task(i);
+            const float gv = __ldg(tk.sc) * (ag - off136);
+            const float uv = __ldg(tk.sc + tk.fe) * (au - off136);
+            const float hv = gv / (1.0f + expf(-gv)) * uv;
+            const __half hh = __float2half_rn(hv);
+            if (!isfinite(__half2float(hh)) && isfinite(hv)) latch_status(status, MOE_ERR_RANGE);
+            h[(size_t)tk.slot * fmax + tk.r] = __half_as_ushort(hh);
+        }
+    }
+    if (lane == 0) {
+        if (!ok) {
+            latch_status(status, MOE_ERR_TIMEOUT);
+            for (int j = i; j < issued; ++j)              // copies still in flight land before exit
+                bar_wait(saddr(&bars[warp][j % kGuStages]), (uint32_t)(j / kGuStages) & 1u);
+        }
+        if (!routed_ready) {
+            pdl_wait();
+            pdl_trigger();
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// down + combine, T = 1.  NCH = f / 1024 chunks of 32 K values per lane.
+// CTA: output rows [j0, j0 + nj); warp w: slot u = w / 2 (u < k routed expert ulist[u], u == k the
+// shared expert), half w % 2 of the CTA's rows, streamed kDnRows at a time.
+// ---------------------------------------------------------------------------------------
+template <int NCH>
+__global__ void __launch_bounds__(kDnMaxSlots * kDnSlotWarps * kWarp, 1)
+down_t1_kernel(const uint8_t* __restrict__ down, const float* __restrict__ dn_scale,
+               const uint8_t* __restrict__ sh_down, const float* __restrict__ sh_dn_scale, const uint16_t* h,
+               int fmax, int k, int d, int f, int S, const int32_t* ulist, const float* wts, const int32_t* asc,
+               void* __restrict__ out, int out_bf16, int rj, int* status) {
+    extern __shared__ __align__(128) uint8_t smem[];          // [warps][kDnStages][kDnRows * rowbytes]
+    __shared__ __align__(8) uint64_t bars[kDnMaxSlots * kDnSlotWarps][kDnStages];
+    __shared__ float ys[kDnMaxSlots][kDnRowsMax];
+    __shared__ float gate_w[kDnMaxSlots];
+    const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
+    const int u = warp / kDnSlotWarps, half = warp % kDnSlotWarps;
+    const int j0 = blockIdx.x * rj;
+    const int nj = max(0, min(rj, d - j0));
+    // this warp's rows: [r0, r1) of the CTA's block
+    const int per = (nj + kDnSlotWarps - 1) / kDnSlotWarps;
+    const int r0 = min(nj, half * per), r1 = min(nj, r0 + per);
+    const int nrows = r1 - r0;
+    const int nstages = (nrows + kDnRows - 1) / kDnRows;
+    const bool shared = u == k;
+    const uint32_t rowbytes = (uint32_t)f / 2;
+    const uint32_t stage_bytes = kDnRows * rowbytes;
+    const uint32_t ring = saddr(smem) + (uint32_t)warp * kDnStages * stage_bytes;
+    // routing is final when this grid starts (the gate/up kernel triggered after its own wait)
+    const int e = shared ? -1 : __ldcg(ulist + u);
+    const uint8_t* W = shared ? sh_down : down + (size_t)e * d * rowbytes;
+    const float* sc = shared ? sh_dn_scale : dn_scale + (size_t)e * d;
+    if (u < k && half == 0 && lane == 0) gate_w[u] = __ldcg(wts + __ldcg(asc + u));
+    if (lane == 0) {
+        for (int s = 0; s < kDnStages; ++s) bar_init(saddr(&bars[warp][s]), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    auto issue = [&](int g) {       // stage g: rows r0 + 4g .. (contiguous)
+        const int a = r0 + g * kDnRows, n = min(kDnRows, r1 - a);
+        const uint32_t bar = saddr(&bars[warp][g % kDnStages]);
+        bar_expect_tx(bar, (uint32_t)n * rowbytes);
+        bulk_g2s(ring + (uint32_t)(g % kDnStages) * stage_bytes, W + (size_t)(j0 + a) * rowbytes,
+                 (uint32_t)n * rowbytes, bar);
+    };
+    int issued = 0;
+    if (lane == 0)                  // the weights do not depend on h: start before the wait
+        while (issued < nstages && issued < kDnStages) issue(issued++);
+    pdl_wait();                     // h is complete
+    uint32_t hr[NCH][16];
+#pragma unroll
+    for (int j = 0; j < NCH; ++j) {
+        const int c = lane + kWarp * j;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) pair_cols(ld_cg16(h + (size_t)u * fmax + (size_t)c * 32 + 8 * m), &hr[j][4 * m]);
+    }
+    bool ok = true;
+    int g = 0;
+    for (; g < nstages; ++g) {
+        const int s = g % kDnStages;
+        ok = bar_wait(saddr(&bars[warp][s]), (uint32_t)(g / kDnStages) & 1u);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        const uint32_t st = ring + (uint32_t)s * stage_bytes;
+        const int a = r0 + g * kDnRows, n = min(kDnRows, r1 - a);
+        float acc[kDnRows];
+#pragma unroll
+        for (int q = 0; q < kDnRows; ++q) {
+            float v = 0.0f;
+            if (q < n) {
+#pragma unroll
+                for (int j = 0; j < NCH; ++j) {
+                    const uint4 wv = lds16(st + (uint32_t)q * rowbytes + (uint32_t)(lane + kWarp * j) * 16);
+                    v = dot_word_f16(wv.x, &hr[j][0], v);
+                    v = dot_word_f16(wv.y, &hr[j][4], v);
+                    v = dot_word_f16(wv.z, &hr[j][8], v);
+                    v = dot_word_f16(wv.w, &hr[j][12], v);
+                }
+            }
+            acc[q] = v;
+        }
+        __syncwarp();
+        if (lane == 0 && issued < nstages) issue(issued++);
+#pragma unroll
+        for (int q = 0; q < kDnRows; ++q) {
+            const float v = warp_sum(acc[q]);
+            if (lane == 0 && q < n) ys[u][a + q] = __ldg(sc + j0 + a + q) * v;
+        }
+    }
+    if (lane == 0 && !ok) {
+        latch_status(status, MOE_ERR_TIMEOUT);
+        for (int j = g; j < issued; ++j) bar_wait(saddr(&bars[warp][j % kDnStages]), (uint32_t)(j / kDnStages) & 1u);
+    }
+    __syncthreads();
+    // combine: routed slots in ascending expert order, then the shared expert
+    for (int i = threadIdx.x; i < nj; i += blockDim.x) {
+        float o = 0.0f;
+        for (int s = 0; s < k; ++s) o = fmaf(gate_w[s], ys[s][i], o);
+        if (S) o += ys[k][i];
+        if (out_bf16)
+            static_cast<__nv_bfloat16*>(out)[j0 + i] = __float2bfloat16_rn(o);
+        else
+            static_cast<float*>(out)[j0 + i] = o;
+    }
+}
+
+// Launch that may start while the previous kernel on the stream is still running (when
+// `programmatic`); the kernel itself waits (griddepcontrol.wait) before reading that kernel's
+// results.  Without the attribute the wait returns at once.
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(bool programmatic, Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = programmatic ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+int gu_warps(const LayerDims& L) {
+    const size_t per_warp = (size_t)kGuStages * L.d;     // kGuStages x (gate + up rows of d/2 bytes)
+    const int w = (int)((kSmemLimit - 4096) / per_warp);
+    return w > kGuMaxWarps ? kGuMaxWarps : w;
+}
+size_t dn_smem(const LayerDims& L) {
+    return (size_t)(L.k + L.S) * kDnSlotWarps * kDnStages * kDnRows * (L.f / 2);
+}
+
+}  // namespace
+
+bool decode_t1_supported(const LayerDims& L) {
+    return L.wkind == MOE_W_INT4_ROWSCALE && L.d % 1024 == 0 && L.d / 1024 <= 8 && L.f % 1024 == 0 &&
+           L.f / 1024 <= 4 && (!L.S || L.f_shared == L.f) && L.k + L.S <= kDnMaxSlots && gu_warps(L) >= 4 &&
+           dn_smem(L) <= kSmemLimit - 4096;  // 4 KB left for static shared memory
+}
+
+cudaError_t prepare_decode(const LayerDims& L) {
+    if (!decode_t1_supported(L)) return cudaSuccess;
+    // opt each kernel into all the dynamic shared memory its static part leaves free
+    cudaError_t e = cudaSuccess;
+    auto opt_in = [](const void* fn) {
+        cudaFuncAttributes fa;
+        cudaError_t r = cudaFuncGetAttributes(&fa, fn);
+        if (r != cudaSuccess) return r;
+        return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)(kSmemLimit - fa.sharedSizeBytes));
+    };
+#define QE_ATTR(KERN) \
+    if (e == cudaSuccess) e = opt_in((const void*)KERN);
+    QE_ATTR(gateup_t1_kernel<1>) QE_ATTR(gateup_t1_kernel<2>) QE_ATTR(gateup_t1_kernel<3>) QE_ATTR(gateup_t1_kernel<4>)
+    QE_ATTR(gateup_t1_kernel<5>) QE_ATTR(gateup_t1_kernel<6>) QE_ATTR(gateup_t1_kernel<7>) QE_ATTR(gateup_t1_kernel<8>)
+    QE_ATTR(down_t1_kernel<1>) QE_ATTR(down_t1_kernel<2>) QE_ATTR(down_t1_kernel<3>) QE_ATTR(down_t1_kernel<4>)
+#undef QE_ATTR
+    return e;
+}
+
+cudaError_t launch_decode_t1(const LayerDims& L, const moe_weights& W, const uint16_t* x, const Workspace& ws,
+                             void* out, int num_sms, const Launch& ctx) {
+    const int fmax = L.f;
+    const int nchx = L.d / 1024, nchf = L.f / 1024;
+    const int guw = gu_warps(L);
+    const size_t gu_smem = (size_t)guw * kGuStages * L.d;
+    cudaError_t e = cudaSuccess;
+    prof_mark(ctx.prof, MOE_KERNEL_GATEUP, true, ctx.s);
+#define QE_GU(N)                                                                                                      \
+    case N:                                                                                                           \
+        e = launch_pdl(L.pdl != 0, gateup_t1_kernel<N>, dim3(num_sms), dim3(guw * kWarp), gu_smem, ctx.s,              \
+                       (const uint8_t*)W.gate_up, W.gate_up_scale, (const uint8_t*)W.shared_gate_up,                  \
+                       W.shared_gate_up_scale, x, L.k, L.d, L.f, L.f_shared, L.S, (const int32_t*)ws.ulist, ws.h,     \
+                       fmax, ws.status);                                                                              \
+        break;
+    switch (nchx) {
+        QE_GU(1) QE_GU(2) QE_GU(3) QE_GU(4) QE_GU(5) QE_GU(6) QE_GU(7) QE_GU(8)
+        default: return cudaErrorInvalidValue;
+    }
+#undef QE_GU
+    prof_mark(ctx.prof, MOE_KERNEL_GATEUP, false, ctx.s);
+    if (e != cudaSuccess) return e;
+    ++*ctx.launches;
+    int rj = (L.d + num_sms - 1) / num_sms;
+    if (rj > kDnRowsMax) rj = kDnRowsMax;
+    const unsigned grid = (unsigned)((L.d + rj - 1) / rj);
+    const unsigned threads = (unsigned)(L.k + L.S) * kDnSlotWarps * kWarp;
+    const size_t dsm = dn_smem(L);
+    prof_mark(ctx.prof, MOE_KERNEL_DOWN, true, ctx.s);
+#define QE_DN(N)                                                                                                      \
+    case N:                                                                                                           \
+        e = launch_pdl(L.pdl != 0, down_t1_kernel<N>, dim3(grid), dim3(threads), dsm, ctx.s, (const uint8_t*)W.down,   \
+                       W.down_scale, (const uint8_t*)W.shared_down, W.shared_down_scale, (const uint16_t*)ws.h, fmax, \
+                       L.k, L.d, L.f, L.S, (const int32_t*)ws.ulist, (const float*)ws.wts, (const int32_t*)ws.asc,    \
+                       out, L.out_bf16, rj, ws.status);                                                              \
+        break;
+    switch (nchf) {
+        QE_DN(1) QE_DN(2) QE_DN(3) QE_DN(4)
+        default: return cudaErrorInvalidValue;
+    }
+#undef QE_DN
+    prof_mark(ctx.prof, MOE_KERNEL_DOWN, false, ctx.s);
+    if (e != cudaSuccess) return e;
+    ++*ctx.launches;
+    return cudaSuccess;
+}
+
+}  // namespace qe

@@ -55,7 +55,16 @@ __device__ __forceinline__ uint4 ld_stream16(const void* p) {
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
     return v;
 }
-// Read-only 16-byte load that may stay in L1 (activations reused by many warps).
+// Coherent 16-byte load through L2 only.  Required for data written by a kernel whose lifetime
+// overlaps the reader's (programmatic dependent launch): the .nc path may serve stale lines.
+__device__ __forceinline__ uint4 ld_cg16(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p) : "memory");
+    return v;
+}
+// Read-only 16-byte load that may stay in L1 (activations reused by many warps).  Only for data
+// that no kernel running at the same time can write.
 __device__ __forceinline__ uint4 ld_ro16(const void* p) {
     uint4 v;
     asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -104,11 +113,13 @@ struct Workspace {
     uint16_t* xg;          // [slots][d] bf16: x gathered per slot, K order permuted in groups of 8
     int32_t* groups;       // [max_groups][4]: (expert or -1, first slot, tokens, unused)
     int32_t* n_groups;     // [2]: routed groups, shared groups
+    uint32_t* counter;     // [1]: blocks done in the fused small-batch router (reset to 0 by the last)
 };
 
 struct LayerDims {
     int d, f, E, k, S, f_shared, router, wkind, out_bf16;
     float scaling;
+    int pdl = 1;           // chain dependent kernels with programmatic dependent launch
 };
 
 // Optional per-kernel event timing (defined in layer.cu).  `prof` may be null.
@@ -133,6 +144,14 @@ cudaError_t launch_router(const LayerDims& L, const float* router_w, const float
                           const uint16_t* x, int T, double* logits, double* xsum, int32_t* idx, float* wts,
                           int32_t* asc, const Launch& ctx);
 cudaError_t launch_bucket(const LayerDims& L, int T, const Workspace& ws, const Launch& ctx);
+// Small batches: logits, top-k, gate weights and bucket tables in one launch.
+constexpr int kRouteSmallMaxT = 32;
+cudaError_t launch_route_small(const LayerDims& L, const float* router_w, const float* router_bias, const uint16_t* x,
+                               int T, const Workspace& ws, const Launch& ctx);
+// One token, int4 experts: gate/up and down+combine kernels (decode1.cu).
+bool decode_t1_supported(const LayerDims& L);
+cudaError_t launch_decode_t1(const LayerDims& L, const moe_weights& W, const uint16_t* x, const Workspace& ws,
+                             void* out, int num_sms, const Launch& ctx);
 cudaError_t launch_decode_experts(const LayerDims& L, const moe_weights& W, const uint16_t* x, int T,
                                   const Workspace& ws, int num_sms, const Launch& ctx);
 cudaError_t launch_combine(const LayerDims& L, int T, const Workspace& ws, void* out, const Launch& ctx);

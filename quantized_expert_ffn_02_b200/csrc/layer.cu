@@ -83,6 +83,7 @@ struct moe_layer {
     qe::Profiler prof;
     qe::PrefillPlan* plan = nullptr;     // TMA maps of the grouped-GEMM path (null if unsupported)
     int64_t prefill_min_tokens = 128;    // batches at least this large take the grouped-GEMM path
+    bool t1_kernels = false;             // the dedicated single-token decode kernels apply
 };
 
 namespace {
@@ -126,6 +127,7 @@ size_t carve(const moe_config& c, size_t max_groups, char* base, qe::Workspace* 
     w.h = (uint16_t*)take(sizeof(uint16_t) * slots * fmax);
     w.Y = (float*)take(sizeof(float) * slots * (size_t)c.d);
     w.status = (int32_t*)take(sizeof(int32_t));
+    w.counter = (uint32_t*)take(sizeof(uint32_t));
     if (max_groups) {
         w.xg = (uint16_t*)take(sizeof(uint16_t) * slots * (size_t)c.d);
         w.groups = (int32_t*)take(sizeof(int32_t) * 4 * max_groups);
@@ -248,6 +250,7 @@ moe_status moe_layer_create(const moe_config* cfg, const moe_weights* w, moe_lay
             return MOE_ERR_CUDA;
         }
     }
+    L->t1_kernels = qe::decode_t1_supported(L->dims);
     L->last_stream = nullptr;
     *out = L;
     return MOE_OK;
@@ -275,16 +278,26 @@ moe_status moe_forward(moe_layer* L, const uint16_t* x, int32_t T, void* out, mo
     int launches = 0;
     const qe::Launch ctx{s, &launches, &L->prof};
     const qe::Workspace& ws = L->ws;
-    cudaError_t e = qe::launch_router(L->dims, L->w.router_w, L->w.router_bias, x, T, ws.logits, ws.xsum, ws.idx,
-                                      ws.wts, ws.asc, ctx);
-    if (e == cudaSuccess) e = qe::launch_bucket(L->dims, T, ws, ctx);
-    if (e == cudaSuccess) {
-        if (L->plan && T >= L->prefill_min_tokens)
-            e = qe::launch_prefill_experts(L->dims, L->plan, L->w, x, T, ws, L->num_sms, ctx);
-        else
-            e = qe::launch_decode_experts(L->dims, L->w, x, T, ws, L->num_sms, ctx);
+    const bool gemm = L->plan && T >= L->prefill_min_tokens;
+    cudaError_t e;
+    if (T <= qe::kRouteSmallMaxT) {
+        e = qe::launch_route_small(L->dims, L->w.router_w, L->w.router_bias, x, T, ws, ctx);
+    } else {
+        e = qe::launch_router(L->dims, L->w.router_w, L->w.router_bias, x, T, ws.logits, ws.xsum, ws.idx, ws.wts,
+                              ws.asc, ctx);
+        if (e == cudaSuccess) e = qe::launch_bucket(L->dims, T, ws, ctx);
     }
-    if (e == cudaSuccess) e = qe::launch_combine(L->dims, T, ws, out, ctx);
+    if (e == cudaSuccess) {
+        if (gemm) {
+            e = qe::launch_prefill_experts(L->dims, L->plan, L->w, x, T, ws, L->num_sms, ctx);
+            if (e == cudaSuccess) e = qe::launch_combine(L->dims, T, ws, out, ctx);
+        } else if (T == 1 && L->t1_kernels) {
+            e = qe::launch_decode_t1(L->dims, L->w, x, ws, out, L->num_sms, ctx);
+        } else {
+            e = qe::launch_decode_experts(L->dims, L->w, x, T, ws, L->num_sms, ctx);
+            if (e == cudaSuccess) e = qe::launch_combine(L->dims, T, ws, out, ctx);
+        }
+    }
     L->last_stream = s;
     L->last_launches = launches;
     return from_cuda(e);
@@ -336,9 +349,41 @@ moe_status moe_layer_set_option(moe_layer* L, int32_t option, int64_t value) {
             if (value < 1) return MOE_ERR_INVALID_ARG;
             L->prefill_min_tokens = value;
             return MOE_OK;
+        case MOE_OPT_SINGLE_TOKEN_KERNELS:
+            if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+            L->t1_kernels = value == 1 && qe::decode_t1_supported(L->dims);
+            return MOE_OK;
+        case MOE_OPT_PROGRAMMATIC_LAUNCH:
+            if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+            L->dims.pdl = (int)value;
+            return MOE_OK;
         default:
             return MOE_ERR_INVALID_ARG;
     }
+}
+
+moe_status moe_layer_debug_read(moe_layer* L, int32_t item, void* dst, int64_t bytes) {
+    if (!L || !dst || bytes < 0) return MOE_ERR_INVALID_ARG;
+    const size_t T = (size_t)L->cfg.max_tokens, k = (size_t)L->cfg.top_k, E = (size_t)L->cfg.n_experts;
+    const size_t slots = T * k + T * (size_t)L->dims.S;
+    const size_t fmax = L->dims.S && L->dims.f_shared > L->dims.f ? (size_t)L->dims.f_shared : (size_t)L->dims.f;
+    const void* src = nullptr;
+    size_t n = 0;
+    switch (item) {
+        case MOE_DEBUG_H: src = L->ws.h; n = 2 * slots * fmax; break;
+        case MOE_DEBUG_Y: src = L->ws.Y; n = 4 * slots * (size_t)L->cfg.d; break;
+        case MOE_DEBUG_IDX: src = L->ws.idx; n = 4 * T * k; break;
+        case MOE_DEBUG_W: src = L->ws.wts; n = 4 * T * k; break;
+        case MOE_DEBUG_ASC: src = L->ws.asc; n = 4 * T * k; break;
+        case MOE_DEBUG_ULIST: src = L->ws.ulist; n = 4 * E; break;
+        case MOE_DEBUG_CNT: src = L->ws.cnt; n = 4 * E; break;
+        case MOE_DEBUG_XSUM: src = L->ws.xsum; n = 8 * T; break;
+        default: return MOE_ERR_INVALID_ARG;
+    }
+    if ((size_t)bytes < n) n = (size_t)bytes;
+    cudaError_t e = L->last_stream ? cudaStreamSynchronize(L->last_stream) : cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpy(dst, src, n, cudaMemcpyDeviceToHost);
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status moe_layer_get_option(const moe_layer* L, int32_t option, int64_t* value) {
@@ -346,6 +391,8 @@ moe_status moe_layer_get_option(const moe_layer* L, int32_t option, int64_t* val
     switch (option) {
         case MOE_OPT_PREFILL_MIN_TOKENS: *value = L->prefill_min_tokens; return MOE_OK;
         case MOE_OPT_PREFILL_AVAILABLE: *value = L->plan ? 1 : 0; return MOE_OK;
+        case MOE_OPT_SINGLE_TOKEN_KERNELS: *value = L->t1_kernels ? 1 : 0; return MOE_OK;
+        case MOE_OPT_PROGRAMMATIC_LAUNCH: *value = L->dims.pdl; return MOE_OK;
         default: return MOE_ERR_INVALID_ARG;
     }
 }

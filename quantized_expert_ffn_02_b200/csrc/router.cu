@@ -147,7 +147,222 @@ topk_kernel(const double* __restrict__ logits, const float* __restrict__ bias, i
     }
 }
 
+// ---------------------------------------------------------------------------------------
+// Small batches (T <= 32): one launch for logits, top-k, gate weights and bucketing.
+// grid = E blocks of 256 threads, block e computes logits[t][e] for every token; the last block
+// to finish (an atomic counter, reset by that block) selects and buckets all T tokens.
+// ---------------------------------------------------------------------------------------
+constexpr int kSmallThreads = 256;
+constexpr int kSmallMaxT = 32;
+constexpr int kSmallMaxE = 1024;
+
+template <int MAXPER>
+__device__ void warp_select(const double* __restrict__ lg, const float* __restrict__ bias, int E, int k, int router,
+                            float scaling, int lane, int32_t* idx_out, float* w_out, int32_t* asc_out) {
+    double key[MAXPER];
+    uint32_t taken = 0;
+#pragma unroll
+    for (int m = 0; m < MAXPER; ++m) {
+        const int e = lane + kWarp * m;
+        double kv = -INFINITY;
+        if (e < E) {
+            const double l = __ldcg(lg + e);       // written by other blocks: read through L2
+            kv = router == MOE_ROUTER_SIGMOID_BIAS ? 1.0 / (1.0 + exp(-l)) + (bias ? (double)bias[e] : 0.0) : l;
+            if (isnan(kv)) kv = -INFINITY;
+        } else {
+            taken |= 1u << m;
+        }
+        key[m] = kv;
+    }
+    int my_e = -1;
+    for (int r = 0; r < k; ++r) {
+        double bk = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int m = 0; m < MAXPER; ++m) {
+            const int e = lane + kWarp * m;
+            if (!(taken >> m & 1u) && beats(key[m], e, bk, bi)) { bk = key[m]; bi = e; }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const double ok = __shfl_xor_sync(0xffffffffu, bk, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (beats(ok, oi, bk, bi)) { bk = ok; bi = oi; }
+        }
+        if ((bi % kWarp) == lane) taken |= 1u << (bi / kWarp);
+        if (lane == r) my_e = bi;
+    }
+    const bool mine = lane < k;
+    const double l = mine ? __ldcg(lg + my_e) : 0.0;
+    double num, den;
+    if (router == MOE_ROUTER_SIGMOID_BIAS) {
+        num = mine ? 1.0 / (1.0 + exp(-l)) : 0.0;
+        den = warp_sum_d(num);
+    } else {
+        double m = mine ? l : -INFINITY;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+        num = mine ? exp(l - m) : 0.0;
+        den = warp_sum_d(num);
+    }
+    int pos = 0;
+    for (int r2 = 0; r2 < k; ++r2) {
+        const int e2 = __shfl_sync(0xffffffffu, my_e, r2);
+        if (mine && e2 < my_e) ++pos;
+    }
+    if (mine) {
+        idx_out[lane] = my_e;
+        w_out[lane] = (float)((double)scaling * num / den);
+        asc_out[pos] = lane;
+    }
+}
+
+template <int MAXPER>
+__global__ void __launch_bounds__(kSmallThreads, 2)
+route_small_kernel(const float* __restrict__ wr, const float* __restrict__ bias, const uint16_t* __restrict__ x, int T,
+                   int d, int E, int k, int router, float scaling, double* __restrict__ logits,
+                   double* __restrict__ xsum, int32_t* __restrict__ idx, float* __restrict__ wts,
+                   int32_t* __restrict__ asc, int32_t* __restrict__ cnt, int32_t* __restrict__ off,
+                   int32_t* __restrict__ perm, int32_t* __restrict__ slot_of, int32_t* __restrict__ ulist,
+                   int32_t* __restrict__ n_unique, unsigned int* __restrict__ counter) {
+    __shared__ double red[kSmallThreads / kWarp][kSmallMaxT];
+    __shared__ double redx[kSmallThreads / kWarp];
+    __shared__ int s_cnt[kSmallMaxE], s_off[kSmallMaxE], s_scan[kSmallThreads];
+    __shared__ int am_last;
+    const int e = blockIdx.x, tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
+    // A kernel launched after this one with programmatic dependent launch may start now: it
+    // waits (griddepcontrol.wait) before it reads anything written here.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // ---- logits of expert e for every token
+    // all of this thread's router-row loads in flight at once (d <= 14336: at most 14 per thread)
+    constexpr int kMaxC = 14;
+    const float4* wrow = reinterpret_cast<const float4*>(wr + (size_t)e * d);
+    const int nc = (d / 4 - tid + kSmallThreads - 1) / kSmallThreads;
+    float4 wv[kMaxC];
+#pragma unroll
+    for (int j = 0; j < kMaxC; ++j)
+        if (j < nc) wv[j] = __ldg(wrow + tid + kSmallThreads * j);
+    for (int t = 0; t < T; ++t) {
+        const uint2* xr2 = reinterpret_cast<const uint2*>(x + (size_t)t * d) + tid;
+        uint2 xv[kMaxC];
+#pragma unroll
+        for (int j = 0; j < kMaxC; ++j)
+            if (j < nc) xv[j] = __ldg(xr2 + kSmallThreads * j);
+        double a = 0.0;
+#pragma unroll
+        for (int j = 0; j < kMaxC; ++j) {
+            if (j < nc) {
+                a = fma((double)__uint_as_float(xv[j].x << 16), (double)wv[j].x, a);
+                a = fma((double)__uint_as_float(xv[j].x & 0xffff0000u), (double)wv[j].y, a);
+                a = fma((double)__uint_as_float(xv[j].y << 16), (double)wv[j].z, a);
+                a = fma((double)__uint_as_float(xv[j].y & 0xffff0000u), (double)wv[j].w, a);
+            }
+        }
+        a = warp_sum_d(a);
+        if (lane == 0) red[warp][t] = a;
+    }
+    __syncthreads();
+    if (tid < T) {
+        double s = 0.0;
+        for (int w = 0; w < kSmallThreads / kWarp; ++w) s += red[w][tid];
+        logits[(size_t)tid * E + e] = s;
+    }
+    // ---- sum of x for the tokens t with t % E == e (one block per token)
+    for (int t = e; t < T; t += E) {
+        double s = 0.0;
+        for (int i = tid; i < d; i += kSmallThreads) s += (double)bf16_bits_to_f32(x[(size_t)t * d + i]);
+        s = warp_sum_d(s);
+        __syncthreads();
+        if (lane == 0) redx[warp] = s;
+        __syncthreads();
+        if (tid == 0) {
+            double tot = 0.0;
+            for (int w = 0; w < kSmallThreads / kWarp; ++w) tot += redx[w];
+            xsum[t] = tot;
+        }
+    }
+    // ---- the last block to finish selects and buckets
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) am_last = atomicAdd(counter, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!am_last) return;
+    __threadfence();
+    for (int t = warp; t < T; t += kSmallThreads / kWarp)
+        warp_select<MAXPER>(logits + (size_t)t * E, bias, E, k, router, scaling, lane, idx + (size_t)t * k,
+                            wts + (size_t)t * k, asc + (size_t)t * k);
+    for (int i = tid; i < E; i += kSmallThreads) s_cnt[i] = 0;
+    __syncthreads();
+    __threadfence_block();
+    for (int i = tid; i < T * k; i += kSmallThreads) atomicAdd(&s_cnt[idx[i]], 1);
+    __syncthreads();
+    // exclusive scan of the counts (each thread owns a run of experts) and of the used flags
+    const int per = (E + kSmallThreads - 1) / kSmallThreads;
+    const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
+    int sum = 0, used = 0;
+    for (int i = e0; i < e1; ++i) { sum += s_cnt[i]; used += s_cnt[i] > 0; }
+    s_scan[tid] = sum | (used << 16);       // T*k <= 1024 < 2^16 and E <= 1024 < 2^16
+    __syncthreads();
+    for (int o = 1; o < kSmallThreads; o <<= 1) {
+        const int add = tid >= o ? s_scan[tid - o] : 0;
+        __syncthreads();
+        s_scan[tid] += add;
+        __syncthreads();
+    }
+    int base = tid ? s_scan[tid - 1] : 0;
+    int run = base & 0xffff, urun = base >> 16;
+    for (int i = e0; i < e1; ++i) {
+        const int c = s_cnt[i];
+        s_off[i] = run;
+        cnt[i] = c;
+        off[i] = run;
+        if (c > 0) ulist[urun++] = i;
+        run += c;
+    }
+    if (tid == kSmallThreads - 1) {
+        off[E] = s_scan[tid] & 0xffff;
+        *n_unique = s_scan[tid] >> 16;
+    }
+    __syncthreads();
+    // stable placement in token order (the k experts of a token are distinct)
+    if (warp == 0) {
+        for (int t = 0; t < T; ++t) {
+            if (lane < k) {
+                const int ex = idx[(size_t)t * k + lane];
+                const int p = s_off[ex]++;
+                perm[p] = t * k + lane;
+                slot_of[(size_t)t * k + lane] = p;
+            }
+            __syncwarp();
+        }
+    }
+    if (tid == 0) *counter = 0u;
+}
+
 }  // namespace
+
+cudaError_t launch_route_small(const LayerDims& L, const float* router_w, const float* router_bias, const uint16_t* x,
+                               int T, const Workspace& ws, const Launch& ctx) {
+    if (T == 0) return cudaSuccess;
+    const float* bias = L.router == MOE_ROUTER_SIGMOID_BIAS ? router_bias : nullptr;
+    unsigned int* counter = reinterpret_cast<unsigned int*>(ws.counter);
+    if (L.E <= 32)
+        QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,
+                  (route_small_kernel<1><<<L.E, kSmallThreads, 0, ctx.s>>>(
+                      router_w, bias, x, T, L.d, L.E, L.k, L.router, L.scaling, ws.logits, ws.xsum, ws.idx, ws.wts,
+                      ws.asc, ws.cnt, ws.off, ws.perm, ws.slot_of, ws.ulist, ws.n_unique, counter)));
+    else if (L.E <= 256)
+        QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,
+                  (route_small_kernel<8><<<L.E, kSmallThreads, 0, ctx.s>>>(
+                      router_w, bias, x, T, L.d, L.E, L.k, L.router, L.scaling, ws.logits, ws.xsum, ws.idx, ws.wts,
+                      ws.asc, ws.cnt, ws.off, ws.perm, ws.slot_of, ws.ulist, ws.n_unique, counter)));
+    else
+        QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,
+                  (route_small_kernel<32><<<L.E, kSmallThreads, 0, ctx.s>>>(
+                      router_w, bias, x, T, L.d, L.E, L.k, L.router, L.scaling, ws.logits, ws.xsum, ws.idx, ws.wts,
+                      ws.asc, ws.cnt, ws.off, ws.perm, ws.slot_of, ws.ulist, ws.n_unique, counter)));
+    return cudaSuccess;
+}
 
 // The opt-in is set to the whole 227 KB once per device, so that layers of different widths
 // can coexist; each launch still asks only for its own tile.

@@ -156,10 +156,16 @@ def test_glm_route_bitexact(glm, T, offset):
 def test_glm_batch_union_reads_each_expert_once_per_call(glm):
     # the union result of a batch equals the per-token results (same token, same output)
     x = glm["x32"]
-    out_b = run_forward(glm["layer"], x)
-    for i in (0, 7, 31):
-        out_1 = run_forward(glm["layer"], x[i:i + 1])
-        check_close(out_1, out_b[i:i + 1].astype(np.float64), rel_l2=1e-5, max_rms=1e-4)
+    layer = glm["layer"]
+    out_b = run_forward(layer, x)
+    for t1, tol in ((False, 1e-5), (True, 1e-4)):
+        # the same kernels give nearly the same sums; the single-token kernels add in another order,
+        # and an fp16 rounding of h can flip, so their bound is looser (still far inside the spec)
+        layer.set_single_token_kernels(t1)
+        for i in (0, 7, 31):
+            out_1 = run_forward(layer, x[i:i + 1])
+            check_close(out_1, out_b[i:i + 1].astype(np.float64), rel_l2=tol, max_rms=10 * tol)
+    layer.set_single_token_kernels(True)
 
 
 # ------------------------------------------------------------------------------------------
