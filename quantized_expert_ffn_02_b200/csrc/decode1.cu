@@ -146,17 +146,21 @@ gateup_t1_kernel(const uint8_t* __restrict__ gate_up, const float* __restrict__ 
                  const uint8_t* __restrict__ sh_gate_up, const float* __restrict__ sh_gu_scale,
                  const uint16_t* __restrict__ x, int k, int d, int f, int f_sh, int S, const int32_t* ulist,
                  uint16_t* __restrict__ h, int fmax, int* status) {
-    extern __shared__ __align__(128) uint8_t smem[];          // [warps][kGuStages][2 * rowbytes]
+    // [warps][kGuStages][gate row | up row | 16 B holding the gate scale | 16 B holding the up scale]
+    extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bars[kGuMaxWarps][kGuStages];
+    __shared__ int s_ulist[kGuMaxWarps][kDnMaxSlots];      // this warp's copy of the routed experts
     const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
     const int nwarps_cta = blockDim.x / kWarp;
     const int gw = blockIdx.x * nwarps_cta + warp;
     const int nw = gridDim.x * nwarps_cta;
     const uint32_t rowbytes = (uint32_t)d / 2;
+    const uint32_t stage_bytes = 2 * rowbytes + 32;
     const int n_shared_tasks = S ? f_sh : 0;
     const int n_tasks = n_shared_tasks + k * f;
     const int my_tasks = gw < n_tasks ? (n_tasks - gw + nw - 1) / nw : 0;
-    const uint32_t ring = saddr(smem) + (uint32_t)warp * kGuStages * 2 * rowbytes;
+    const uint32_t ring = saddr(smem) + (uint32_t)warp * kGuStages * stage_bytes;
+    const uint8_t* ring_g = smem + (size_t)warp * kGuStages * stage_bytes;
     if (lane == 0) {
         for (int s = 0; s < kGuStages; ++s) bar_init(saddr(&bars[warp][s]), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -177,11 +181,12 @@ gateup_t1_kernel(const uint8_t* __restrict__ gate_up, const float* __restrict__ 
             if (!routed_ready) {
                 pdl_wait();
                 pdl_trigger();          // the down kernel may now read the routing
+                for (int q = 0; q < k; ++q) s_ulist[warp][q] = __ldcg(ulist + q);
                 routed_ready = true;
             }
             const int t2 = t - n_shared_tasks;
             const int u = t2 / f, r = t2 % f;
-            const int e = __ldcg(ulist + u);
+            const int e = s_ulist[warp][u];
             tk.gate = gate_up + ((size_t)e * 2 * f + r) * rowbytes;
             tk.sc = gu_scale + (size_t)e * 2 * f + r;
             tk.r = r;
@@ -190,22 +195,29 @@ gateup_t1_kernel(const uint8_t* __restrict__ gate_up, const float* __restrict__ 
         }
         return tk;
     };
-    // lane 0 issues task i into stage i % kGuStages
+    // lane 0 issues task i into stage i % kGuStages: both rows, and the 16-byte aligned slivers of
+    // the scale arrays that hold their two scales (scale arrays are 16-byte aligned and a routed
+    // expert's scales start at a multiple of 4 floats)
+    auto sliver = [](const float* p) { return reinterpret_cast<const float*>((uintptr_t)p & ~(uintptr_t)15); };
     auto issue = [&](int i) {
         const GuTask tk = task(i);
         const uint32_t bar = saddr(&bars[warp][i % kGuStages]);
-        const uint32_t dst = ring + (uint32_t)(i % kGuStages) * 2 * rowbytes;
-        bar_expect_tx(bar, 2 * rowbytes);
+        const uint32_t dst = ring + (uint32_t)(i % kGuStages) * stage_bytes;
+        bar_expect_tx(bar, stage_bytes);
         bulk_g2s(dst, tk.gate, rowbytes, bar);
         bulk_g2s(dst + rowbytes, tk.gate + (size_t)tk.fe * rowbytes, rowbytes, bar);
+        bulk_g2s(dst + 2 * rowbytes, sliver(tk.sc), 16, bar);
+        bulk_g2s(dst + 2 * rowbytes + 16, sliver(tk.sc + tk.fe), 16, bar);
     };
     int issued = 0;
     if (lane == 0)      // prologue: shared-expert rows only (they need no routing)
         while (issued < my_tasks && issued < kGuStages && gw + issued * nw < n_shared_tasks) issue(issued++);
 
     // the token's activations: lane owns chunks lane + 32 j
+    // sum of x: each lane's share in fp32, the 32 partials in fp64 (the offset removed per row is
+    // 136 times this sum; its error stays far below the rounding of the fp32 row sums)
     uint32_t xr[NCH][16];
-    double xs = 0.0;
+    float xsl = 0.0f;
 #pragma unroll
     for (int j = 0; j < NCH; ++j) {
         const int c = lane + kWarp * j;
@@ -216,10 +228,10 @@ gateup_t1_kernel(const uint8_t* __restrict__ gate_up, const float* __restrict__ 
             const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                xs += (double)__uint_as_float(ws[q] << 16) + (double)__uint_as_float(ws[q] & 0xffff0000u);
+                xsl += __uint_as_float(ws[q] << 16) + __uint_as_float(ws[q] & 0xffff0000u);
         }
     }
-    xs = warp_sum_d(xs);
+    const double xs = warp_sum_d((double)xsl);
     const float off136 = 136.0f * (float)xs;
 
     bool ok = true;
@@ -230,7 +242,7 @@ gateup_t1_kernel(const uint8_t* __restrict__ gate_up, const float* __restrict__ 
         ok = bar_wait(saddr(&bars[warp][s]), (uint32_t)(i / kGuStages) & 1u);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
-        const uint32_t st = ring + (uint32_t)s * 2 * rowbytes;
+        const uint32_t st = ring + (uint32_t)s * stage_bytes;
         float ag = 0.0f, au = 0.0f;
 #pragma unroll
         for (int j = 0; j < NCH; ++j) {
@@ -245,15 +257,18 @@ gateup_t1_kernel(const uint8_t* __restrict__ gate_up, const float* __restrict__ 
             ag = dot_word_bf16(G.w, &xr[j][12], ag);
             au = dot_word_bf16(U.w, &xr[j][12], au);
         }
+        // the row index and the two scales of this task, read before the stage is handed back
+        const GuTask tk = task(i);
+        const float* scs = reinterpret_cast<const float*>(ring_g + (size_t)s * stage_bytes + 2 * rowbytes);
+        const float sg = scs[(uintptr_t)tk.sc / 4 & 3], su = scs[4 + ((uintptr_t)(tk.sc + tk.fe) / 4 & 3)];
         __syncwarp();                                          // stage s is free again
         if (lane == 0)
             while (issued < my_tasks && issued < i + 1 + kGuStages) issue(issued++);
         ag = warp_sum(ag);
         au = warp_sum(au);
         if (lane == 0) {
-            const GuTask tk = task(i);
-            const float gv = __ldg(tk.sc) * (ag - off136);
-            const float uv = __ldg(tk.sc + tk.fe) * (au - off136);
+            const float gv = sg * (ag - off136);
+            const float uv = su * (au - off136);
             const float hv = gv / (1.0f + expf(-gv)) * uv;
             const __half hh = __float2half_rn(hv);
             if (!isfinite(__half2float(hh)) && isfinite(hv)) latch_status(status, MOE_ERR_RANGE);
@@ -321,6 +336,8 @@ down_t1_kernel(const uint8_t* __restrict__ down, const float* __restrict__ dn_sc
     int issued = 0;
     if (lane == 0)                  // the weights do not depend on h: start before the wait
         while (issued < nstages && issued < kDnStages) issue(issued++);
+    // lane q holds the scale of this warp's row q (a warp has at most 32 rows)
+    const float my_sc = lane < nrows ? __ldg(sc + j0 + r0 + lane) : 0.0f;
     pdl_wait();                     // h is complete
     uint32_t hr[NCH][16];
 #pragma unroll
@@ -359,7 +376,8 @@ down_t1_kernel(const uint8_t* __restrict__ down, const float* __restrict__ dn_sc
 #pragma unroll
         for (int q = 0; q < kDnRows; ++q) {
             const float v = warp_sum(acc[q]);
-            if (lane == 0 && q < n) ys[u][a + q] = __ldg(sc + j0 + a + q) * v;
+            const float s_row = __shfl_sync(0xffffffffu, my_sc, (a - r0 + q) & 31);
+            if (lane == 0 && q < n) ys[u][a + q] = s_row * v;
         }
     }
     if (lane == 0 && !ok) {
@@ -398,8 +416,9 @@ cudaError_t launch_pdl(bool programmatic, Kern kernel, dim3 grid, dim3 block, si
     return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+size_t gu_stage_bytes(const LayerDims& L) { return (size_t)L.d + 32; }   // two rows of d/2 bytes + scales
 int gu_warps(const LayerDims& L) {
-    const size_t per_warp = (size_t)kGuStages * L.d;     // kGuStages x (gate + up rows of d/2 bytes)
+    const size_t per_warp = (size_t)kGuStages * gu_stage_bytes(L);
     const int w = (int)((kSmemLimit - 4096) / per_warp);
     return w > kGuMaxWarps ? kGuMaxWarps : w;
 }
@@ -440,7 +459,7 @@ cudaError_t launch_decode_t1(const LayerDims& L, const moe_weights& W, const uin
     const int fmax = L.f;
     const int nchx = L.d / 1024, nchf = L.f / 1024;
     const int guw = gu_warps(L);
-    const size_t gu_smem = (size_t)guw * kGuStages * L.d;
+    const size_t gu_smem = (size_t)guw * kGuStages * gu_stage_bytes(L);
     cudaError_t e = cudaSuccess;
     prof_mark(ctx.prof, MOE_KERNEL_GATEUP, true, ctx.s);
 #define QE_GU(N)                                                                                                      \

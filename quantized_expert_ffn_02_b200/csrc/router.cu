@@ -65,6 +65,83 @@ router_logits_kernel(const float* __restrict__ wr, const uint16_t* __restrict__ 
     }
 }
 
+// ---------------------------------------------------------------------------------------
+// Large batches: logits = X Wr^T as a tiled fp64 GEMM.  A CTA computes 64 tokens x 64 experts;
+// every x and w element is converted to fp64 once per tile (into shared memory) and each thread
+// keeps a 4 x 4 register tile.  The next K chunk's global loads are in flight while the current
+// chunk is multiplied.  CTAs of the first expert tile also write sum_i x[t][i].
+// ---------------------------------------------------------------------------------------
+constexpr int kRgT = 64, kRgE = 64, kRgK = 32, kRgThreads = 256;
+
+__global__ void __launch_bounds__(kRgThreads)
+router_gemm_kernel(const float* __restrict__ wr, const uint16_t* __restrict__ x, int T, int d, int E,
+                   double* __restrict__ logits, double* __restrict__ xsum) {
+    __shared__ double xs[kRgK][kRgT + 1];
+    __shared__ double ws[kRgK][kRgE + 1];
+    const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+    const int t0 = blockIdx.x * kRgT, e0 = blockIdx.y * kRgE;
+    // loader roles: 4 threads per token row (8 bf16 each) and per expert row (8 fp32 each)
+    const int lr = tid / 4, lc = (tid % 4) * 8;
+    const bool xrow_ok = t0 + lr < T;
+    const bool sum_x = blockIdx.y == 0;
+    const uint16_t* xrow = x + (size_t)(xrow_ok ? t0 + lr : 0) * d + lc;
+    const float* wrow = wr + (size_t)(e0 + lr) * d + lc;
+    uint4 xv = xrow_ok ? ld_ro16(xrow) : make_uint4(0, 0, 0, 0);
+    float4 wa = __ldg(reinterpret_cast<const float4*>(wrow)), wb = __ldg(reinterpret_cast<const float4*>(wrow) + 1);
+    double acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+    double xpart = 0.0;
+    for (int k0 = 0; k0 < d; k0 += kRgK) {
+        // convert the staged chunk into shared memory (K-major)
+        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const double lo = (double)__uint_as_float(xw[q] << 16), hi = (double)__uint_as_float(xw[q] & 0xffff0000u);
+            xs[lc + 2 * q][lr] = lo;
+            xs[lc + 2 * q + 1][lr] = hi;
+            if (sum_x) xpart += lo + hi;
+        }
+        const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+        for (int q = 0; q < 8; ++q) ws[lc + q][lr] = (double)wv[q];
+        __syncthreads();
+        // next chunk's loads go out before this chunk is multiplied
+        if (k0 + kRgK < d) {
+            xv = xrow_ok ? ld_ro16(xrow + k0 + kRgK) : make_uint4(0, 0, 0, 0);
+            wa = __ldg(reinterpret_cast<const float4*>(wrow + k0 + kRgK));
+            wb = __ldg(reinterpret_cast<const float4*>(wrow + k0 + kRgK) + 1);
+        }
+#pragma unroll 8
+        for (int kk = 0; kk < kRgK; ++kk) {
+            double a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = xs[kk][4 * ty + i];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) b[j] = ws[kk][4 * tx + j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int t = t0 + 4 * ty + i;
+        if (t < T)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) logits[(size_t)t * E + e0 + 4 * tx + j] = acc[i][j];
+    }
+    if (sum_x) {     // the 4 loader threads of a token are adjacent lanes
+        xpart += __shfl_xor_sync(0xffffffffu, xpart, 1);
+        xpart += __shfl_xor_sync(0xffffffffu, xpart, 2);
+        if ((tid & 3) == 0 && xrow_ok) xsum[t0 + lr] = xpart;
+    }
+}
+
 struct KeyIdx {
     double key;
     int idx;
@@ -377,10 +454,17 @@ cudaError_t launch_router(const LayerDims& L, const float* router_w, const float
                           int32_t* asc, const Launch& ctx) {
     if (T == 0) return cudaSuccess;
     const cudaStream_t s = ctx.s;
-    const size_t smem = (size_t)kRouterTokens * L.d * sizeof(uint16_t);
-    dim3 grid((L.E + kRouterWarps - 1) / kRouterWarps, (T + kRouterTokens - 1) / kRouterTokens);
-    QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,
-              (router_logits_kernel<<<grid, kRouterWarps * kWarp, smem, s>>>(router_w, x, T, L.d, L.E, logits, xsum)));
+    if (T >= kRgT && L.E % kRgE == 0 && L.d % kRgK == 0) {
+        dim3 grid((unsigned)((T + kRgT - 1) / kRgT), (unsigned)(L.E / kRgE));
+        QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,
+                  (router_gemm_kernel<<<grid, kRgThreads, 0, s>>>(router_w, x, T, L.d, L.E, logits, xsum)));
+    } else {
+        const size_t smem = (size_t)kRouterTokens * L.d * sizeof(uint16_t);
+        dim3 grid((L.E + kRouterWarps - 1) / kRouterWarps, (T + kRouterTokens - 1) / kRouterTokens);
+        QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,
+                  (router_logits_kernel<<<grid, kRouterWarps * kWarp, smem, s>>>(router_w, x, T, L.d, L.E, logits,
+                                                                                  xsum)));
+    }
     const int tpb = 8;
     const unsigned g = (unsigned)((T + tpb - 1) / tpb);
     const float* bias = L.router == MOE_ROUTER_SIGMOID_BIAS ? router_bias : nullptr;
