@@ -63,6 +63,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--t1-mode", type=int, default=None, choices=[0, 1, 2],
+                    help="single-token path: 2 one launch, 1 three kernels, 0 general kernels (default: the library's)")
     ap.add_argument("--experts", type=int, default=None,
                     help="override E (smaller device footprint for profiler captures; same per-token work)")
     a = ap.parse_args()
@@ -264,8 +266,11 @@ def kernel_work(cfg, T, n_unique):
     # the single-token kernel adds the slots itself and writes the output; the others write y per slot
     dn = dn_w + (T * cfg.d * 4 if T == 1 else slots * cfg.d * 4)
     mac = T * cfg.k * cfg.d * cfg.f + T * S * cfg.d * cfg.f_shared
+    # the single launch (T = 1): router matrix and bias, x, every expert byte, h written and read
+    # back, the output
+    fused = cfg.E * cfg.d * 4 + cfg.E * 4 + gu + dn_w + slots * fmax * 2 + cfg.d * 4
     return {"gateup": ("hbm", gu), "down": ("hbm", dn), "gemm_gateup": ("tensor", 4 * mac),
-            "gemm_down": ("tensor", 2 * mac)}
+            "gemm_down": ("tensor", 2 * mac), "fused": ("hbm", fused)}
 
 
 def source_sha(paths):
@@ -349,6 +354,8 @@ def run_ours(a, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     T = cfg.T
     layer, W = build_device_layer(cfg, a.seed, T, dev)
+    if a.t1_mode is not None:
+        layer.set_single_token_mode(a.t1_mode)
     # every rank is an independent replica with its own tokens
     n_batches = a.warmup + a.steps if T <= 32 else 4
     token_base = rank * 1_000_000

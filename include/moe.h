@@ -174,9 +174,14 @@ void moe_layer_destroy(moe_layer *layer);
  *   MOE_OPT_PREFILL_AVAILABLE   (read only) 1 if this layer has the grouped-GEMM path.
  * Setting an option is host-only and takes effect at the next moe_forward.
  */
-/*   MOE_OPT_SINGLE_TOKEN_KERNELS 1 (default): a T = 1 batch uses the dedicated single-token
- *                               kernels when the shape allows (int4, d and f multiples of 1024,
- *                               f_shared == f, k + shared <= 10); 0: the general decode kernels.
+/*   MOE_OPT_SINGLE_TOKEN_KERNELS how a T = 1 batch runs when the shape allows (int4 weights, d a
+ *                               multiple of 1024 up to 8192, f_shared == f, k + shared <= 10):
+ *                               2 (default where f is 1024 or 2048 and E <= 256): the whole layer
+ *                               in one cooperative launch (router, top-k, gate/up, down, combine);
+ *                               1: the fused router launch, then the single-token gate/up and
+ *                               down+combine kernels; 0: the general decode kernels.  A request
+ *                               for a mode the shape does not allow falls back to the next lower
+ *                               one; get returns the mode in use.  Same results within tolerance.
  */
 /*   MOE_OPT_PROGRAMMATIC_LAUNCH  1 (default): chained kernels of the single-token path start
  *                               early with programmatic dependent launch and wait on the device
@@ -196,10 +201,16 @@ moe_status moe_layer_get_option(const moe_layer *layer, int32_t option, int64_t 
  *   MOE_DEBUG_Y      y per slot, fp32 [slots][d] (not written by the single-token kernels)
  *   MOE_DEBUG_IDX / MOE_DEBUG_W / MOE_DEBUG_ASC   int32 / fp32 / int32 [T][k]
  *   MOE_DEBUG_ULIST  int32 [E] unique chosen experts, ascending;  MOE_DEBUG_CNT int32 [E]
+ *                    (CNT is not written by the single-launch T = 1 path)
  *   MOE_DEBUG_XSUM   fp64 [T]
+ *   MOE_DEBUG_TRACE  uint64 [SMs][16]: for the single-launch T = 1 path, the %globaltimer value (ns)
+ *                    at which each CTA passed its phase boundaries: 0 start, 1 x in registers,
+ *                    2 router pieces stored, 3 shared rows done, 4 first grid barrier passed,
+ *                    5 router pieces gathered, 6 experts selected, 7 routed gate/up done, 8 h
+ *                    complete, 9 down done, 10 output stored (11..15 unused)
  */
 enum { MOE_DEBUG_H = 0, MOE_DEBUG_Y = 1, MOE_DEBUG_IDX = 2, MOE_DEBUG_W = 3, MOE_DEBUG_ASC = 4,
-       MOE_DEBUG_ULIST = 5, MOE_DEBUG_CNT = 6, MOE_DEBUG_XSUM = 7 };
+       MOE_DEBUG_ULIST = 5, MOE_DEBUG_CNT = 6, MOE_DEBUG_XSUM = 7, MOE_DEBUG_TRACE = 8 };
 moe_status moe_layer_debug_read(moe_layer *layer, int32_t item, void *dst, int64_t bytes);
 
 /* Bytes of device workspace the layer holds. */
@@ -227,7 +238,8 @@ enum {
     MOE_KERNEL_GATHER = 6,          /* prefill: x rows gathered per expert */
     MOE_KERNEL_GEMM_GATEUP = 7,     /* prefill: tcgen05 grouped GEMM gate/up + SiLU */
     MOE_KERNEL_GEMM_DOWN = 8,       /* prefill: tcgen05 grouped GEMM down */
-    MOE_KERNEL_COUNT = 9
+    MOE_KERNEL_FUSED = 9,           /* decode, T = 1: the whole layer in one cooperative launch */
+    MOE_KERNEL_COUNT = 10
 };
 /*
  * moe_route_noalloc -- the routing step of moe_route, for callers that must not allocate device

@@ -26,8 +26,9 @@ EXPORTS = (
     "moe_layer_set_option", "moe_layer_get_option", "moe_layer_debug_read",
 )
 MOE_OPT_PREFILL_MIN_TOKENS, MOE_OPT_PREFILL_AVAILABLE, MOE_OPT_SINGLE_TOKEN_KERNELS, MOE_OPT_PROGRAMMATIC_LAUNCH = 0, 1, 2, 3
-DEBUG_ITEMS = {"h": 0, "y": 1, "idx": 2, "w": 3, "asc": 4, "ulist": 5, "cnt": 6, "xsum": 7}
-KERNELS = ("router_logits", "topk", "bucket", "gateup", "down", "combine", "gather", "gemm_gateup", "gemm_down")
+DEBUG_ITEMS = {"h": 0, "y": 1, "idx": 2, "w": 3, "asc": 4, "ulist": 5, "cnt": 6, "xsum": 7, "trace": 8}
+KERNELS = ("router_logits", "topk", "bucket", "gateup", "down", "combine", "gather", "gemm_gateup", "gemm_down",
+           "fused")
 
 
 class MoeError(RuntimeError):
@@ -229,8 +230,16 @@ class MoELayer:
     def last_launches(self) -> int:
         return moe_layer_last_launches(self.handle)
 
-    def set_single_token_kernels(self, on: bool):
-        moe_layer_set_option(self.handle, MOE_OPT_SINGLE_TOKEN_KERNELS, 1 if on else 0)
+    def set_single_token_mode(self, mode: int) -> int:
+        """T = 1 path: 2 one cooperative launch, 1 router + two single-token kernels, 0 general
+        kernels.  A mode the shape does not allow falls back to the next lower one; returns the
+        mode in use."""
+        moe_layer_set_option(self.handle, MOE_OPT_SINGLE_TOKEN_KERNELS, int(mode))
+        return self.single_token_mode
+
+    @property
+    def single_token_mode(self) -> int:
+        return moe_layer_get_option(self.handle, MOE_OPT_SINGLE_TOKEN_KERNELS)
 
     def debug_read(self, item: str, dst):
         moe_layer_debug_read(self.handle, item, dst)

@@ -114,7 +114,13 @@ struct Workspace {
     int32_t* groups;       // [max_groups][4]: (expert or -1, first slot, tokens, unused)
     int32_t* n_groups;     // [2]: routed groups, shared groups
     uint32_t* counter;     // [1]: blocks done in the fused small-batch router (reset to 0 by the last)
+    // single-launch decode path
+    double* rpart;         // [E][d / 1024]: pieces of the router logits
+    unsigned long long* gbar;  // [1]: grid-barrier arrivals (only grows)
+    unsigned long long* trace; // [kTraceCtas][kTraceStamps]: phase timestamps of that path
 };
+constexpr int kTraceCtas = 1024;
+constexpr int kTraceStamps = 16;
 
 struct LayerDims {
     int d, f, E, k, S, f_shared, router, wkind, out_bf16;
@@ -152,6 +158,12 @@ cudaError_t launch_route_small(const LayerDims& L, const float* router_w, const 
 bool decode_t1_supported(const LayerDims& L);
 cudaError_t launch_decode_t1(const LayerDims& L, const moe_weights& W, const uint16_t* x, const Workspace& ws,
                              void* out, int num_sms, const Launch& ctx);
+// One token, int4 experts, the whole layer in one cooperative launch (decode_fused.cu).
+bool decode_fused_shape_ok(const LayerDims& L);
+cudaError_t prepare_decode_fused(const LayerDims& L, int num_sms, bool* usable);
+size_t decode_fused_rpart_count(const LayerDims& L);
+cudaError_t launch_decode_fused(const LayerDims& L, const moe_weights& W, const uint16_t* x, const Workspace& ws,
+                                void* out, int num_sms, const Launch& ctx);
 cudaError_t launch_decode_experts(const LayerDims& L, const moe_weights& W, const uint16_t* x, int T,
                                   const Workspace& ws, int num_sms, const Launch& ctx);
 cudaError_t launch_combine(const LayerDims& L, int T, const Workspace& ws, void* out, const Launch& ctx);

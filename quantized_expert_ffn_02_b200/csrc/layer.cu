@@ -83,7 +83,8 @@ struct moe_layer {
     qe::Profiler prof;
     qe::PrefillPlan* plan = nullptr;     // TMA maps of the grouped-GEMM path (null if unsupported)
     int64_t prefill_min_tokens = 128;    // batches at least this large take the grouped-GEMM path
-    bool t1_kernels = false;             // the dedicated single-token decode kernels apply
+    int t1_mode = 0;                     // T = 1: 2 single launch, 1 single-token kernels, 0 general
+    bool fused_ok = false;               // the single-launch path is usable for this layer
 };
 
 namespace {
@@ -128,6 +129,9 @@ size_t carve(const moe_config& c, size_t max_groups, char* base, qe::Workspace* 
     w.Y = (float*)take(sizeof(float) * slots * (size_t)c.d);
     w.status = (int32_t*)take(sizeof(int32_t));
     w.counter = (uint32_t*)take(sizeof(uint32_t));
+    w.rpart = (double*)take(sizeof(double) * E * (c.d / 1024 > 0 ? (size_t)c.d / 1024 : 1));
+    w.gbar = (unsigned long long*)take(sizeof(unsigned long long));
+    w.trace = (unsigned long long*)take(sizeof(unsigned long long) * qe::kTraceCtas * qe::kTraceStamps);
     if (max_groups) {
         w.xg = (uint16_t*)take(sizeof(uint16_t) * slots * (size_t)c.d);
         w.groups = (int32_t*)take(sizeof(int32_t) * 4 * max_groups);
@@ -221,6 +225,7 @@ moe_status moe_layer_create(const moe_config* cfg, const moe_weights* w, moe_lay
     if (e == cudaSuccess) e = qe::prepare_router(L->dims);
     if (e == cudaSuccess) e = qe::prepare_bucket(L->dims);
     if (e == cudaSuccess) e = qe::prepare_decode(L->dims);
+    if (e == cudaSuccess) e = qe::prepare_decode_fused(L->dims, L->num_sms, &L->fused_ok);
     const bool gemm = qe::prefill_supported(L->dims);
     if (e == cudaSuccess && gemm) e = qe::prepare_prefill(L->dims);
     if (e != cudaSuccess) {
@@ -250,7 +255,7 @@ moe_status moe_layer_create(const moe_config* cfg, const moe_weights* w, moe_lay
             return MOE_ERR_CUDA;
         }
     }
-    L->t1_kernels = qe::decode_t1_supported(L->dims);
+    L->t1_mode = L->fused_ok ? 2 : qe::decode_t1_supported(L->dims) ? 1 : 0;
     L->last_stream = nullptr;
     *out = L;
     return MOE_OK;
@@ -280,6 +285,12 @@ moe_status moe_forward(moe_layer* L, const uint16_t* x, int32_t T, void* out, mo
     const qe::Workspace& ws = L->ws;
     const bool gemm = L->plan && T >= L->prefill_min_tokens;
     cudaError_t e;
+    if (T == 1 && L->t1_mode == 2) {
+        e = qe::launch_decode_fused(L->dims, L->w, x, ws, out, L->num_sms, ctx);
+        L->last_stream = s;
+        L->last_launches = launches;
+        return from_cuda(e);
+    }
     if (T <= qe::kRouteSmallMaxT) {
         e = qe::launch_route_small(L->dims, L->w.router_w, L->w.router_bias, x, T, ws, ctx);
     } else {
@@ -291,7 +302,7 @@ moe_status moe_forward(moe_layer* L, const uint16_t* x, int32_t T, void* out, mo
         if (gemm) {
             e = qe::launch_prefill_experts(L->dims, L->plan, L->w, x, T, ws, L->num_sms, ctx);
             if (e == cudaSuccess) e = qe::launch_combine(L->dims, T, ws, out, ctx);
-        } else if (T == 1 && L->t1_kernels) {
+        } else if (T == 1 && L->t1_mode >= 1) {
             e = qe::launch_decode_t1(L->dims, L->w, x, ws, out, L->num_sms, ctx);
         } else {
             e = qe::launch_decode_experts(L->dims, L->w, x, T, ws, L->num_sms, ctx);
@@ -349,10 +360,14 @@ moe_status moe_layer_set_option(moe_layer* L, int32_t option, int64_t value) {
             if (value < 1) return MOE_ERR_INVALID_ARG;
             L->prefill_min_tokens = value;
             return MOE_OK;
-        case MOE_OPT_SINGLE_TOKEN_KERNELS:
-            if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
-            L->t1_kernels = value == 1 && qe::decode_t1_supported(L->dims);
+        case MOE_OPT_SINGLE_TOKEN_KERNELS: {
+            if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;
+            int m = (int)value;
+            if (m == 2 && !L->fused_ok) m = 1;
+            if (m == 1 && !qe::decode_t1_supported(L->dims)) m = 0;
+            L->t1_mode = m;
             return MOE_OK;
+        }
         case MOE_OPT_PROGRAMMATIC_LAUNCH:
             if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
             L->dims.pdl = (int)value;
@@ -378,6 +393,7 @@ moe_status moe_layer_debug_read(moe_layer* L, int32_t item, void* dst, int64_t b
         case MOE_DEBUG_ULIST: src = L->ws.ulist; n = 4 * E; break;
         case MOE_DEBUG_CNT: src = L->ws.cnt; n = 4 * E; break;
         case MOE_DEBUG_XSUM: src = L->ws.xsum; n = 8 * T; break;
+        case MOE_DEBUG_TRACE: src = L->ws.trace; n = 8 * (size_t)L->num_sms * qe::kTraceStamps; break;
         default: return MOE_ERR_INVALID_ARG;
     }
     if ((size_t)bytes < n) n = (size_t)bytes;
@@ -391,7 +407,7 @@ moe_status moe_layer_get_option(const moe_layer* L, int32_t option, int64_t* val
     switch (option) {
         case MOE_OPT_PREFILL_MIN_TOKENS: *value = L->prefill_min_tokens; return MOE_OK;
         case MOE_OPT_PREFILL_AVAILABLE: *value = L->plan ? 1 : 0; return MOE_OK;
-        case MOE_OPT_SINGLE_TOKEN_KERNELS: *value = L->t1_kernels ? 1 : 0; return MOE_OK;
+        case MOE_OPT_SINGLE_TOKEN_KERNELS: *value = L->t1_mode; return MOE_OK;
         case MOE_OPT_PROGRAMMATIC_LAUNCH: *value = L->dims.pdl; return MOE_OK;
         default: return MOE_ERR_INVALID_ARG;
     }
@@ -421,7 +437,7 @@ moe_status moe_profile_read(moe_layer* L, int32_t kernel, double* total_ms, int6
 
 const char* moe_kernel_name(int32_t kernel) {
     static const char* names[MOE_KERNEL_COUNT] = {"router_logits", "topk", "bucket", "gateup", "down", "combine",
-                                                  "gather", "gemm_gateup", "gemm_down"};
+                                                  "gather", "gemm_gateup", "gemm_down", "fused"};
     return (kernel >= 0 && kernel < MOE_KERNEL_COUNT) ? names[kernel] : "unknown";
 }
 

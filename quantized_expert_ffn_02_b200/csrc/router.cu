@@ -6,6 +6,7 @@
 // product bf16 * fp32 is exact in fp64, so the only rounding is in the sums and the top-k
 // boundary is decided at fp64 resolution.  Equal keys go to the lower expert index.
 #include "internal.cuh"
+#include "topk.cuh"
 
 namespace qe {
 namespace {
@@ -142,15 +143,7 @@ router_gemm_kernel(const float* __restrict__ wr, const uint16_t* __restrict__ x,
     }
 }
 
-struct KeyIdx {
-    double key;
-    int idx;
-};
-__device__ __forceinline__ bool beats(double ka, int ia, double kb, int ib) {
-    return ka > kb || (ka == kb && ia < ib);
-}
-
-// One warp per token: keys, k rounds of warp arg-max, gate weights.
+// One warp per token: top-k and gate weights.
 // Writes idx[t][r] / w[t][r] in rank order and asc[t][p] = the rank whose expert is the
 // p-th smallest of the token's k experts.
 template <int MAXPER>
@@ -160,67 +153,19 @@ topk_kernel(const double* __restrict__ logits, const float* __restrict__ bias, i
     const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
     const int t = blockIdx.x * (blockDim.x / kWarp) + warp;
     if (t >= T) return;
-    const double* lg = logits + (size_t)t * E;
-    double key[MAXPER];
-    uint32_t taken = 0;
+    double lg[MAXPER];
 #pragma unroll
     for (int m = 0; m < MAXPER; ++m) {
         const int e = lane + kWarp * m;
-        double kv = -INFINITY;
-        if (e < E) {
-            const double l = lg[e];
-            if (router == MOE_ROUTER_SIGMOID_BIAS)
-                kv = 1.0 / (1.0 + exp(-l)) + (bias ? (double)bias[e] : 0.0);
-            else
-                kv = l;
-            if (isnan(kv)) kv = -INFINITY;     // keeps every pick a valid expert index
-        } else {
-            taken |= 1u << m;
-        }
-        key[m] = kv;
+        lg[m] = e < E ? logits[(size_t)t * E + e] : 0.0;
     }
-    int my_e = -1;          // lane r < k ends up holding the rank-r expert
-    for (int r = 0; r < k; ++r) {
-        double bk = -INFINITY;
-        int bi = 0x7fffffff;
-#pragma unroll
-        for (int m = 0; m < MAXPER; ++m) {
-            const int e = lane + kWarp * m;
-            if (!(taken >> m & 1u) && beats(key[m], e, bk, bi)) { bk = key[m]; bi = e; }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const double ok = __shfl_xor_sync(0xffffffffu, bk, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (beats(ok, oi, bk, bi)) { bk = ok; bi = oi; }
-        }
-        if ((bi % kWarp) == lane) taken |= 1u << (bi / kWarp);
-        if (lane == r) my_e = bi;
-    }
-    // gate weights over the chosen k (fp64, rounded once to fp32)
-    const bool mine = lane < k;
-    const double l = mine ? lg[my_e] : 0.0;
-    double num, den;
-    if (router == MOE_ROUTER_SIGMOID_BIAS) {
-        num = mine ? 1.0 / (1.0 + exp(-l)) : 0.0;
-        den = warp_sum_d(num);
-    } else {
-        double m = mine ? l : -INFINITY;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
-        num = mine ? exp(l - m) : 0.0;
-        den = warp_sum_d(num);
-    }
-    // position of this rank in ascending expert order
-    int pos = 0;
-    for (int r2 = 0; r2 < k; ++r2) {
-        const int e2 = __shfl_sync(0xffffffffu, my_e, r2);
-        if (mine && e2 < my_e) ++pos;
-    }
-    if (mine) {
-        idx_out[(size_t)t * k + lane] = my_e;
-        w_out[(size_t)t * k + lane] = (float)((double)scaling * num / den);
-        if (asc_out) asc_out[(size_t)t * k + pos] = lane;
+    float bv[MAXPER];
+    load_bias<MAXPER>(bias, E, lane, bv);
+    const TopkPick p = warp_topk<MAXPER>(lg, bv, E, k, router, scaling, lane);
+    if (lane < k) {
+        idx_out[(size_t)t * k + lane] = p.e;
+        w_out[(size_t)t * k + lane] = p.w;
+        if (asc_out) asc_out[(size_t)t * k + p.pos] = lane;
     }
 }
 
@@ -233,64 +178,23 @@ constexpr int kSmallThreads = 256;
 constexpr int kSmallMaxT = 32;
 constexpr int kSmallMaxE = 1024;
 
+// Selection for one token whose logits other blocks wrote (read through L2).
 template <int MAXPER>
 __device__ void warp_select(const double* __restrict__ lg, const float* __restrict__ bias, int E, int k, int router,
                             float scaling, int lane, int32_t* idx_out, float* w_out, int32_t* asc_out) {
-    double key[MAXPER];
-    uint32_t taken = 0;
+    double l[MAXPER];
 #pragma unroll
     for (int m = 0; m < MAXPER; ++m) {
         const int e = lane + kWarp * m;
-        double kv = -INFINITY;
-        if (e < E) {
-            const double l = __ldcg(lg + e);       // written by other blocks: read through L2
-            kv = router == MOE_ROUTER_SIGMOID_BIAS ? 1.0 / (1.0 + exp(-l)) + (bias ? (double)bias[e] : 0.0) : l;
-            if (isnan(kv)) kv = -INFINITY;
-        } else {
-            taken |= 1u << m;
-        }
-        key[m] = kv;
+        l[m] = e < E ? __ldcg(lg + e) : 0.0;
     }
-    int my_e = -1;
-    for (int r = 0; r < k; ++r) {
-        double bk = -INFINITY;
-        int bi = 0x7fffffff;
-#pragma unroll
-        for (int m = 0; m < MAXPER; ++m) {
-            const int e = lane + kWarp * m;
-            if (!(taken >> m & 1u) && beats(key[m], e, bk, bi)) { bk = key[m]; bi = e; }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const double ok = __shfl_xor_sync(0xffffffffu, bk, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (beats(ok, oi, bk, bi)) { bk = ok; bi = oi; }
-        }
-        if ((bi % kWarp) == lane) taken |= 1u << (bi / kWarp);
-        if (lane == r) my_e = bi;
-    }
-    const bool mine = lane < k;
-    const double l = mine ? __ldcg(lg + my_e) : 0.0;
-    double num, den;
-    if (router == MOE_ROUTER_SIGMOID_BIAS) {
-        num = mine ? 1.0 / (1.0 + exp(-l)) : 0.0;
-        den = warp_sum_d(num);
-    } else {
-        double m = mine ? l : -INFINITY;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
-        num = mine ? exp(l - m) : 0.0;
-        den = warp_sum_d(num);
-    }
-    int pos = 0;
-    for (int r2 = 0; r2 < k; ++r2) {
-        const int e2 = __shfl_sync(0xffffffffu, my_e, r2);
-        if (mine && e2 < my_e) ++pos;
-    }
-    if (mine) {
-        idx_out[lane] = my_e;
-        w_out[lane] = (float)((double)scaling * num / den);
-        asc_out[pos] = lane;
+    float bv[MAXPER];
+    load_bias<MAXPER>(bias, E, lane, bv);
+    const TopkPick p = warp_topk<MAXPER>(l, bv, E, k, router, scaling, lane);
+    if (lane < k) {
+        idx_out[lane] = p.e;
+        w_out[lane] = p.w;
+        asc_out[p.pos] = lane;
     }
 }
 

@@ -111,12 +111,23 @@ def glm():
     layer.close()
 
 
-def test_glm_decode_t1(glm):
-    for t in DECODE_TOKENS:
-        x = _glm_x(1, t)
-        ref = glm["oracle"].forward(x)
-        out = run_forward(glm["layer"], x)
-        check_close(out, ref["out"])
+@pytest.mark.parametrize("mode", [2, 1, 0])
+def test_glm_decode_t1(glm, mode):
+    layer = glm["layer"]
+    assert layer.set_single_token_mode(mode) == mode
+    try:
+        for t in DECODE_TOKENS:
+            x = _glm_x(1, t)
+            ref = glm["oracle"].forward(x)
+            out = run_forward(layer, x)
+            check_close(out, ref["out"])
+            if mode == 2:
+                # the single launch also leaves the routing tables of its one token
+                idx = np.zeros(layer.cfg.top_k, np.int32)
+                layer.debug_read("idx", idx)
+                assert np.array_equal(idx, ref["idx"][0])
+    finally:
+        layer.set_single_token_mode(2)
 
 
 def test_glm_union_t2(glm):
@@ -158,14 +169,14 @@ def test_glm_batch_union_reads_each_expert_once_per_call(glm):
     x = glm["x32"]
     layer = glm["layer"]
     out_b = run_forward(layer, x)
-    for t1, tol in ((False, 1e-5), (True, 1e-4)):
+    for mode, tol in ((0, 1e-5), (1, 1e-4), (2, 1e-4)):
         # the same kernels give nearly the same sums; the single-token kernels add in another order,
         # and an fp16 rounding of h can flip, so their bound is looser (still far inside the spec)
-        layer.set_single_token_kernels(t1)
+        assert layer.set_single_token_mode(mode) == mode
         for i in (0, 7, 31):
             out_1 = run_forward(layer, x[i:i + 1])
             check_close(out_1, out_b[i:i + 1].astype(np.float64), rel_l2=tol, max_rms=10 * tol)
-    layer.set_single_token_kernels(True)
+    layer.set_single_token_mode(2)
 
 
 # ------------------------------------------------------------------------------------------
