@@ -144,6 +144,30 @@ def make_batches(cfg, T, n, seed, token_offset, device):
 
 
 # ------------------------------------------------------------------------------------------
+# replicas (one process per GPU, no data-path collective)
+# ------------------------------------------------------------------------------------------
+
+def replica_token_base(rank: int) -> int:
+    """First token of a rank's own stream: every replica decodes different tokens."""
+    return rank * 1_000_000
+
+
+def slowest_rank_ms(ms: float, dist, device) -> float:
+    """The largest of the ranks' timed-region durations (the job is as slow as its slowest rank)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, steps: int, T: int, max_ms: float) -> float:
+    """Whole-job throughput: the tokens every rank processed over the slowest rank's time."""
+    return world * steps * T / (max_ms / 1e3)
+
+
+# ------------------------------------------------------------------------------------------
 # clocks during the timed region
 # ------------------------------------------------------------------------------------------
 
@@ -358,7 +382,7 @@ def run_ours(a, rank, world, local_rank):
         layer.set_single_token_mode(a.t1_mode)
     # every rank is an independent replica with its own tokens
     n_batches = a.warmup + a.steps if T <= 32 else 4
-    token_base = rank * 1_000_000
+    token_base = replica_token_base(rank)
     xs = make_batches(cfg, T, n_batches, a.seed, token_base, dev)
     out = torch.empty((T, cfg.d), dtype=torch.int16 if cfg.out_bf16 else torch.float32, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -408,11 +432,8 @@ def run_ours(a, rank, world, local_rank):
     prof = layer.profile_read()
     if layer.last_error() != qe.MOE_OK:
         raise RuntimeError("device status after timing: " + qe.status_str(layer.last_error()))
-    if dist:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = world * a.steps * T / (total_ms / 1e3)
+    total_ms = slowest_rank_ms(total_ms, dist, dev)
+    value = job_tokens_per_s(world, a.steps, T, total_ms)
 
     # end to end: host buffers through the C ABI, copies inside the timed region
     xh = [bx(a.warmup + i).cpu().pin_memory() for i in range(min(a.steps, len(xs)))]
@@ -429,11 +450,8 @@ def run_ours(a, rank, world, local_rank):
     t1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = t0.elapsed_time(t1)
-    if dist:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": world * e2e_steps * T / (e2e_ms / 1e3), "unit": "tokens/s",
+    e2e_ms = slowest_rank_ms(e2e_ms, dist, dev)
+    e2e = {"value": job_tokens_per_s(world, e2e_steps, T, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": T * cfg.d * 2, "d2h_bytes_per_step": T * cfg.d * out.element_size()}
 
     # roofline of the dominant kernel (device time measured by the library's event pairs)

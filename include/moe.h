@@ -207,7 +207,8 @@ moe_status moe_layer_get_option(const moe_layer *layer, int32_t option, int64_t 
  *                    at which each CTA passed its phase boundaries: 0 start, 1 x in registers,
  *                    2 router pieces stored, 3 shared rows done, 4 first grid barrier passed,
  *                    5 router pieces gathered, 6 experts selected, 7 routed gate/up done, 8 h
- *                    complete, 9 down done, 10 output stored (11..15 unused)
+ *                    complete, 9 down done, 10 output stored, 11 x in shared memory, 12..15
+ *                    steps of the selection (candidates, ranks, gate weights, proxy fence)
  */
 enum { MOE_DEBUG_H = 0, MOE_DEBUG_Y = 1, MOE_DEBUG_IDX = 2, MOE_DEBUG_W = 3, MOE_DEBUG_ASC = 4,
        MOE_DEBUG_ULIST = 5, MOE_DEBUG_CNT = 6, MOE_DEBUG_XSUM = 7, MOE_DEBUG_TRACE = 8 };

@@ -35,6 +35,19 @@ __device__ __forceinline__ bool bar_try(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// The same test, but the thread may sleep in the instruction (up to about 1 ms) until the phase
+// completes, instead of spinning and taking issue slots from the warps that compute.
+__device__ __forceinline__ bool bar_try_sleep(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(1000000u)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ uint64_t now_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -44,7 +57,7 @@ __device__ __forceinline__ uint64_t now_ns() {
 __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
     if (bar_try(bar, parity)) return true;
     const uint64_t t0 = now_ns();
-    while (!bar_try(bar, parity))
+    while (!bar_try_sleep(bar, parity))
         if (now_ns() - t0 > kWaitLimitNs) return false;
     return true;
 }
@@ -58,6 +71,10 @@ __device__ __forceinline__ uint4 lds16(uint32_t a) {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
     return v;
+}
+
+__device__ __forceinline__ void sts16(uint32_t a, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
 // 8 bf16 of columns 8m..8m+7 -> four registers holding (col i, col i+4), i = 0..3
@@ -87,6 +104,27 @@ __device__ __forceinline__ float dot_word_f16(uint32_t w, const uint32_t* hp, fl
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const uint32_t p = hsub2_u32(lop_sel_xor(w >> (4 * i), kNib, kF16Magic), kF16Magic);
+        unsigned short wl, wh, hl, hh;
+        halves(p, wl, wh);
+        halves(hp[i], hl, hh);
+        acc = fma_f16(wl, hl, acc);
+        acc = fma_f16(wh, hh, acc);
+    }
+    return acc;
+}
+
+// acc += sum over the 8 codes of word w of (3/2 + s/16) * h.  The nibble goes to the top four
+// mantissa bits of an fp16 1.0 (mask 0x03C0 per half), so the pair reads 1 + (n ^ 8) / 16 =
+// 3/2 + s/16 exactly, one shift and one LOP3 per pair and no subtraction.  The caller recovers
+// sum s h = 16 acc - 24 sum h; the offset is small next to the codes, so the cancellation costs
+// only a few units of fp32 rounding.
+constexpr uint32_t kF16TopMask = 0x03C003C0u;
+constexpr uint32_t kF16TopMagic = 0x3E003E00u;   // fp16 1.5 in each half: bit 9 flips the nibble's sign
+__device__ __forceinline__ float dot_word_f16top(uint32_t w, const uint32_t* hp, float acc) {
+    const uint32_t src[4] = {w << 6, w << 2, w >> 2, w >> 6};   // nibble pair i -> bits 6..9, 22..25
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t p = lop_sel_xor(src[i], kF16TopMask, kF16TopMagic);
         unsigned short wl, wh, hl, hh;
         halves(p, wl, wh);
         halves(hp[i], hl, hh);

@@ -113,6 +113,7 @@ struct Workspace {
     uint16_t* xg;          // [slots][d] bf16: x gathered per slot, K order permuted in groups of 8
     int32_t* groups;       // [max_groups][4]: (expert or -1, first slot, tokens, unused)
     int32_t* n_groups;     // [2]: routed groups, shared groups
+    float* xsum_slot;      // [slots]: sum of x of each slot's token (gate/up GEMM epilogue)
     uint32_t* counter;     // [1]: blocks done in the fused small-batch router (reset to 0 by the last)
     // single-launch decode path
     double* rpart;         // [E][d / 1024]: pieces of the router logits

@@ -136,6 +136,7 @@ size_t carve(const moe_config& c, size_t max_groups, char* base, qe::Workspace* 
         w.xg = (uint16_t*)take(sizeof(uint16_t) * slots * (size_t)c.d);
         w.groups = (int32_t*)take(sizeof(int32_t) * 4 * max_groups);
         w.n_groups = (int32_t*)take(sizeof(int32_t) * 2);
+        w.xsum_slot = (float*)take(sizeof(float) * slots);
     }
     uint16_t* xs = (uint16_t*)take(sizeof(uint16_t) * T * (size_t)c.d);
     void* os = (void*)take(sizeof(float) * T * (size_t)c.d);

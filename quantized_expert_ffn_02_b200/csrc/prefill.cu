@@ -173,22 +173,29 @@ __device__ __forceinline__ uint32_t idesc_f16(int n, bool bf16) {
     return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
-// 8 int4 codes of one word -> four registers holding the exact codes of columns (i, i+4) as a
-// pair of 16-bit floats: magic | (nibble ^ 8) is 136 + s (bf16) or 1032 + s (fp16), then one
-// packed subtraction of the magic leaves s.
+// 8 int4 codes of one word -> four registers holding the codes of columns (i, i+4) as a pair of
+// 16-bit floats.
+//   GEMM-1 (bf16): the nibble goes to the top four mantissa bits of a bf16 1.0, so the pair reads
+//     1 + (n ^ 8) / 16 = 3/2 + s/16 exactly (one shift and one LOP3 per pair); the epilogue takes
+//     sum s x = 16 D - 24 sum x back out of the accumulator D, with sum x per slot from the gather.
+//   GEMM-2 (fp16): magic | (nibble ^ 8) is 1032 + s, and one packed subtraction of the magic leaves
+//     s exactly.
 template <bool BF16>
 __device__ __forceinline__ void unpack_word(uint32_t w, uint32_t* out) {
-    constexpr uint32_t kMask = 0x000F000Fu;
-    constexpr uint32_t kMagic = BF16 ? 0x43084308u : 0x64086408u;
+    if (BF16) {
+        const uint32_t src[4] = {w << 3, w >> 1, w >> 5, w >> 9};   // nibble pair i -> bits 3..6, 19..22
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t p = lop_sel_xor(w >> (4 * i), kMask, kMagic);
-        uint32_t s;
-        if (BF16)
-            asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(s) : "r"(p), "r"(kMagic));
-        else
+        for (int i = 0; i < 4; ++i) out[i] = lop_sel_xor(src[i], 0x00780078u, 0x3FC03FC0u);
+    } else {
+        constexpr uint32_t kMask = 0x000F000Fu;
+        constexpr uint32_t kMagic = 0x64086408u;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t p = lop_sel_xor(w >> (4 * i), kMask, kMagic);
+            uint32_t s;
             asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(s) : "r"(p), "r"(kMagic));
-        out[i] = s;
+            out[i] = s;
+        }
     }
 }
 
@@ -220,6 +227,7 @@ struct GemmArgs {
     int ld_out;               // h row stride (fmax) or Y row stride (d)
     void* out;                // h (fp16 bits) or Y (fp32)
     int* status;
+    const float* xsum_slot;   // gate/up: sum of x of each slot's token
 };
 
 template <bool GATED>
@@ -441,8 +449,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     const int n = c0 + i;
                     if (n < tl.n) {
                         if (GATED) {
-                            const float g = s0 * __uint_as_float(v0[i]);
-                            const float u = s1 * __uint_as_float(v1[i]);
+                            const float xs24 = 24.0f * __ldg(args.xsum_slot + tl.slot0 + n);
+                            const float g = s0 * fmaf(16.0f, __uint_as_float(v0[i]), -xs24);
+                            const float u = s1 * fmaf(16.0f, __uint_as_float(v1[i]), -xs24);
                             const float hv = g / (1.0f + expf(-g)) * u;
                             const __half hh = __float2half_rn(hv);
                             if (!isfinite(__half2float(hh)) && isfinite(hv)) latch_status(status, MOE_ERR_RANGE);
@@ -479,8 +488,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 // gather: xg[slot] = x[token of slot] with K permuted within groups of 8 as [0,4,1,5,2,6,3,7]
 // ---------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
-gather_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int T, int k, int S, int d,
-              uint16_t* __restrict__ xg) {
+gather_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, const double* __restrict__ xsum,
+              int T, int k, int S, int d, uint16_t* __restrict__ xg, float* __restrict__ xsum_slot) {
     const int per_row = d / 8;
     const size_t total = (size_t)T * (k + S) * per_row;
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
@@ -493,6 +502,7 @@ gather_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, 
         o.z = __byte_perm(v.y, v.w, 0x5410);
         o.w = __byte_perm(v.y, v.w, 0x7632);
         reinterpret_cast<uint4*>(xg + (size_t)slot * d)[c] = o;
+        if (c == 0) xsum_slot[slot] = (float)xsum[t];
     }
 }
 
@@ -638,13 +648,13 @@ cudaError_t launch_prefill_experts(const LayerDims& L, const PrefillPlan* p, con
     const size_t work = (size_t)T * (L.k + L.S) * (L.d / 8);
     const unsigned gg = (unsigned)std::min<size_t>((work + 255) / 256, (size_t)num_sms * 16);
     QE_LAUNCH(ctx, MOE_KERNEL_GATHER,
-              (gather_kernel<<<gg, 256, 0, ctx.s>>>(x, ws.perm, T, L.k, L.S, L.d, ws.xg)));
+              (gather_kernel<<<gg, 256, 0, ctx.s>>>(x, ws.perm, ws.xsum, T, L.k, L.S, L.d, ws.xg, ws.xsum_slot)));
     GemmArgs a1{groups, ws.n_groups, W.gate_up_scale, W.shared_gate_up_scale, 2 * L.f, L.f, L.S ? L.f_shared : L.f,
-                L.f / BM, L.S ? L.f_shared / BM : 1, L.d, L.d, fmax, ws.h, ws.status};
+                L.f / BM, L.S ? L.f_shared / BM : 1, L.d, L.d, fmax, ws.h, ws.status, ws.xsum_slot};
     QE_LAUNCH(ctx, MOE_KERNEL_GEMM_GATEUP,
               (gemm_kernel<true><<<num_sms, kGemmThreads, gemm_smem_bytes(true), ctx.s>>>(p->a1, p->a1_sh, p->b1, a1)));
     GemmArgs a2{groups, ws.n_groups, W.down_scale, W.shared_down_scale, L.d, L.f, L.S ? L.f_shared : L.f,
-                L.d / BM, L.d / BM, L.f, L.S ? L.f_shared : L.f, L.d, ws.Y, ws.status};
+                L.d / BM, L.d / BM, L.f, L.S ? L.f_shared : L.f, L.d, ws.Y, ws.status, nullptr};
     QE_LAUNCH(ctx, MOE_KERNEL_GEMM_DOWN,
               (gemm_kernel<false><<<num_sms, kGemmThreads, gemm_smem_bytes(false), ctx.s>>>(p->a2, p->a2_sh, p->b2, a2)));
     return cudaSuccess;
