@@ -42,8 +42,8 @@ namespace {
 
 using namespace dec;
 
-constexpr int kFzMaxWarps = 12;
-constexpr int kFzStages = 3;
+constexpr int kFzMaxWarps = 16;
+constexpr int kFzStages = 2;
 constexpr int kFzMaxSlots = 10;       // k routed experts + the shared one
 constexpr int kFzMaxPer = 8;          // experts per lane in the selection: E <= 256
 constexpr int kFzRowsMax = 64;        // output rows per CTA
@@ -229,8 +229,8 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
-    // x (2d bytes) into the stage-2 region, once per CTA
-    const uint32_t xraw_s = st_s(2) - (uint32_t)warp * stage_bytes;   // stage 2 of warp 0
+    // x (2d bytes) into the last stage's region, once per CTA
+    const uint32_t xraw_s = st_s(kFzStages - 1) - (uint32_t)warp * stage_bytes;
     if (tid == 0) {
         bar_expect_tx(saddr(&s_xbar), 2u * d);
         bulk_g2s(xraw_s, a.x, 2u * d, saddr(&s_xbar));
@@ -334,8 +334,8 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
     const float my_bias = a.bias && tid < E ? a.bias[tid] : 0.0f;
     __syncthreads();                                       // x is pre-paired
     stamp(1);
-    // the shared expert's rows need no routing: queue them now (stages 0 and 1; stage 2 keeps x in
-    // plain order for the router pieces)
+    // the shared expert's rows need no routing: queue them now (all stages but the last, which
+    // keeps x in plain order for the router pieces)
     if (lane == 0)
         while (issued < my_sh && issued < kFzStages - 1) issue(issued++);
     // the shared expert's down rows of this CTA are read last: start pulling them into L2
@@ -352,7 +352,7 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
         const double v = warp_sum_d(router_piece(rw, xraw_s + 2048u * p, lane));
         if (lane == 0) __stcg(a.rpart + u, v);
     }
-    __syncthreads();                                       // stage 2 is free
+    __syncthreads();                                       // the last stage is free
     if (tid == 0) {                                        // barrier 0: every piece is stored
         const unsigned long long old = arrive(a.bar);
         s_base = old - old % (2ull * G);
