@@ -67,19 +67,24 @@ router_logits_kernel(const float* __restrict__ wr, const uint16_t* __restrict__ 
 }
 
 // ---------------------------------------------------------------------------------------
-// Large batches: logits = X Wr^T as a tiled fp64 GEMM.  A CTA computes 64 tokens x 64 experts;
-// every x and w element is converted to fp64 once per tile (into shared memory) and each thread
-// keeps a 4 x 4 register tile.  The next K chunk's global loads are in flight while the current
-// chunk is multiplied.  CTAs of the first expert tile also write sum_i x[t][i].
+// Large batches: logits = X Wr^T as a tiled fp64 GEMM on the fp64 tensor cores (mma.sync
+// m8n8k4.f64: the only tensor-core form with fp64 operands and accumulator).  A CTA computes
+// 64 tokens x 64 experts; every x and w element is converted to fp64 once per tile (into shared
+// memory, K-major, rows padded to 68 so that a fragment load meets no bank conflict); warp
+// (wm, wn) of the 2 x 4 warp grid owns 32 tokens x 16 experts, i.e. 4 x 2 tiles of 8 x 8.  The
+// next K chunk's global loads are in flight while the current chunk is multiplied.  CTAs of the
+// first expert tile also write sum_i x[t][i].
 // ---------------------------------------------------------------------------------------
 constexpr int kRgT = 64, kRgE = 64, kRgK = 32, kRgThreads = 256;
 
 __global__ void __launch_bounds__(kRgThreads)
 router_gemm_kernel(const float* __restrict__ wr, const uint16_t* __restrict__ x, int T, int d, int E,
                    double* __restrict__ logits, double* __restrict__ xsum) {
-    __shared__ double xs[kRgK][kRgT + 1];
-    __shared__ double ws[kRgK][kRgE + 1];
-    const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+    __shared__ double xs[kRgK][kRgT + 4];
+    __shared__ double ws[kRgK][kRgE + 4];
+    const int tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
+    const int wm = warp / 4, wn = warp % 4;                // 32 tokens x 16 experts per warp
+    const int g = lane / 4, tq = lane % 4;                 // fragment row / column group
     const int t0 = blockIdx.x * kRgT, e0 = blockIdx.y * kRgE;
     // loader roles: 4 threads per token row (8 bf16 each) and per expert row (8 fp32 each)
     const int lr = tid / 4, lc = (tid % 4) * 8;
@@ -89,11 +94,11 @@ router_gemm_kernel(const float* __restrict__ wr, const uint16_t* __restrict__ x,
     const float* wrow = wr + (size_t)(e0 + lr) * d + lc;
     uint4 xv = xrow_ok ? ld_ro16(xrow) : make_uint4(0, 0, 0, 0);
     float4 wa = __ldg(reinterpret_cast<const float4*>(wrow)), wb = __ldg(reinterpret_cast<const float4*>(wrow) + 1);
-    double acc[4][4];
+    double acc[4][2][2];                                   // [token tile][expert tile][c0, c1]
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+        for (int j = 0; j < 2; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
     double xpart = 0.0;
     for (int k0 = 0; k0 < d; k0 += kRgK) {
         // convert the staged chunk into shared memory (K-major)
@@ -115,26 +120,35 @@ router_gemm_kernel(const float* __restrict__ wr, const uint16_t* __restrict__ x,
             wa = __ldg(reinterpret_cast<const float4*>(wrow + k0 + kRgK));
             wb = __ldg(reinterpret_cast<const float4*>(wrow + k0 + kRgK) + 1);
         }
-#pragma unroll 8
-        for (int kk = 0; kk < kRgK; ++kk) {
-            double a[4], b[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = xs[kk][4 * ty + i];
+        for (int kk = 0; kk < kRgK; kk += 4) {
+            // A fragment (8 x 4, row-major): lane (g, tq) holds A[g][tq]; B (4 x 8, column-major):
+            // B[tq][g]; C (8 x 8): C[g][2 tq], C[g][2 tq + 1]
+            double a[4], b[2];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) b[j] = ws[kk][4 * tx + j];
+            for (int i = 0; i < 4; ++i) a[i] = xs[kk + tq][32 * wm + 8 * i + g];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) b[j] = ws[kk + tq][16 * wn + 8 * j + g];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+                for (int j = 0; j < 2; ++j)
+                    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+                                 : "+d"(acc[i][j][0]), "+d"(acc[i][j][1])
+                                 : "d"(a[i]), "d"(b[j]));
         }
         __syncthreads();
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int t = t0 + 4 * ty + i;
+        const int t = t0 + 32 * wm + 8 * i + g;
         if (t < T)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) logits[(size_t)t * E + e0 + 4 * tx + j] = acc[i][j];
+            for (int j = 0; j < 2; ++j) {
+                const int e = e0 + 16 * wn + 8 * j + 2 * tq;
+                logits[(size_t)t * E + e] = acc[i][j][0];
+                logits[(size_t)t * E + e + 1] = acc[i][j][1];
+            }
     }
     if (sum_x) {     // the 4 loader threads of a token are adjacent lanes
         xpart += __shfl_xor_sync(0xffffffffu, xpart, 1);
