@@ -25,9 +25,12 @@
 // on the order of its terms.
 //
 // Roles (192 threads, one CTA per SM, persistent over tiles):
-//   warp 0    TMA producer (packed A rows, B tile)              smem ring of kStages
+//   warp 0    TMA producer of the packed A rows                 smem ring of 128 KB (16 or 32 stages)
+//   warp 10   TMA producer of the B tiles                       smem ring of kBStages
 //   warp 1    TMEM allocator and MMA issuer                      TMEM A ring of kAStages
-//   warps 2-5 converters (A rows -> TMEM), then the epilogue     thread <-> TMEM lane
+//   warps 2-9 converters (A rows -> TMEM), then the epilogue     thread <-> TMEM lane; two sets
+//             of four (one warp per TMEM lane quarter each) take alternate K steps and alternate
+//             16-column blocks of the epilogue
 // Every wait is bounded (about 2 s); on expiry the CTA latches MOE_ERR_TIMEOUT, drains what it
 // issued, frees its TMEM and returns.
 #include "internal.cuh"
@@ -50,9 +53,11 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN = 128;
 constexpr int BK = 64;
-constexpr int kStages = 6;
-constexpr int kAStages = 4;
-constexpr int kGemmThreads = 192;
+constexpr int kBStages = 4;                           // B tiles (x or h, from L2) in shared memory
+constexpr uint32_t kASmBytes = 128 * 1024;            // packed A tiles (from HBM) in shared memory
+constexpr int kASmStagesMax = 32;
+constexpr int kAStages = 4;                           // converted A tiles in TMEM
+constexpr int kGemmThreads = 352;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kPackedTile = BM * BK / 2;         // 4 KB of packed int4 per 128 x 64 tile
 constexpr uint32_t kBTile = BN * BK * 2;              // 16 KB of bf16 / fp16
@@ -275,44 +280,55 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA_sh,
             const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
     constexpr int NA = GATED ? 2 : 1;                     // A tiles per stage
-    constexpr uint32_t kStageBytes = NA * kPackedTile + kBTile;
+    // The packed weights stream from HBM and need many bytes in flight; B comes from L2.  So A and
+    // B have rings of their own, A's much deeper.
+    constexpr int kSA = (int)(kASmBytes / (NA * kPackedTile));   // A stages: 16 (gate/up) or 32
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned working area: B tiles first (swizzle atoms), then packed A tiles
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (base - raw);
-    const uint32_t sB = base;                             // kStages x 16 KB
-    const uint32_t sA = base + kStages * kBTile;          // kStages x NA x 4 KB
-    uint8_t* gA = gbase + kStages * kBTile;
-    __shared__ __align__(8) uint64_t bars[2 * kStages + 2 * kAStages + 3];
+    const uint32_t sB = base;                             // kBStages x 16 KB
+    const uint32_t sA = base + kBStages * kBTile;         // kSA x NA x 4 KB
+    uint8_t* gA = gbase + kBStages * kBTile;
+    __shared__ __align__(8) uint64_t bars[2 * kASmStagesMax + 2 * kBStages + 2 * kAStages + 3];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
-    __shared__ int consumed_sh[4];
-    __shared__ int issued_sh;
+    __shared__ int consumed_sh[8];                        // A stages consumed by each converter warp
+    __shared__ int issued_sh;                             // A stages issued
+    __shared__ int b_issued_sh, b_consumed_sh;
     const uint32_t bar0 = smem_u32(bars);
-    auto full_bar = [&](int s) { return bar0 + 8u * s; };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
-    auto afull_bar = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
-    auto aempty_bar = [&](int s) { return bar0 + 8u * (2 * kStages + kAStages + s); };
-    const uint32_t accfull_bar = bar0 + 8u * (2 * kStages + 2 * kAStages);
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };                       // A landed (smem)
+    auto empty_bar = [&](int s) { return bar0 + 8u * (kSA + s); };              // A converted
+    auto bfull_bar = [&](int s) { return bar0 + 8u * (2 * kSA + s); };          // B landed
+    auto bempty_bar = [&](int s) { return bar0 + 8u * (2 * kSA + kBStages + s); };   // B consumed
+    auto afull_bar = [&](int s) { return bar0 + 8u * (2 * kSA + 2 * kBStages + s); };  // A in TMEM
+    auto aempty_bar = [&](int s) { return bar0 + 8u * (2 * kSA + 2 * kBStages + kAStages + s); };
+    const uint32_t accfull_bar = bar0 + 8u * (2 * kSA + 2 * kBStages + 2 * kAStages);
     const uint32_t accempty_bar = accfull_bar + 8u;
     const uint32_t final_bar = accfull_bar + 16u;
 
     const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kSA; ++s) {
             mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), 1 + 4);
+            mbar_init(empty_bar(s), 4);
+        }
+        for (int s = 0; s < kBStages; ++s) {
+            mbar_init(bfull_bar(s), 1);
+            mbar_init(bempty_bar(s), 1);
         }
         for (int s = 0; s < kAStages; ++s) {
             mbar_init(afull_bar(s), 4);
             mbar_init(aempty_bar(s), 1);
         }
         mbar_init(accfull_bar, 1);
-        mbar_init(accempty_bar, 4);
+        mbar_init(accempty_bar, 8);
         mbar_init(final_bar, 1);
         abort_flag = 0;
         issued_sh = 0;
+        b_issued_sh = 0;
+        b_consumed_sh = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -344,13 +360,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 const Tile tl = decode_tile<GATED>(args, t, nr);
                 const CUtensorMap* mapA = tl.shared ? &tmA_sh : &tmA;
                 for (int kk = 0; kk < tl.ksteps; ++kk, ++ks) {
-                    const int s = ks % kStages;
-                    if (!(ok = wait_bar(empty_bar(s), ((ks / kStages) & 1) ^ 1, abortp, status))) break;
-                    mbar_expect_tx(full_bar(s), kStageBytes);
+                    const int s = ks % kSA;
+                    if (!(ok = wait_bar(empty_bar(s), ((ks / kSA) & 1) ^ 1, abortp, status))) break;
+                    mbar_expect_tx(full_bar(s), NA * kPackedTile);
                     tma_load_2d(sA + s * NA * kPackedTile, mapA, full_bar(s), kk * (BK / 2), tl.a_row0);
                     if (GATED) tma_load_2d(sA + s * NA * kPackedTile + kPackedTile, mapA, full_bar(s), kk * (BK / 2),
                                            tl.a_row1);
-                    tma_load_2d(sB + s * kBTile, &tmB, full_bar(s), kk * BK, tl.slot0);
                 }
             }
             issued_sh = ks;
@@ -367,8 +382,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 if (!(ok = wait_bar(accempty_bar, (tc & 1) ^ 1, abortp, status))) break;
                 tc_fence_after();
                 for (int kk = 0; kk < tl.ksteps; ++kk, ++ks) {
-                    const int s = ks % kStages, sa = ks % kAStages;
-                    if (!(ok = wait_bar(full_bar(s), (ks / kStages) & 1, abortp, status))) break;
+                    const int s = ks % kBStages, sa = ks % kAStages;
+                    if (!(ok = wait_bar(bfull_bar(s), (ks / kBStages) & 1, abortp, status))) break;
                     if (!(ok = wait_bar(afull_bar(sa), (ks / kAStages) & 1, abortp, status))) break;
                     tc_fence_after();
                     const uint64_t bdesc = sw128_desc(sB + s * kBTile);
@@ -379,19 +394,38 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                         mma_f16(acc0, a0 + 8 * j, bdesc + 2 * j, idesc, acc);
                         if (GATED) mma_f16(acc1, a0 + BK / 2 + 8 * j, bdesc + 2 * j, idesc, acc);
                     }
-                    mma_commit(empty_bar(s));
+                    mma_commit(bempty_bar(s));
                     mma_commit(aempty_bar(sa));
                 }
                 if (ok) mma_commit(accfull_bar);
             }
+            b_consumed_sh = ks;
             // drain: every MMA issued so far completes before TMEM is released
             mma_commit(final_bar);
             wait_bar_drain(final_bar, 0);
         }
         __syncwarp();
+    } else if (warp == 10) {
+        // ------------------------------------------------------------------ TMA producer of B
+        if (lane == 0) {
+            int ks = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+                const Tile tl = decode_tile<GATED>(args, t, nr);
+                for (int kk = 0; kk < tl.ksteps; ++kk, ++ks) {
+                    const int s = ks % kBStages;
+                    if (!(ok = wait_bar(bempty_bar(s), ((ks / kBStages) & 1) ^ 1, abortp, status))) break;
+                    mbar_expect_tx(bfull_bar(s), kBTile);
+                    tma_load_2d(sB + s * kBTile, &tmB, bfull_bar(s), kk * BK, tl.slot0);
+                }
+            }
+            b_issued_sh = ks;
+        }
+        __syncwarp();
     } else {
         // ------------------------------------------------------------------ converters + epilogue
         const int q = warp & 3;                            // TMEM lane quarter of this warp
+        const int set = (warp - 2) / 4;                    // K steps with ks % 2 == set
         const int r = 32 * q + lane;                       // tile row owned by this thread
         const uint32_t lane_off = (uint32_t)(32 * q) << 16;
         int ks = 0, tc = 0;
@@ -399,8 +433,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tc) {
             const Tile tl = decode_tile<GATED>(args, t, nr);
             for (int kk = 0; kk < tl.ksteps; ++kk, ++ks) {
-                const int s = ks % kStages, sa = ks % kAStages;
-                ok = wait_bar(full_bar(s), (ks / kStages) & 1, abortp, status);
+                if ((ks & 1) != set) continue;
+                const int s = ks % kSA, sa = ks % kAStages;
+                ok = wait_bar(full_bar(s), (ks / kSA) & 1, abortp, status);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 // packed rows, 32-byte swizzle: the 16-byte halves of rows with bit 2 set are swapped
@@ -439,7 +474,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             const int nmma = (tl.n + 15) & ~15;
             const float s0 = __ldg(tl.sc0 + r);
             const float s1 = GATED ? __ldg(tl.sc1 + r) : 0.0f;
-            for (int c0 = 0; c0 < nmma; c0 += 16) {
+            for (int c0 = 16 * set; c0 < nmma; c0 += 32) {
                 uint32_t v0[16], v1[16];
                 tmem_ld16(acc0 + c0 + lane_off, v0);
                 if (GATED) tmem_ld16(acc1 + c0 + lane_off, v1);
@@ -468,15 +503,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             __syncwarp();
             if (lane == 0) mbar_arrive(accempty_bar);
         }
-        if (lane == 0) consumed_sh[q] = ks;
+        if (lane == 0) consumed_sh[warp - 2] = ks;
     }
 
     __syncthreads();
     // drain TMA copies that were issued but not consumed (only after an abort)
     if (warp == 0 && lane == 0) {
         int consumed = consumed_sh[0];
-        for (int i = 1; i < 4; ++i) consumed = min(consumed, consumed_sh[i]);
-        for (int k2 = consumed; k2 < issued_sh; ++k2) wait_bar_drain(full_bar(k2 % kStages), (k2 / kStages) & 1);
+        for (int i = 1; i < 8; ++i) consumed = min(consumed, consumed_sh[i]);
+        for (int k2 = consumed; k2 < issued_sh; ++k2) wait_bar_drain(full_bar(k2 % kSA), (k2 / kSA) & 1);
+        for (int k2 = b_consumed_sh; k2 < b_issued_sh; ++k2)
+            wait_bar_drain(bfull_bar(k2 % kBStages), (k2 / kBStages) & 1);
     }
     tc_fence_before();
     __syncthreads();
@@ -550,7 +587,8 @@ schedule_kernel(const int32_t* __restrict__ cnt, const int32_t* __restrict__ off
 }
 
 size_t gemm_smem_bytes(bool gated) {
-    return 1024 + (size_t)kStages * (kBTile + (gated ? 2 : 1) * kPackedTile);
+    (void)gated;
+    return 1024 + (size_t)kBStages * kBTile + kASmBytes;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
