@@ -63,6 +63,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's tokens per step (smaller cases for profiling)")
     ap.add_argument("--t1-mode", type=int, default=None, choices=[0, 1, 2],
                     help="single-token path: 2 one launch, 1 three kernels, 0 general kernels (default: the library's)")
     ap.add_argument("--experts", type=int, default=None,
@@ -370,6 +372,8 @@ def run_ours(a, rank, world, local_rank):
     cfg = syn.CONFIGS[a.workload]
     if a.experts:
         cfg = dataclasses.replace(cfg, E=a.experts)
+    if a.tokens:
+        cfg = dataclasses.replace(cfg, T=a.tokens)
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     dist = None

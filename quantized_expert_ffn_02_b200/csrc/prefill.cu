@@ -65,6 +65,12 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;      // 2 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
+__device__ __forceinline__ uint4 lds_v4(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
 }
@@ -287,10 +293,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     // 1024-byte aligned working area: B tiles first (swizzle atoms), then packed A tiles
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
-    uint8_t* gbase = smem_raw + (base - raw);
     const uint32_t sB = base;                             // kBStages x 16 KB
     const uint32_t sA = base + kBStages * kBTile;         // kSA x NA x 4 KB
-    uint8_t* gA = gbase + kBStages * kBTile;
     __shared__ __align__(8) uint64_t bars[2 * kASmStagesMax + 2 * kBStages + 2 * kAStages + 3];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
@@ -443,9 +447,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 uint32_t regs[32];
 #pragma unroll
                 for (int a = 0; a < NA; ++a) {
-                    const uint8_t* rowp = gA + (size_t)s * NA * kPackedTile + a * kPackedTile + r * 32;
-                    const uint4 lo = *reinterpret_cast<const uint4*>(rowp + 16 * sw);
-                    const uint4 hi = *reinterpret_cast<const uint4*>(rowp + 16 * (sw ^ 1));
+                    // explicit shared-memory loads (a generic load waits on the long scoreboard)
+                    const uint32_t rowp = sA + (uint32_t)(s * NA + a) * kPackedTile + (uint32_t)r * 32u;
+                    const uint4 lo = lds_v4(rowp + 16u * sw);
+                    const uint4 hi = lds_v4(rowp + 16u * (sw ^ 1));
                     const uint32_t words[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
                     if (a == 0) {
                         ok = wait_bar(aempty_bar(sa), ((ks / kAStages) & 1) ^ 1, abortp, status);
