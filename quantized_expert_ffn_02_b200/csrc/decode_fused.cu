@@ -302,15 +302,21 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
                 bar_wait(saddr(&bars[warp][q % kFzStages]), (uint32_t)(q / kFzStages) & 1u);
     };
 
-    // ---- A: x (one bulk copy per CTA) first, then this warp's first router piece, both ahead of
-    //      the stream of expert rows, so that the router's inputs are not queued behind it
+    // ---- A: x (one bulk copy per CTA) and this warp's first router piece, both ahead of the
+    //      stream of expert rows, so that the router's inputs are not queued behind it
     const int n_units = E * nch;
+    // this warp's first router piece: its loads (coalesced, 512 bytes per instruction) are in
+    // flight while x lands and is rearranged
+    float4 rw[8];
+    if (gw < n_units) {
+        const int e = gw / nch, p = gw - e * nch;
+        load_router_piece(a.router_w + (size_t)e * d + 1024 * p, lane, rw);
+    }
     bool ok = __all_sync(0xffffffffu, bar_wait(saddr(&s_xbar), 0u));
     stamp(11);
     // x pre-paired into its own region (group g = columns 8g .. 8g + 7 goes to row g % 4 of chunk
     // g / 4), and the sum of x: thread i adds groups i, i + threads, ... (fp32), each warp's
-    // total goes to shared memory (fp64).  This runs before any other load is issued: shared
-    // memory traffic queued behind a burst of global loads would wait for them.
+    // total goes to shared memory (fp64).
     {
         float xsl = 0.0f;
         for (int g = tid; g < d / 8; g += blockDim.x) {
@@ -325,12 +331,7 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
         const double wsum = warp_sum_d((double)xsl);
         if (lane == 0) s_xpart[warp] = wsum;
     }
-    // this warp's first router piece and this thread's selection bias
-    float4 rw[8];
-    if (gw < n_units) {
-        const int e = gw / nch, p = gw - e * nch;
-        load_router_piece(a.router_w + (size_t)e * d + 1024 * p, lane, rw);
-    }
+    // this thread's selection bias
     const float my_bias = a.bias && tid < E ? a.bias[tid] : 0.0f;
     __syncthreads();                                       // x is pre-paired
     stamp(1);
