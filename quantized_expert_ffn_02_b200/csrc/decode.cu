@@ -391,11 +391,14 @@ cudaError_t launch_experts_t(const LayerDims& L, const moe_weights& W, const uin
 cudaError_t launch_decode_experts(const LayerDims& L, const moe_weights& W, const uint16_t* x, int T,
                                   const Workspace& ws, int num_sms, const Launch& ctx) {
     if (T == 0) return cudaSuccess;
+    // Tokens per pass over a row: small groups keep the register count low enough for two CTAs
+    // per SM (more loads in flight); a bucket larger than the group takes more passes over rows
+    // that are then in L2.  Batch-union decode buckets hold one or two tokens almost always.
     if (L.wkind == MOE_W_INT4_ROWSCALE)
-        return T == 1 ? launch_experts_t<MOE_W_INT4_ROWSCALE, 1>(L, W, x, T, ws, num_sms, ctx)
-                      : launch_experts_t<MOE_W_INT4_ROWSCALE, 4>(L, W, x, T, ws, num_sms, ctx);
-    return T == 1 ? launch_experts_t<MOE_W_BF16, 1>(L, W, x, T, ws, num_sms, ctx)
-                  : launch_experts_t<MOE_W_BF16, 4>(L, W, x, T, ws, num_sms, ctx);
+        return T <= 4 ? launch_experts_t<MOE_W_INT4_ROWSCALE, 1>(L, W, x, T, ws, num_sms, ctx)
+                      : launch_experts_t<MOE_W_INT4_ROWSCALE, 2>(L, W, x, T, ws, num_sms, ctx);
+    return T <= 4 ? launch_experts_t<MOE_W_BF16, 1>(L, W, x, T, ws, num_sms, ctx)
+                  : launch_experts_t<MOE_W_BF16, 2>(L, W, x, T, ws, num_sms, ctx);
 }
 
 cudaError_t launch_combine(const LayerDims& L, int T, const Workspace& ws, void* out, const Launch& ctx) {
