@@ -295,8 +295,10 @@ def kernel_work(cfg, T, n_unique):
     # the single launch (T = 1): router matrix and bias, x, every expert byte, h written and read
     # back, the output
     fused = cfg.E * cfg.d * 4 + cfg.E * 4 + gu + dn_w + slots * fmax * 2 + cfg.d * 4
+    # router kernels: the fp32 router matrix and x read, fp64 logits written
+    router = cfg.E * cfg.d * 4 + T * cfg.d * 2 + T * cfg.E * 8
     return {"gateup": ("hbm", gu), "down": ("hbm", dn), "gemm_gateup": ("tensor", 4 * mac),
-            "gemm_down": ("tensor", 2 * mac), "fused": ("hbm", fused)}
+            "gemm_down": ("tensor", 2 * mac), "fused": ("hbm", fused), "router_logits": ("hbm", router)}
 
 
 def source_sha(paths):

@@ -61,7 +61,7 @@ __device__ __forceinline__ void member(const Slots& b, int j, const int32_t* per
 // gate/up + SiLU
 // ---------------------------------------------------------------------------------------
 template <int WK, int TG>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 gateup_kernel(const uint8_t* __restrict__ gate_up, const float* __restrict__ gu_scale,
               const uint8_t* __restrict__ sh_gate_up, const float* __restrict__ sh_gu_scale,
               const uint16_t* __restrict__ x, const double* __restrict__ xsum, int T, int k, int d, int f,
@@ -114,12 +114,26 @@ gateup_kernel(const uint8_t* __restrict__ gate_up, const float* __restrict__ gu_
 #pragma unroll
                 for (int j = 0; j < TG; ++j) acc[rr][j] = 0.0f;
 
-            for (int c = lane; c < nchunk; c += kWarp) {
-                uint4 wv[2 * R];
+            // the next chunk's rows are in flight while this chunk is multiplied
+            uint4 wn[2 * R];
+            auto load_rows = [&](int c, uint4 (&dst)[2 * R]) {
 #pragma unroll
                 for (int rr = 0; rr < 2 * R; ++rr) {
                     const int row = rr < R ? r0 + rr : fe + r0 + (rr - R);
-                    wv[rr] = ld_stream16(W + (size_t)row * rowbytes + (size_t)c * 16);
+                    dst[rr] = ld_stream16(W + (size_t)row * rowbytes + (size_t)c * 16);
+                }
+            };
+            // (one-token passes only: with more tokens per pass the registers run out)
+            constexpr bool kAhead = TG == 1;
+            if (kAhead && lane < nchunk) load_rows(lane, wn);
+            for (int c = lane; c < nchunk; c += kWarp) {
+                uint4 wv[2 * R];
+                if (kAhead) {
+#pragma unroll
+                    for (int rr = 0; rr < 2 * R; ++rr) wv[rr] = wn[rr];
+                    if (c + kWarp < nchunk) load_rows(c + kWarp, wn);
+                } else {
+                    load_rows(c, wv);
                 }
 #pragma unroll
                 for (int j = 0; j < TG; ++j) {
@@ -206,7 +220,7 @@ gateup_kernel(const uint8_t* __restrict__ gate_up, const float* __restrict__ gu_
 // down: Y[slot][j] = scale[j] * sum_r q[j][r] h[slot][r]
 // ---------------------------------------------------------------------------------------
 template <int WK, int TG>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 down_kernel(const uint8_t* __restrict__ down, const float* __restrict__ dn_scale,
             const uint8_t* __restrict__ sh_down, const float* __restrict__ sh_dn_scale,
             const uint16_t* __restrict__ h, int fmax, int T, int k, int d, int f, int f_sh, int S,
@@ -259,10 +273,26 @@ down_kernel(const uint8_t* __restrict__ down, const float* __restrict__ dn_scale
             for (int rr = 0; rr < R; ++rr)
 #pragma unroll
                 for (int j = 0; j < TG; ++j) acc[rr][j] = 0.0f;
+            // the next chunk's rows are in flight while this chunk is multiplied
+            // (one-token passes only: with more tokens per pass the registers run out)
+            constexpr bool kAhead = TG == 1;
+            uint4 wn[R];
+            if (kAhead && lane < nchunk)
+#pragma unroll
+                for (int rr = 0; rr < R; ++rr) wn[rr] = ld_stream16(W + (size_t)(j0 + rr) * rowbytes + (size_t)lane * 16);
             for (int c = lane; c < nchunk; c += kWarp) {
                 uint4 wv[R];
+                if (kAhead) {
 #pragma unroll
-                for (int rr = 0; rr < R; ++rr) wv[rr] = ld_stream16(W + (size_t)(j0 + rr) * rowbytes + (size_t)c * 16);
+                    for (int rr = 0; rr < R; ++rr) wv[rr] = wn[rr];
+                    if (c + kWarp < nchunk)
+#pragma unroll
+                        for (int rr = 0; rr < R; ++rr)
+                            wn[rr] = ld_stream16(W + (size_t)(j0 + rr) * rowbytes + (size_t)(c + kWarp) * 16);
+                } else {
+#pragma unroll
+                    for (int rr = 0; rr < R; ++rr) wv[rr] = ld_stream16(W + (size_t)(j0 + rr) * rowbytes + (size_t)c * 16);
+                }
 #pragma unroll
                 for (int j = 0; j < TG; ++j) {
                     if (j < ng) {
@@ -391,9 +421,10 @@ cudaError_t launch_experts_t(const LayerDims& L, const moe_weights& W, const uin
 cudaError_t launch_decode_experts(const LayerDims& L, const moe_weights& W, const uint16_t* x, int T,
                                   const Workspace& ws, int num_sms, const Launch& ctx) {
     if (T == 0) return cudaSuccess;
-    // Tokens per pass over a row: small groups keep the register count low enough for two CTAs
-    // per SM (more loads in flight); a bucket larger than the group takes more passes over rows
-    // that are then in L2.  Batch-union decode buckets hold one or two tokens almost always.
+    // Tokens per pass over a row.  Small batches: one, with the next chunk's rows in flight.
+    // Larger batches: two, which keeps the passes of the shared expert (every token) few; either
+    // way the register count allows two CTAs per SM, and a bucket larger than the group takes
+    // more passes over rows that are by then in L2.
     if (L.wkind == MOE_W_INT4_ROWSCALE)
         return T <= 4 ? launch_experts_t<MOE_W_INT4_ROWSCALE, 1>(L, W, x, T, ws, num_sms, ctx)
                       : launch_experts_t<MOE_W_INT4_ROWSCALE, 2>(L, W, x, T, ws, num_sms, ctx);
