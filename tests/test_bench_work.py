@@ -1,0 +1,51 @@
+"""The algorithmic work bench.py divides by device time (the roofline's `achieved`), checked
+against sizes written out from the layer's definition.  No GPU.
+
+- The container of the colibrì README stores an int4 expert as packed codes plus one fp32 scale
+  per output row; the iliria page gives about 19 MB per GLM expert, scales 0.22 % of the bytes.
+- The expert FFN is three d x f matrices per expert (gate, up, down): 2 flops per multiply-add
+  and per token slot.
+"""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import synthetic as syn  # noqa: E402
+
+GLM = syn.CONFIGS["glm_decode"]
+EXPERT = 18_915_328          # 3 * 2048 * 6144 / 2 bytes of codes + (2 * 2048 + 6144) * 4 bytes of scales
+
+
+def test_expert_bytes_match_the_container():
+    assert bench.expert_bytes(GLM) == EXPERT
+    codes = 3 * 2048 * 6144 // 2
+    assert abs((EXPERT - codes) / codes - 0.00217) < 1e-5        # the page's 0.22 % of scales
+
+
+def test_single_token_step_bytes():
+    w = bench.kernel_work(GLM, 1, 8)
+    kind, fused = w["fused"]
+    assert kind == "hbm"
+    router = 256 * 6144 * 4 + 256 * 4                  # fp32 router matrix and bias
+    x, h, out = 6144 * 2, 9 * 2048 * 2, 6144 * 4       # x read, h written and read back, y written
+    assert fused == 9 * EXPERT + router + x + 2 * h + out
+
+
+def test_gemm_flops_count_every_token_slot():
+    cfg = syn.CONFIGS["glm_prefill"]
+    w = bench.kernel_work(cfg, 2048, 200)              # flops do not depend on the unique experts
+    slots = 2048 * 8 + 2048                             # routed slots + the shared expert's
+    assert w["gemm_gateup"] == ("tensor", 2 * 2 * slots * 6144 * 2048)
+    assert w["gemm_down"] == ("tensor", 2 * slots * 6144 * 2048)
+    total = w["gemm_gateup"][1] + w["gemm_down"][1]
+    assert total == pytest.approx(1.392e12, rel=1e-3)  # 2 T (k + 1) 3 d f
+
+
+def test_job_throughput_counts_all_ranks():
+    assert bench.job_tokens_per_s(4, 100, 2, 50.0) == pytest.approx(4 * 100 * 2 / 0.05)
+    assert bench.replica_token_base(3) != bench.replica_token_base(2)
