@@ -3,26 +3,36 @@
 // For one token the layer reads each weight byte once, so its time is the time to stream the
 // router matrix and k + 1 experts from HBM.  Separate kernels for the router, gate/up and down
 // each pay the ramp of a fresh grid and leave HBM idle while the previous grid drains; here one
-// persistent CTA per SM runs the three steps back to back and keeps its copies in flight across
-// the joins:
+// persistent CTA per SM (16 warps) runs the steps back to back and keeps its copies in flight
+// across the joins.  Shared memory holds x, rearranged once per CTA so that a lane's 32-column
+// chunk loads without bank conflicts, and one ring of two TMA stages per warp (a gate row, the
+// matching up row and two 16-byte slivers holding their scales).
 //
-//   A  router + shared expert.  Every warp first queues its shared-expert gate/up row pairs (they
-//      need no routing) into its ring of TMA stages, then computes its piece of the router logits
-//      (fp64, one expert x 1024 columns per unit) and stores it.  The CTA arrives on a grid
-//      barrier, and the warps reduce their shared rows while the other CTAs arrive.
-//   B  selection.  Warp 0 of every CTA waits for the barrier, sums the pieces (the same order in
-//      every CTA, so every CTA selects the same experts) and runs the top-k; the k experts and
-//      gate weights go to shared memory.
-//   C  routed gate/up: row pairs of the k experts, h = SiLU(gate) * up in fp16 (global, L2).
-//      A warp that has finished its row pairs queues its first down rows (they do not depend on h),
-//      then the CTA arrives on the second grid barrier, after which every h is complete.
+//   A  router + shared expert.  One bulk copy brings x in; each warp's first router piece (one
+//      expert x 1024 columns, coalesced loads) is in flight meanwhile.  The warps rearrange x,
+//      sum it, queue their shared-expert row pairs (they need no routing), compute their router
+//      pieces in fp64 and store them.  The CTA arrives on grid barrier 0, and the warps reduce
+//      their shared rows while the other CTAs arrive.
+//   B  selection, by the whole CTA: one bulk copy gathers every piece; thread e sums expert e's
+//      pieces (the same order in every CTA, so every CTA selects the same experts) and forms an
+//      order-preserving integer key; the k best of each warp's 32 experts become candidates, and
+//      each candidate's rank among the candidates is its overall rank.  The k experts (ascending)
+//      and their gate weights go to shared memory.
+//   C  routed gate/up: row pairs of the k experts, strided over every warp of the grid;
+//      h = SiLU(gate) * up in fp16 (global, L2), the SiLU of 32 row pairs at a time.  A warp that
+//      has finished its row pairs queues its first down rows (they do not depend on h), then the
+//      CTA arrives on grid barrier 1, after which every h is complete.
 //   D  down + combine: CTA b owns output rows [b d / G, (b + 1) d / G) of every slot (the k
 //      routed experts in ascending index order, then the shared expert); its warps split the
 //      (slot, row) list, and the CTA adds the slots with their gate weights and stores y.
 //
-// Dequantisation and the precision of each step are those of decode1.cu (bf16 136 + s for
-// gate/up with the offset removed through the sum of x; exact fp16 s for down; fp32
-// accumulation; h rounded to fp16).  The router logits accumulate in fp64.
+// Dequantisation: gate/up as bf16 136 + s (one LOP3 per two codes) with the offset removed
+// through the sum of x; down as fp16 3/2 + s/16 (one shift and one LOP3 per two codes) with the
+// offset removed through the sum of h.  Products are exact, sums fp32, h is rounded to fp16; the
+// router logits accumulate in fp64.
+//
+// Phase timestamps (%globaltimer, thread 0 of each CTA) go to the workspace for the layer's
+// debug read.
 //
 // The grid barrier counts arrivals in a 64-bit word that only grows.  Every CTA arrives exactly
 // once at each of the two barriers of a launch, also on its error paths, so a launch starts with
