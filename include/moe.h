@@ -139,8 +139,8 @@ moe_status moe_route(moe_layer *layer, const uint16_t *x, int32_t T, int32_t *id
  * moe_forward -- the whole layer, steps 1 to 4.
  *   x    device, [T][d] bf16
  *   out  device, [T][d] fp32, or bf16 when cfg->out_bf16 (written)
- *   0 <= T <= max_tokens.  Asynchronous and host-sync free (it can be captured in a CUDA
- *   graph).  Calls on one layer must not overlap on the device (they share its workspace).
+ *   0 <= T <= max_tokens.  Asynchronous: no host synchronisation and no allocation.  Calls on
+ *   one layer must not overlap on the device (they share its workspace).
  */
 moe_status moe_forward(moe_layer *layer, const uint16_t *x, int32_t T, void *out, moe_stream stream);
 
@@ -182,6 +182,9 @@ void moe_layer_destroy(moe_layer *layer);
  *                               down+combine kernels; 0: the general decode kernels.  A request
  *                               for a mode the shape does not allow falls back to the next lower
  *                               one; get returns the mode in use.  Same results within tolerance.
+ *                               Mode 2 is a cooperative launch of one CTA per SM: it starts when
+ *                               every SM can take its CTA, so kernels of other streams running at
+ *                               the same time delay it.
  */
 /*   MOE_OPT_PROGRAMMATIC_LAUNCH  1 (default): chained kernels of the single-token path start
  *                               early with programmatic dependent launch and wait on the device
