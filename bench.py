@@ -48,7 +48,7 @@ WORKLOADS = {
     "granite": "Granite-1B-a400m-like MoE layer decode, T=1, d=1024, E=32, top-8 softmax, f=512 bf16",
     "tiny": "tiny MoE layer, T=4, d=256, E=8, top-2 softmax, f=128 int4",
 }
-DEFAULT_STEPS = {"glm_decode": 400, "glm_union2": 300, "glm_union32": 100, "glm_prefill": 30, "granite": 2000,
+DEFAULT_STEPS = {"glm_decode": 2000, "glm_union2": 1000, "glm_union32": 200, "glm_prefill": 60, "granite": 2000,
                  "tiny": 200}
 FLUSH_BYTES = 512 << 20
 
