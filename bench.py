@@ -164,6 +164,15 @@ def slowest_rank_ms(ms: float, dist, device) -> float:
     return float(t.item())
 
 
+def step_percentiles(step_ms) -> dict:
+    """p10 / p50 / p90 of the per-step device times (ms), nearest-rank."""
+    v = sorted(float(t) for t in step_ms)
+    if not v:
+        return {}
+    pick = lambda q: v[min(len(v) - 1, max(0, int(round(q * (len(v) - 1)))))]  # noqa: E731
+    return {"p10": pick(0.10), "p50": pick(0.50), "p90": pick(0.90)}
+
+
 def job_tokens_per_s(world: int, steps: int, T: int, max_ms: float) -> float:
     """Whole-job throughput: the tokens every rank processed over the slowest rank's time."""
     return world * steps * T / (max_ms / 1e3)
@@ -428,13 +437,14 @@ def run_ours(a, rank, world, local_rank):
         if dist:
             dist.barrier()
         layer.profile(False)
-        return sum(s.elapsed_time(e) for s, e in evs)
+        return [s.elapsed_time(e) for s, e in evs]
 
     clocks = Clocks(local_rank)
     clocks.start()
-    total_ms = timed_pass(False)
+    step_ms = timed_pass(False)
     clk = clocks.stop()
-    prof_ms = timed_pass(True)
+    total_ms = sum(step_ms)
+    prof_ms = sum(timed_pass(True))
     prof = layer.profile_read()
     if layer.last_error() != qe.MOE_OK:
         raise RuntimeError("device status after timing: " + qe.status_str(layer.last_error()))
@@ -489,7 +499,7 @@ def run_ours(a, rank, world, local_rank):
     ms_per_step = total_ms / a.steps
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
-        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "ms_per_step": ms_per_step, "step_ms_percentiles": step_percentiles(step_ms), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int4xbf16->f32" if cfg.wkind == syn.W_INT4 else "bf16->f32", "data": "synthetic",
         "config": {"workload": a.workload, "desc": WORKLOADS[a.workload], "tokens_per_step": T,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",

@@ -49,3 +49,11 @@ def test_gemm_flops_count_every_token_slot():
 def test_job_throughput_counts_all_ranks():
     assert bench.job_tokens_per_s(4, 100, 2, 50.0) == pytest.approx(4 * 100 * 2 / 0.05)
     assert bench.replica_token_base(3) != bench.replica_token_base(2)
+
+
+def test_step_percentiles():
+    assert bench.step_percentiles([]) == {}
+    p = bench.step_percentiles([5.0, 1.0, 3.0, 2.0, 4.0])
+    assert p == {"p10": 1.0, "p50": 3.0, "p90": 5.0}
+    q = bench.step_percentiles(range(101))
+    assert (q["p10"], q["p50"], q["p90"]) == (10.0, 50.0, 90.0)
