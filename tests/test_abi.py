@@ -61,3 +61,29 @@ def test_argument_errors_need_no_device(lib):
     assert lib.moe_last_error(None) == qe.MOE_ERR_INVALID_ARG
     lib.moe_layer_destroy(None)
     assert lib.moe_layer_workspace_bytes(None) == 0
+
+
+def _header_enum_values():
+    """name -> value for every `NAME = <int>` inside the header's enums."""
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return {n: int(v) for n, v in re.findall(r"\b(MOE_[A-Z0-9_]+)\s*=\s*(\d+)", text)}
+
+
+def test_binding_constants_match_the_header():
+    enums = _header_enum_values()
+    for name, value in enums.items():
+        if hasattr(qe, name):
+            assert getattr(qe, name) == value, name
+    # debug items and kernel names of the binding, in the header's numbering
+    for item, value in qe.DEBUG_ITEMS.items():
+        assert enums["MOE_DEBUG_" + item.upper()] == value
+    assert len(qe.KERNELS) == enums["MOE_KERNEL_COUNT"]
+    for i, name in enumerate(qe.KERNELS):
+        key = "MOE_KERNEL_" + name.upper()
+        assert enums[key] == i, key
+
+
+def test_kernel_names_of_the_library(lib):
+    for i, name in enumerate(qe.KERNELS):
+        assert qe.moe_kernel_name(i) == name
