@@ -265,20 +265,44 @@ def oracle_sample_tokens(cfg, name):
     return {"glm_union2": 2, "glm_union32": 2, "glm_prefill": 2}.get(name, cfg.T)
 
 
-def time_oracle(cfg, name, seed, budget_s, min_calls=1, max_calls=None):
+def time_oracle(cfg, name, seed, budget_s, min_calls=1, max_calls=None, threads=None, layer=None):
+    """The oracle's tokens/s on a bounded sample of the workload: calls of oracle_sample_tokens
+    tokens until budget_s has passed.  threads: OpenMP threads for this timing only (default:
+    all host cores).  layer: a (layer, x) pair from an earlier call, to skip building it again."""
     import oracle
     n_tok = oracle_sample_tokens(cfg, name)
-    x = syn.gen_x(cfg, seed, T=n_tok)
-    L = oracle_sample_layer(cfg, seed, x)
-    calls, t0 = 0, time.perf_counter()
-    while True:
-        L.forward(x)
-        calls += 1
-        el = time.perf_counter() - t0
-        if calls >= min_calls and (el >= budget_s or (max_calls and calls >= max_calls)):
-            break
-    return {"value": calls * n_tok / el, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{calls} oracle calls of {n_tok} token(s) of the {name} workload ({el:.1f} s on host cores)"}
+    if layer is None:
+        x = syn.gen_x(cfg, seed, T=n_tok)
+        layer = (oracle_sample_layer(cfg, seed, x), x)
+    L, x = layer
+    all_cores = oracle.num_threads()
+    if threads:
+        oracle.set_num_threads(threads)
+    try:
+        cores = oracle.num_threads()
+        calls, t0 = 0, time.perf_counter()
+        while True:
+            L.forward(x)
+            calls += 1
+            el = time.perf_counter() - t0
+            if calls >= min_calls and (el >= budget_s or (max_calls and calls >= max_calls)):
+                break
+    finally:
+        if threads:
+            oracle.set_num_threads(all_cores)
+    where = "host cores" if cores > 1 else "one host core"
+    return {"value": calls * n_tok / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{calls} oracle calls of {n_tok} token(s) of the {name} workload ({el:.1f} s on {where})",
+            "layer": layer}
+
+
+def cpu_baseline(cfg, name, seed, budget_s):
+    """The oracle on all host cores, plus the same sample on one core (a quarter of the budget)."""
+    res = time_oracle(cfg, name, seed, budget_s)
+    one = time_oracle(cfg, name, seed, budget_s / 4, threads=1, layer=res.pop("layer"))
+    one.pop("layer")
+    res["single_core"] = {k: one[k] for k in ("value", "unit", "cores", "sample")}
+    return res
 
 
 # ------------------------------------------------------------------------------------------
@@ -515,7 +539,7 @@ def run_ours(a, rank, world, local_rank):
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        line["cpu_baseline"] = time_oracle(cfg, a.workload, a.seed, a.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(cfg, a.workload, a.seed, a.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     layer.close()

@@ -68,6 +68,8 @@ def lib():
         L.oracle_forward.argtypes = [ctypes.POINTER(_Layer), P, I32, I32, P, P, P, P]
         L.oracle_expert_ffn.argtypes = [ctypes.POINTER(_Layer), I32, P, P, P, P, P]
         L.oracle_num_threads.argtypes = []
+        L.oracle_set_num_threads.argtypes = [ctypes.c_int]
+        L.oracle_set_num_threads.restype = None
         _lib = L
     return _lib
 
@@ -83,6 +85,11 @@ def _check(rc: int, what: str):
 
 def num_threads() -> int:
     return int(lib().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of the following calls (results do not depend on it)."""
+    lib().oracle_set_num_threads(int(n))
 
 
 # ----------------------------------------------------------------------------------------

@@ -423,3 +423,16 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* Threads of the following oracle calls (n >= 1): only the timing of the CPU baseline on one
+ * core uses it.  The results do not depend on it: every parallel loop writes disjoint outputs
+ * and each sum runs in its own fixed order inside one thread. */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

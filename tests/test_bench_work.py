@@ -57,3 +57,30 @@ def test_step_percentiles():
     assert p == {"p10": 1.0, "p50": 3.0, "p90": 5.0}
     q = bench.step_percentiles(range(101))
     assert (q["p10"], q["p50"], q["p90"]) == (10.0, 50.0, 90.0)
+
+
+def test_cpu_baseline_times_all_cores_and_one():
+    import oracle
+    cores = oracle.num_threads()
+    res = bench.cpu_baseline(syn.CONFIGS["tiny"], "tiny", 0, 0.2)
+    assert res["kind"] == "oracle" and res["unit"] == "tokens/s" and res["value"] > 0
+    assert res["cores"] == cores and "layer" not in res
+    one = res["single_core"]
+    assert one["cores"] == 1 and one["value"] > 0 and "one host core" in one["sample"]
+    assert oracle.num_threads() == cores                # the thread count is put back
+
+
+def test_oracle_result_does_not_depend_on_threads():
+    import oracle
+    cfg = syn.CONFIGS["tiny"]
+    x = syn.gen_x(cfg, 0, T=cfg.T)
+    L = bench.oracle_sample_layer(cfg, 0, x)
+    cores = oracle.num_threads()
+    many = L.forward(x)
+    oracle.set_num_threads(1)
+    try:
+        one = L.forward(x)
+    finally:
+        oracle.set_num_threads(cores)
+    for key in ("out", "idx", "w", "gap"):
+        assert many[key].tobytes() == one[key].tobytes()
