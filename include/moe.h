@@ -207,8 +207,8 @@ moe_status moe_layer_get_option(const moe_layer *layer, int32_t option, int64_t 
  *                    (CNT is not written by the single-launch T = 1 path)
  *   MOE_DEBUG_XSUM   fp64 [T]
  *   MOE_DEBUG_TRACE  uint64 [SMs][16]: for the single-launch T = 1 path, the %globaltimer value (ns)
- *                    at which each CTA passed its phase boundaries: 0 start, 1 x in registers,
- *                    2 router pieces stored, 3 shared rows done, 4 first grid barrier passed,
+ *                    at which each CTA passed its phase boundaries: 0 start, 1 x rearranged
+ *                    in shared memory, 2 router pieces stored, 3 shared rows done, 4 first grid barrier passed,
  *                    5 router pieces gathered, 6 experts selected, 7 routed gate/up done, 8 h
  *                    complete, 9 down done, 10 output stored, 11 x in shared memory, 12..15
  *                    steps of the selection (candidates, ranks, gate weights, proxy fence)
