@@ -20,7 +20,8 @@ MOE_W_INT4_ROWSCALE, MOE_W_BF16 = 0, 1
 
 # Every symbol that include/moe.h declares.
 EXPORTS = (
-    "moe_pack_int4", "moe_layer_create", "moe_route", "moe_forward", "moe_forward_host", "moe_last_error",
+    "moe_pack_int4", "moe_layer_create", "moe_route", "moe_forward", "moe_forward_host", "moe_forward_host_async",
+    "moe_last_error",
     "moe_layer_destroy", "moe_layer_workspace_bytes", "moe_layer_last_launches", "moe_status_str",
     "moe_profile_enable", "moe_profile_read", "moe_kernel_name", "moe_route_noalloc",
     "moe_layer_set_option", "moe_layer_get_option", "moe_layer_debug_read",
@@ -66,6 +67,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         L.moe_route.argtypes = [P, P, I32, P, P, P]
         L.moe_forward.argtypes = [P, P, I32, P, P]
         L.moe_forward_host.argtypes = [P, P, I32, P, P]
+        L.moe_forward_host_async.argtypes = [P, P, I32, P, P]
         L.moe_last_error.argtypes = [P]
         L.moe_layer_destroy.argtypes = [P]
         L.moe_layer_destroy.restype = None
@@ -84,7 +86,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         L.moe_layer_get_option.argtypes = [P, I32, ctypes.POINTER(I64)]
         L.moe_layer_debug_read.argtypes = [P, I32, P, I64]
         for n in ("moe_pack_int4", "moe_layer_create", "moe_route", "moe_forward", "moe_forward_host",
-                  "moe_last_error", "moe_profile_enable", "moe_profile_read", "moe_route_noalloc",
+                  "moe_forward_host_async", "moe_last_error", "moe_profile_enable", "moe_profile_read", "moe_route_noalloc",
                   "moe_layer_set_option", "moe_layer_get_option", "moe_layer_debug_read"):
             getattr(L, n).restype = ctypes.c_int
         _lib = L
@@ -139,6 +141,13 @@ def moe_forward(layer: int, x, T: int, out, stream=None):
 def moe_forward_host(layer: int, x_host, T: int, out_host, stream=None):
     """x_host / out_host are CPU tensors (pinned for asynchronous copies)."""
     _check(load().moe_forward_host(layer, _ptr(x_host), T, _ptr(out_host), _stream(stream)), "moe_forward_host")
+
+
+def moe_forward_host_async(layer: int, x_host, T: int, out_host, stream=None):
+    """moe_forward_host without the final wait: the host buffers may be reused, and out_host read,
+    once the stream has passed the call."""
+    _check(load().moe_forward_host_async(layer, _ptr(x_host), T, _ptr(out_host), _stream(stream)),
+           "moe_forward_host_async")
 
 
 def moe_last_error(layer: int) -> int:
@@ -220,6 +229,9 @@ class MoELayer:
 
     def forward_host(self, x_host, out_host, stream=None):
         moe_forward_host(self.handle, x_host, x_host.shape[0], out_host, stream)
+
+    def forward_host_async(self, x_host, out_host, stream=None):
+        moe_forward_host_async(self.handle, x_host, x_host.shape[0], out_host, stream)
 
     def last_error(self) -> int:
         return moe_last_error(self.handle)

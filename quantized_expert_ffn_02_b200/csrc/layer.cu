@@ -315,7 +315,8 @@ moe_status moe_forward(moe_layer* L, const uint16_t* x, int32_t T, void* out, mo
     return from_cuda(e);
 }
 
-moe_status moe_forward_host(moe_layer* L, const uint16_t* x_host, int32_t T, void* out_host, moe_stream stream) {
+moe_status moe_forward_host_async(moe_layer* L, const uint16_t* x_host, int32_t T, void* out_host,
+                                  moe_stream stream) {
     if (!L || T < 0 || T > L->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
@@ -326,9 +327,13 @@ moe_status moe_forward_host(moe_layer* L, const uint16_t* x_host, int32_t T, voi
     if (e != cudaSuccess) return from_cuda(e);
     moe_status st = moe_forward(L, L->x_stage, T, L->out_stage, stream);
     if (st != MOE_OK) return st;
-    e = cudaMemcpyAsync(out_host, L->out_stage, obytes, cudaMemcpyDeviceToHost, s);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-    return from_cuda(e);
+    return from_cuda(cudaMemcpyAsync(out_host, L->out_stage, obytes, cudaMemcpyDeviceToHost, s));
+}
+
+moe_status moe_forward_host(moe_layer* L, const uint16_t* x_host, int32_t T, void* out_host, moe_stream stream) {
+    const moe_status st = moe_forward_host_async(L, x_host, T, out_host, stream);
+    if (st != MOE_OK || T == 0) return st;
+    return from_cuda(cudaStreamSynchronize((cudaStream_t)stream));
 }
 
 moe_status moe_last_error(moe_layer* L) {

@@ -57,6 +57,8 @@ def test_argument_errors_need_no_device(lib):
     assert lib.moe_pack_int4(None, 4, 7, None, None, None) == qe.MOE_ERR_INVALID_ARG      # odd cols
     assert lib.moe_pack_int4(None, 0, 8, None, None, None) == qe.MOE_OK                  # nothing to do
     assert lib.moe_forward(None, None, 1, None, None) == qe.MOE_ERR_INVALID_ARG
+    assert lib.moe_forward_host(None, None, 1, None, None) == qe.MOE_ERR_INVALID_ARG
+    assert lib.moe_forward_host_async(None, None, 1, None, None) == qe.MOE_ERR_INVALID_ARG
     assert lib.moe_route(None, None, 1, None, None, None) == qe.MOE_ERR_INVALID_ARG
     assert lib.moe_last_error(None) == qe.MOE_ERR_INVALID_ARG
     lib.moe_layer_destroy(None)

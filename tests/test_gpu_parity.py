@@ -288,6 +288,17 @@ def test_forward_host_matches_device():
     oh = torch.empty((cfg.T, cfg.d), dtype=torch.float32).pin_memory()
     layer.forward_host(xh, oh)
     assert np.array_equal(oh.numpy(), dev_out)
+    # the asynchronous form: several calls in a row on one stream, one wait at the end; each
+    # call's output lands in its own pinned buffer, in stream order
+    outs = [torch.empty((cfg.T, cfg.d), dtype=torch.float32).pin_memory() for _ in range(3)]
+    xs = [xh, torch.from_numpy(x[::-1].copy().view(np.int16)).pin_memory(), xh]
+    for xi, oi in zip(xs, outs):
+        layer.forward_host_async(xi, oi)
+    torch.cuda.synchronize()
+    assert layer.last_error() == 0
+    assert np.array_equal(outs[0].numpy(), dev_out)
+    assert np.array_equal(outs[2].numpy(), dev_out)
+    assert np.array_equal(outs[1].numpy(), run_forward(layer, x[::-1].copy()))
     layer.close()
 
 
