@@ -158,9 +158,9 @@ moe_status moe_forward_host(moe_layer *layer, const uint16_t *x_host, int32_t T,
  * x, the layer and the device->host copy of out are enqueued on `stream` and the call returns.
  * Calls on one stream may follow each other at once: stream order keeps each call's copies and
  * kernels apart from the next call's, although they share the layer's staging area.  x_host
- * must stay unchanged, and out_host is complete, only once the stream has passed the call (an
- * event or a synchronize); with pinned buffers the copies are asynchronous to the host,
- * with pageable ones the runtime may wait inside the call.  Asynchronous.
+ * must stay unchanged until the stream has passed the call (an event or a synchronize), and
+ * out_host holds the result only from then on.  With pinned buffers the copies are asynchronous
+ * to the host; with pageable ones the runtime may wait inside the call.  Asynchronous.
  */
 moe_status moe_forward_host_async(moe_layer *layer, const uint16_t *x_host, int32_t T, void *out_host,
                                   moe_stream stream);
