@@ -84,3 +84,19 @@ def test_oracle_result_does_not_depend_on_threads():
         oracle.set_num_threads(cores)
     for key in ("out", "idx", "w", "gap"):
         assert many[key].tobytes() == one[key].tobytes()
+
+
+def test_traffic_is_reported_only_for_unchanged_sources():
+    import json
+    rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    for kernel in ("fused", "gemm_gateup", "gemm_down"):
+        r = rec[kernel]
+        fresh = bench.source_sha(r["sources"]) == r["source_sha"]
+        assert bench.traffic_for(kernel) == (r["bytes_per_launch"] if fresh else None)
+        assert r["bytes_per_launch"] > 0
+    assert bench.traffic_for("no_such_kernel") is None
+
+
+def test_traffic_is_null_once_a_source_changes(monkeypatch):
+    monkeypatch.setattr(bench, "source_sha", lambda paths: "0" * 16)
+    assert bench.traffic_for("fused") is None
