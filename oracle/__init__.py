@@ -24,7 +24,7 @@ _SRC = os.path.join(_HERE, "oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 ROUTER_SOFTMAX, ROUTER_SIGMOID = 0, 1
-W_INT4, W_BF16, W_INT8 = 0, 1, 2
+W_INT4, W_BF16, W_INT8, W_INT2 = 0, 1, 2, 3
 MODE_PER_TOKEN, MODE_UNION, MODE_DENSE = 0, 1, 2
 ERR = {0: "ok", 1: "range (non-finite input)", 2: "missing expert", 3: "bad argument", 4: "out of memory"}
 
@@ -64,6 +64,10 @@ def lib():
         L.oracle_pack_int4.argtypes = [P, I64, I64, P, P]
         L.oracle_unpack_int4.argtypes = [P, I64, I64, P]
         L.oracle_unpack_int4.restype = None
+        L.oracle_quantize_tier.argtypes = [P, I64, I64, I32, P, P]
+        L.oracle_pack_int2.argtypes = [P, I64, I64, P, P]
+        L.oracle_unpack_int2.argtypes = [P, I64, I64, P]
+        L.oracle_unpack_int2.restype = None
         L.oracle_route.argtypes = [ctypes.POINTER(_Layer), P, I32, P, P, P, P]
         L.oracle_forward.argtypes = [ctypes.POINTER(_Layer), P, I32, I32, P, P, P, P]
         L.oracle_expert_ffn.argtypes = [ctypes.POINTER(_Layer), I32, P, P, P, P, P]
@@ -123,6 +127,36 @@ def unpack_int4(packed: np.ndarray, cols: int) -> np.ndarray:
     rows = packed.shape[0]
     q = np.empty((rows, cols), np.int8)
     lib().oracle_unpack_int4(_p(packed), rows, cols, _p(q))
+    return q
+
+
+def quantize_tier(w: np.ndarray, bits: int):
+    """The b-bit tier (2, 4 or 8) in the int8 container: (q int8 [rows][cols], scales fp32 [rows])."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    rows, cols = w.shape
+    q = np.empty((rows, cols), np.int8)
+    s = np.empty(rows, np.float32)
+    _check(lib().oracle_quantize_tier(_p(w), rows, cols, int(bits), _p(q), _p(s)), "quantize_tier")
+    return q, s
+
+
+def pack_int2(w: np.ndarray, allow_nonfinite: bool = False):
+    """Packed int2: (bytes u8 [rows][cols/4], scales fp32 [rows])."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    rows, cols = w.shape
+    p = np.empty((rows, cols // 4), np.uint8)
+    s = np.empty(rows, np.float32)
+    rc = lib().oracle_pack_int2(_p(w), rows, cols, _p(p), _p(s))
+    if not (allow_nonfinite and rc == 1):
+        _check(rc, "pack_int2")
+    return p, s
+
+
+def unpack_int2(packed: np.ndarray, cols: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    rows = packed.shape[0]
+    q = np.empty((rows, cols), np.int8)
+    lib().oracle_unpack_int2(_p(packed), rows, cols, _p(q))
     return q
 
 

@@ -21,8 +21,9 @@
  *              after them (open-1b-verify, "Tensor mapping": w_gate_up split at the
  *              row boundary; iliria, "What's implemented": gate+up fused).
  *   weights    packed int4 with one fp32 scale per output row, dequantised on use
- *              (colibri README, "What's implemented": int8 / packed int4, per-row
- *              scales, dequant-on-use), or bf16, or the int8 container.
+ *              (colibri README, "What's implemented": int8 / packed int4 / packed int2,
+ *              per-row scales, dequant-on-use), or bf16, or the int8 container (which
+ *              holds the codes of any tier, one per byte), or packed int2.
  *   combine    out[t] = sum over chosen experts in ascending index of w * y, plus the
  *              shared expert with weight 1 (colibri README, "What's implemented":
  *              shared expert).
@@ -43,7 +44,7 @@
 #include <string.h>
 
 enum { ORACLE_ROUTER_SOFTMAX = 0, ORACLE_ROUTER_SIGMOID = 1 };
-enum { ORACLE_W_INT4 = 0, ORACLE_W_BF16 = 1, ORACLE_W_INT8 = 2 };
+enum { ORACLE_W_INT4 = 0, ORACLE_W_BF16 = 1, ORACLE_W_INT8 = 2, ORACLE_W_INT2 = 3 };
 enum { ORACLE_MODE_PER_TOKEN = 0, ORACLE_MODE_UNION = 1, ORACLE_MODE_DENSE = 2 };
 enum { ORACLE_OK = 0, ORACLE_ERR_RANGE = 1, ORACLE_ERR_MISSING_EXPERT = 2, ORACLE_ERR_ARG = 3,
        ORACLE_ERR_NOMEM = 4 };
@@ -53,7 +54,7 @@ typedef struct {
     double scaling;
     const float *router_w;          /* [E][d] */
     const float *router_bias;       /* [E] or NULL */
-    const void *const *gate_up;     /* [E] pointers to [2f][d/2] u8 | [2f][d] bf16 | [2f][d] s8 */
+    const void *const *gate_up;     /* [E] pointers to [2f][d/2] u8 | [2f][d] bf16 | [2f][d] s8 | [2f][d/4] u8 */
     const float *const *gate_up_scale;  /* [E] pointers to [2f] (int4 / int8) */
     const void *const *down;        /* [E] pointers to [d][f/2] u8 | [d][f] bf16 | [d][f] s8 */
     const float *const *down_scale;     /* [E] pointers to [d] */
@@ -81,6 +82,13 @@ static int nibble_value(uint8_t byte, int high)
     return n >= 8 ? n - 16 : n;     /* two's-complement 4-bit value */
 }
 
+/* Code i (0..3) of a packed int2 byte: bits 2i .. 2i+1, a two's-complement 2-bit value. */
+static int crumb_value(uint8_t byte, int i)
+{
+    int n = (byte >> (2 * i)) & 3;
+    return n >= 2 ? n - 4 : n;
+}
+
 /* One weight of a [rows][cols] matrix in the layer's storage kind, dequantised, in fp64.
  * The product q * s is exact in fp64 (4-bit times 24-bit significands). */
 static double weight_at(int wkind, const void *m, const float *scale, int64_t row, int64_t col,
@@ -90,6 +98,10 @@ static double weight_at(int wkind, const void *m, const float *scale, int64_t ro
         return bf16_value(((const uint16_t *)m)[row * cols + col]);
     if (wkind == ORACLE_W_INT8)
         return (double)((const int8_t *)m)[row * cols + col] * (double)scale[row];
+    if (wkind == ORACLE_W_INT2) {
+        uint8_t byte = ((const uint8_t *)m)[row * (cols / 4) + col / 4];
+        return (double)crumb_value(byte, (int)(col & 3)) * (double)scale[row];
+    }
     const uint8_t *p = (const uint8_t *)m;
     uint8_t byte = p[row * (cols / 2) + col / 2];
     return (double)nibble_value(byte, (int)(col & 1)) * (double)scale[row];
@@ -145,6 +157,67 @@ void oracle_unpack_int4(const uint8_t *packed, int64_t rows, int64_t cols, int8_
     for (int64_t r = 0; r < rows; ++r)
         for (int64_t c = 0; c < cols; ++c)
             q[r * cols + c] = (int8_t)nibble_value(packed[r * (cols / 2) + c / 2], (int)(c & 1));
+}
+
+/*
+ * The quantiser of the b-bit tier (b = 2, 4 or 8) into the int8 container, one code per byte
+ * (colibri README, "What's implemented": int8 / packed int4 / packed int2 quantisation with
+ * per-row scales).  The same symmetric rule as the int4 tier, with qmax = 2^(b-1) - 1:
+ * per row m = max|w| (fp32), s = m / qmax (fp32 IEEE division), q = clamp(round-half-even(
+ * fp32(w / s)), -qmax - 1, qmax); a zero row has s = 0 and q = 0.  Non-finite input is an
+ * error (its codes are 0).
+ */
+int oracle_quantize_tier(const float *w, int64_t rows, int64_t cols, int32_t bits, int8_t *q, float *scales)
+{
+    if (rows < 0 || cols < 0 || (bits != 2 && bits != 4 && bits != 8)) return ORACLE_ERR_ARG;
+    const float qmax = (float)((1 << (bits - 1)) - 1);
+    const float qmin = -qmax - 1.0f;
+    int bad = 0;
+    for (int64_t r = 0; r < rows; ++r) {
+        const float *row = w + r * cols;
+        float m = 0.0f;
+        for (int64_t c = 0; c < cols; ++c) {
+            if (!isfinite(row[c])) bad = 1;
+            float a = fabsf(row[c]);
+            if (a > m) m = a;
+        }
+        float s = m / qmax;
+        scales[r] = s;
+        for (int64_t c = 0; c < cols; ++c) {
+            float v = 0.0f;
+            if (s != 0.0f && isfinite(row[c])) v = rintf(row[c] / s);
+            if (v > qmax) v = qmax;
+            if (v < qmin) v = qmin;
+            q[r * cols + c] = (int8_t)v;
+        }
+    }
+    return bad ? ORACLE_ERR_RANGE : ORACLE_OK;
+}
+
+/* Packed int2 container: the 2-bit tier's codes, four per byte, column 4j + i of a row in bits
+ * 2i .. 2i+1 of byte j (the lowest column in the lowest bits, as the int4 container puts the
+ * even column in the low nibble).  cols must be a multiple of 4. */
+int oracle_pack_int2(const float *w, int64_t rows, int64_t cols, uint8_t *packed, float *scales)
+{
+    if (rows < 0 || cols < 0 || (cols & 3)) return ORACLE_ERR_ARG;
+    int8_t *q = (int8_t *)malloc((size_t)(rows * cols > 0 ? rows * cols : 1));
+    if (!q) return ORACLE_ERR_NOMEM;
+    int rc = oracle_quantize_tier(w, rows, cols, 2, q, scales);
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < cols / 4; ++j) {
+            uint8_t b = 0;
+            for (int i = 0; i < 4; ++i) b |= (uint8_t)((q[r * cols + 4 * j + i] & 3) << (2 * i));
+            packed[r * (cols / 4) + j] = b;
+        }
+    free(q);
+    return rc;
+}
+
+void oracle_unpack_int2(const uint8_t *packed, int64_t rows, int64_t cols, int8_t *q)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            q[r * cols + c] = (int8_t)crumb_value(packed[r * (cols / 4) + c / 4], (int)(c & 3));
 }
 
 /* ------------------------------------------------------------------------------------ */
@@ -319,7 +392,8 @@ int oracle_forward(const oracle_layer *L, const uint16_t *x, int32_t T, int32_t 
 {
     const int d = L->d, E = L->n_experts, k = L->top_k;
     const int S = L->n_shared > 0 ? 1 : 0;
-    if (T < 0 || k < 1 || k > E || (L->wkind == ORACLE_W_INT4 && ((d & 1) || (L->f & 1))))
+    if (T < 0 || k < 1 || k > E || (L->wkind == ORACLE_W_INT4 && ((d & 1) || (L->f & 1))) ||
+        (L->wkind == ORACLE_W_INT2 && ((d & 3) || (L->f & 3) || (S && (L->f_shared & 3)))))
         return ORACLE_ERR_ARG;
     double *gap_buf = gap ? gap : (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
     int rc = oracle_route(L, x, T, idx, w, NULL, gap_buf);

@@ -146,6 +146,8 @@ ROUTER_SOFTMAX = 0
 ROUTER_SIGMOID = 1
 W_INT4 = 0
 W_BF16 = 1
+W_INT8 = 2          # one code per byte, the int8 tier (scale max|w| / 127)
+W_INT2 = 3          # four codes per byte, the int2 tier (scale max|w| / 1)
 
 
 @dataclasses.dataclass(frozen=True)

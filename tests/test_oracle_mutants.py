@@ -35,6 +35,12 @@ MUTANTS = {
     "shared expert dropped": ("for (int j = 0; j < d; ++j) o[j] += y[j];", "(void)0;"),
     "softmax over all experts": ("for (int r = 0; r < k; ++r) sum += exp(logit[idx[r]] - m);",
                                  "for (int e = 0; e < E; ++e) sum += exp(logit[e] - m);"),
+    "int2 codes read highest bits first": ("int n = (byte >> (2 * i)) & 3;", "int n = (byte >> (6 - 2 * i)) & 3;"),
+    "int2 codes not sign-extended": ("return n >= 2 ? n - 4 : n;", "return n;"),
+    "int2 packer reverses the byte": ("b |= (uint8_t)((q[r * cols + 4 * j + i] & 3) << (2 * i));",
+                                      "b |= (uint8_t)((q[r * cols + 4 * j + i] & 3) << (6 - 2 * i));"),
+    "tier qmax off by one": ("const float qmax = (float)((1 << (bits - 1)) - 1);",
+                             "const float qmax = (float)(1 << (bits - 1));"),
 }
 
 PIN_TESTS = [
@@ -50,6 +56,11 @@ PIN_TESTS = [
     lambda: pins.test_shared_expert_adds_with_weight_one(),
     lambda: pins.test_exact_integer_case(),
     lambda: pins.test_int4_packing_bit_identical_to_int8_container((33, 130)),
+    lambda: pins.test_int2_crumb_layout_golden(),
+    lambda: pins.test_tier_quantiser_golden_rows("int2_rows"),
+    lambda: pins.test_tier_quantiser_golden_rows("int8_rows"),
+    lambda: pins.test_int2_packing_bit_identical_to_int8_container((33, 132)),
+    lambda: pins.test_single_expert_layer_is_textbook_swiglu_other_tiers(oracle.W_INT2, 2),
 ]
 
 
@@ -67,7 +78,8 @@ def test_pins_catch_mutant(name, tmp_path, monkeypatch):
     real = oracle.lib()
     mutant = ctypes.CDLL(str(so))
     for fn in ("oracle_quantize_int8", "oracle_pack_int4", "oracle_unpack_int4", "oracle_route",
-               "oracle_forward", "oracle_expert_ffn", "oracle_num_threads"):
+               "oracle_forward", "oracle_expert_ffn", "oracle_num_threads", "oracle_quantize_tier",
+               "oracle_pack_int2", "oracle_unpack_int2"):
         getattr(mutant, fn).argtypes = getattr(real, fn).argtypes
         getattr(mutant, fn).restype = getattr(real, fn).restype
     monkeypatch.setattr(oracle, "_lib", mutant)

@@ -371,3 +371,115 @@ def test_missing_expert_is_reported():
     L = oracle_layer(cfg, experts=[0])
     with pytest.raises(RuntimeError):
         L.forward(syn.gen_x(cfg, 0))
+
+
+# ------------------------------------------------------------------------------------------
+# The int8 and packed int2 containers (colibri README, "What's implemented": int8 / packed
+# int4 / packed int2 quantisation, per-row scales, bit-identical to the int8 container)
+# ------------------------------------------------------------------------------------------
+
+def _crumbs(byte_values):
+    """2-bit two's-complement codes of each byte, lowest bits first (the golden layout rule)."""
+    b = np.asarray(byte_values, np.int64)
+    c = np.stack([(b >> (2 * i)) & 3 for i in range(4)], axis=-1)
+    return np.where(c >= 2, c - 4, c)
+
+
+def test_int2_crumb_layout_golden():
+    cases = _golden("int2_int8_tiers.json")["crumb_bytes"]["cases"]
+    packed = np.array([[c["byte"]] for c in cases], np.uint8)
+    q = oracle.unpack_int2(packed, 4)
+    assert q.tolist() == [c["codes"] for c in cases]
+
+
+def test_int2_unpack_is_exhaustive_and_pack_inverts_it():
+    packed = np.arange(256, dtype=np.uint8).reshape(256, 1)
+    q = oracle.unpack_int2(packed, 4)
+    assert np.array_equal(q, _crumbs(np.arange(256)))
+    assert q.min() == -2 and q.max() == 1 and len({tuple(r) for r in q.tolist()}) == 256
+    # re-quantising a row whose largest magnitude is 1 (scale 1) reproduces the byte whenever
+    # no code is -2 (the tier's rule never produces -2: |w / s| <= 1)
+    keep = (q != -2).all(axis=1)
+    rows = np.concatenate([q[keep].astype(np.float32), np.full((keep.sum(), 4), [1.0, 0, 0, 0], np.float32)], 1)
+    p, s = oracle.pack_int2(rows)
+    assert (s == 1.0).all()
+    assert (p[:, 0] == packed[keep, 0]).all() and (p[:, 1] == 1).all()
+
+
+@pytest.mark.parametrize("tier", ["int2_rows", "int8_rows"])
+def test_tier_quantiser_golden_rows(tier):
+    g = _golden("int2_int8_tiers.json")[tier]
+    bits = 2 if tier == "int2_rows" else 8
+    for case in g["cases"]:
+        w = np.array([case["w"]], np.float32)
+        q, s = oracle.quantize_tier(w, bits)
+        assert s[0] == np.float32(case["scale"]), case
+        assert q[0].tolist() == case["q"], case
+    for pk in g.get("packed", []):
+        w = np.array([g["cases"][pk["row"]]["w"]], np.float32)
+        p, _ = oracle.pack_int2(w)
+        assert p[0].tolist() == pk["bytes"], pk
+
+
+@pytest.mark.parametrize("shape", [(1, 4), (7, 64), (33, 132), (128, 1024)])
+def test_int2_packing_bit_identical_to_int8_container(shape):
+    rng = np.random.default_rng(sum(shape) + 2)
+    w = (rng.standard_normal(shape) * 0.02).astype(np.float32)
+    q8, s8 = oracle.quantize_tier(w, 2)
+    p, s2 = oracle.pack_int2(w)
+    assert (s2 == s8).all()
+    assert np.array_equal(oracle.unpack_int2(p, shape[1]), q8)
+    assert np.array_equal(_crumbs(p).reshape(shape), q8)         # the layout rule, decoded independently
+    assert q8.min() >= -1 and q8.max() <= 1
+    assert (s8 == np.abs(w).max(axis=1)).all()                     # scale = max|w| / 1
+
+
+def test_int4_tier_of_the_general_quantiser_is_the_int4_container_rule():
+    rng = np.random.default_rng(5)
+    w = (rng.standard_normal((40, 96)) * 0.02).astype(np.float32)
+    q4, s4 = oracle.quantize_int8(w)
+    q, s = oracle.quantize_tier(w, 4)
+    assert np.array_equal(q, q4) and np.array_equal(s, s4)
+
+
+def test_int8_tier_scale_and_range():
+    rng = np.random.default_rng(6)
+    w = (rng.standard_normal((40, 96)) * 0.02).astype(np.float32)
+    q, s = oracle.quantize_tier(w, 8)
+    assert (s == (np.abs(w).max(axis=1) / np.float32(127.0)).astype(np.float32)).all()
+    assert q.min() >= -127 and q.max() <= 127
+    assert (np.abs(q).max(axis=1) == 127).all()                   # the largest magnitude reaches qmax
+    # codes times scales reproduce w to within half a scale step
+    assert (np.abs(q * s[:, None].astype(np.float64) - w) <= 0.5 * s[:, None] * (1 + 1e-6)).all()
+
+
+def test_int2_container_forward_equals_int8_container_forward_bitwise():
+    """The packed int2 container and the int8 container holding the same int2-tier codes and
+    scales give the same layer output bit for bit (only the storage differs)."""
+    cfg = small_config("glm_decode", T=6, d=128, E=8, k=3, f=64, f_shared=32)
+    x = syn.gen_x(cfg, 0)
+    a = oracle_layer(cfg, wkind=oracle.W_INT2).forward(x)["out"]
+    b = oracle_layer(cfg, wkind=oracle.W_INT8, bits=2).forward(x)["out"]
+    assert np.array_equal(a, b)
+
+
+def _dense_tier(layer, e, which, f):
+    """Dense fp64 weights of the int8 or packed int2 container, decoded without the oracle."""
+    ex = layer.shared if e == "shared" else layer.experts[e]
+    a = ex[which]
+    q = _crumbs(a).reshape(a.shape[0], -1) if layer.wkind == oracle.W_INT2 else a
+    return q.astype(np.float64) * ex[which + "_scale"].astype(np.float64)[:, None]
+
+
+@pytest.mark.parametrize("wkind,bits", [(oracle.W_INT2, 2), (oracle.W_INT8, 8)])
+def test_single_expert_layer_is_textbook_swiglu_other_tiers(wkind, bits):
+    cfg = small_config("tiny", T=5, d=96, E=1, k=1, f=40, wkind=wkind)
+    L = oracle_layer(cfg, bits=bits)
+    x = syn.gen_x(cfg, 0)
+    out = L.forward(x)["out"]
+    wgu = torch.from_numpy(_dense_tier(L, 0, "gate_up", cfg.f))
+    wd = torch.from_numpy(_dense_tier(L, 0, "down", cfg.f))
+    xt = torch.from_numpy(syn.bf16_bits_to_fp32(x).astype(np.float64))
+    gate, up = wgu[:cfg.f], wgu[cfg.f:]
+    ref = (torch.nn.functional.silu(xt @ gate.T) * (xt @ up.T)) @ wd.T
+    np.testing.assert_allclose(out, ref.numpy(), rtol=1e-11, atol=1e-13)
