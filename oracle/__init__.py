@@ -49,6 +49,7 @@ class _Layer(ctypes.Structure):
         ("down", ctypes.c_void_p), ("down_scale", ctypes.c_void_p),
         ("shared_gate_up", ctypes.c_void_p), ("shared_gate_up_scale", ctypes.c_void_p),
         ("shared_down", ctypes.c_void_p), ("shared_down_scale", ctypes.c_void_p),
+        ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32), ("top_p", ctypes.c_double),
     ]
 
 
@@ -175,7 +176,10 @@ class Layer:
 
     def __init__(self, d, f, E, k, router, scaling, wkind, router_w, router_bias=None,
                  experts: Optional[Dict[int, dict]] = None, shared: Optional[dict] = None,
-                 f_shared: Optional[int] = None):
+                 f_shared: Optional[int] = None, n_group: int = 1, topk_group: int = 1, top_p: float = 0.0):
+        """n_group / topk_group: group-limited selection (n_group > 1); top_p in (0, 1): adaptive
+        expert top-p (dropped experts come back as index -1 with weight 0)."""
+        self.n_group, self.topk_group, self.top_p = int(n_group), int(topk_group), float(top_p)
         self.d, self.f, self.E, self.k = d, f, E, k
         self.router, self.scaling, self.wkind = router, float(scaling), wkind
         self.router_w = np.ascontiguousarray(router_w, dtype=np.float32)
@@ -207,7 +211,8 @@ class Layer:
             down=ctypes.cast(arrs["down"], ctypes.c_void_p),
             down_scale=ctypes.cast(arrs["down_scale"], ctypes.c_void_p),
             shared_gate_up=_p(sh.get("gate_up")), shared_gate_up_scale=_p(sh.get("gate_up_scale")),
-            shared_down=_p(sh.get("down")), shared_down_scale=_p(sh.get("down_scale")))
+            shared_down=_p(sh.get("down")), shared_down_scale=_p(sh.get("down_scale")),
+            n_group=self.n_group, topk_group=self.topk_group, top_p=self.top_p)
 
     # ------------------------------------------------------------------------------
     def route(self, x_bits: np.ndarray):

@@ -62,6 +62,10 @@ typedef struct {
     const float *shared_gate_up_scale;
     const void *shared_down;
     const float *shared_down_scale;
+    /* router variants (colibri README: "noaux_tc" and the "--topp" adaptive expert top-p knob);
+     * n_group <= 1 and top_p outside (0, 1) leave the plain top-k router */
+    int32_t n_group, topk_group;
+    double top_p;
 } oracle_layer;
 
 /* ------------------------------------------------------------------------------------ */
@@ -224,6 +228,63 @@ void oracle_unpack_int2(const uint8_t *packed, int64_t rows, int64_t cols, int8_
 /* router                                                                                   */
 /* ------------------------------------------------------------------------------------ */
 
+/* Group-limited selection (the DeepSeek-V3 router, "noaux_tc", with n_group > 1): the experts
+ * form n_group contiguous groups of E / n_group; a group's score is the sum of its two largest
+ * keys (its only key for groups of one); the topk_group best groups (score descending, lower group
+ * index first on equal scores) stay selectable, and the experts of every other group are marked
+ * taken, i.e. excluded. */
+static void limit_groups(const oracle_layer *L, const double *key, unsigned char *taken)
+{
+    const int E = L->n_experts, G = L->n_group;
+    if (G <= 1) return;
+    const int per = E / G;
+    double score[64];
+    unsigned char keep[64];
+    for (int g = 0; g < G; ++g) {
+        double b1 = -INFINITY, b2 = -INFINITY;
+        for (int e = g * per; e < (g + 1) * per; ++e) {
+            if (key[e] > b1) { b2 = b1; b1 = key[e]; }
+            else if (key[e] > b2) b2 = key[e];
+        }
+        score[g] = per >= 2 ? b1 + b2 : b1;
+        keep[g] = 0;
+    }
+    for (int r = 0; r < L->topk_group; ++r) {
+        int best = -1;
+        for (int g = 0; g < G; ++g)
+            if (!keep[g] && (best < 0 || score[g] > score[best])) best = g;
+        keep[best] = 1;
+    }
+    for (int e = 0; e < E; ++e)
+        if (!keep[e / per]) taken[e] = 1;
+}
+
+/* Adaptive expert top-p: in rank order, the first m experts whose weights, as a share of the k
+ * weights' total, add up to at least p (1 <= m <= k) are kept; the others are dropped (index -1,
+ * weight 0) and the kept weights are scaled back up to the k weights' total. */
+static void apply_top_p(double p, int k, int32_t *idx, double *w)
+{
+    if (!(p > 0.0 && p < 1.0)) return;
+    double total = 0.0;
+    for (int r = 0; r < k; ++r) total += w[r];
+    double cum = 0.0;
+    int m = k;
+    for (int r = 0; r < k; ++r) {
+        cum += w[r];
+        if (cum / total >= p) { m = r + 1; break; }
+    }
+    double kept = 0.0;
+    for (int r = 0; r < m; ++r) kept += w[r];
+    for (int r = 0; r < k; ++r) {
+        if (r < m) {
+            w[r] = w[r] * (total / kept);
+        } else {
+            w[r] = 0.0;
+            idx[r] = -1;
+        }
+    }
+}
+
 /* Routes one token.  key/logit scratch of length E.  Writes idx[k] (rank order), w[k]
  * (fp64), and the gap between the k-th and (k+1)-th largest key (+inf when k == E). */
 static void route_token(const oracle_layer *L, const uint16_t *xt, double *logit, double *key,
@@ -243,6 +304,7 @@ static void route_token(const oracle_layer *L, const uint16_t *xt, double *logit
         }
         taken[e] = 0;
     }
+    limit_groups(L, key, taken);
     for (int r = 0; r < k; ++r) {
         int best = -1;
         for (int e = 0; e < E; ++e)
@@ -266,6 +328,7 @@ static void route_token(const oracle_layer *L, const uint16_t *xt, double *logit
         for (int r = 0; r < k; ++r) sum += exp(logit[idx[r]] - m);
         for (int r = 0; r < k; ++r) w[r] = L->scaling * exp(logit[idx[r]] - m) / sum;
     }
+    apply_top_p(L->top_p, k, idx, w);
 }
 
 int oracle_route(const oracle_layer *L, const uint16_t *x, int32_t T, int32_t *idx, double *w,
@@ -273,6 +336,9 @@ int oracle_route(const oracle_layer *L, const uint16_t *x, int32_t T, int32_t *i
 {
     const int E = L->n_experts;
     if (L->top_k < 1 || L->top_k > E || T < 0) return ORACLE_ERR_ARG;
+    if (L->n_group > 1 && (L->n_group > 64 || E % L->n_group || L->topk_group < 1 || L->topk_group > L->n_group ||
+                           L->topk_group * (E / L->n_group) < L->top_k))
+        return ORACLE_ERR_ARG;
     int rc = ORACLE_OK;
 #pragma omp parallel
     {
@@ -417,13 +483,15 @@ int oracle_forward(const oracle_layer *L, const uint16_t *x, int32_t T, int32_t 
             if (mode == ORACLE_MODE_PER_TOKEN) {
                 for (int r = 0; r < k && !rc; ++r) {
                     expert_ref ex;
+                    if (si[r] < 0) continue;          /* dropped by top-p */
                     if ((rc = get_expert(L, si[r], &ex))) break;
                     expert_apply(L, &ex, xd, NULL, NULL, h, y);
                     for (int j = 0; j < d; ++j) o[j] += sw[r] * y[j];
                 }
             } else {
                 for (int e = 0; e < E; ++e) gate[e] = 0.0;
-                for (int r = 0; r < k; ++r) gate[si[r]] = sw[r];
+                for (int r = 0; r < k; ++r)
+                    if (si[r] >= 0) gate[si[r]] = sw[r];
                 for (int e = 0; e < E && !rc; ++e) {
                     expert_ref ex;
                     if ((rc = get_expert(L, e, &ex))) break;
@@ -471,6 +539,7 @@ int oracle_forward(const oracle_layer *L, const uint16_t *x, int32_t T, int32_t 
             double *o = out + (int64_t)t * d;
             for (int j = 0; j < d; ++j) o[j] = 0.0;
             for (int r = 0; r < k; ++r) {
+                if (sorted_idx[(int64_t)t * k + r] < 0) continue;     /* dropped by top-p */
                 const double *ys = y_all + ((int64_t)t * slots + r) * d;
                 for (int j = 0; j < d; ++j) o[j] += sorted_w[(int64_t)t * k + r] * ys[j];
             }

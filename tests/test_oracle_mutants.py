@@ -41,6 +41,13 @@ MUTANTS = {
                                       "b |= (uint8_t)((q[r * cols + 4 * j + i] & 3) << (6 - 2 * i));"),
     "tier qmax off by one": ("const float qmax = (float)((1 << (bits - 1)) - 1);",
                              "const float qmax = (float)(1 << (bits - 1));"),
+    "group score is the best key only": ("score[g] = per >= 2 ? b1 + b2 : b1;", "score[g] = b1;"),
+    "equal group scores go to the higher group": (
+        "if (!keep[g] && (best < 0 || score[g] > score[best])) best = g;",
+        "if (!keep[g] && (best < 0 || score[g] >= score[best])) best = g;"),
+    "top-p needs a share above p": ("if (cum / total >= p) { m = r + 1; break; }",
+                                    "if (cum / total > p) { m = r + 1; break; }"),
+    "top-p keeps the weights unscaled": ("w[r] = w[r] * (total / kept);", "w[r] = w[r];"),
 }
 
 PIN_TESTS = [
@@ -61,6 +68,9 @@ PIN_TESTS = [
     lambda: pins.test_tier_quantiser_golden_rows("int8_rows"),
     lambda: pins.test_int2_packing_bit_identical_to_int8_container((33, 132)),
     lambda: pins.test_single_expert_layer_is_textbook_swiglu_other_tiers(oracle.W_INT2, 2),
+    lambda: pins.test_grouped_selection_golden(),
+    lambda: pins.test_grouped_selection_brute_force(oracle.ROUTER_SIGMOID),
+    lambda: pins.test_top_p_golden(),
 ]
 
 

@@ -483,3 +483,119 @@ def test_single_expert_layer_is_textbook_swiglu_other_tiers(wkind, bits):
     gate, up = wgu[:cfg.f], wgu[cfg.f:]
     ref = (torch.nn.functional.silu(xt @ gate.T) * (xt @ up.T)) @ wd.T
     np.testing.assert_allclose(out, ref.numpy(), rtol=1e-11, atol=1e-13)
+
+
+# ------------------------------------------------------------------------------------------
+# Router variants (colibri README: "noaux_tc" and the "--topp" adaptive expert top-p knob)
+# ------------------------------------------------------------------------------------------
+
+def _router_with_logits(logits, k, router=oracle.ROUTER_SOFTMAX, **kw):
+    """An oracle router whose logits for x = (1, 0) are exactly `logits` (fp32 values)."""
+    E = len(logits)
+    wr = np.zeros((E, 2), np.float32)
+    wr[:, 0] = np.asarray(logits, np.float32)
+    x = syn.fp32_to_bf16_bits(np.array([[1.0, 0.0]], np.float32))
+    L = oracle.Layer(2, 4, E, k, router, 1.0, oracle.W_INT4, wr, **kw)
+    return L, x
+
+
+def test_grouped_selection_golden():
+    g = _golden("router_variants.json")["grouped"]
+    L, x = _router_with_logits(g["logits"], g["k"], n_group=g["n_group"], topk_group=g["topk_group"])
+    r = L.route(x)
+    assert r["idx"][0].tolist() == g["idx"]
+    L0, _ = _router_with_logits(g["logits"], g["k"])
+    assert L0.route(x)["idx"][0].tolist() == g["ungrouped_idx"]
+    tie = _golden("router_variants.json")["grouped_tie"]
+    Lt, xt = _router_with_logits(tie["logits"], tie["k"], n_group=tie["n_group"], topk_group=tie["topk_group"])
+    assert Lt.route(xt)["idx"][0].tolist() == tie["idx"]
+    # the weights are the softmax over the chosen logits, as without groups
+    lg = np.array(g["logits"], np.float64)[g["idx"]]
+    np.testing.assert_allclose(r["w"][0], np.exp(lg - lg.max()) / np.exp(lg - lg.max()).sum(), rtol=1e-15)
+
+
+@pytest.mark.parametrize("router", [oracle.ROUTER_SOFTMAX, oracle.ROUTER_SIGMOID])
+def test_grouped_selection_brute_force(router):
+    """The kept groups maximise the summed group score over every topk_group-subset of groups, and
+    the chosen experts maximise the summed key over every k-subset of the kept groups' experts."""
+    E, G, TG, k = 16, 4, 2, 3
+    base = "tiny" if router == oracle.ROUTER_SOFTMAX else "glm_decode"
+    cfg = small_config(base, T=64, d=64, E=E, k=k, f=32, f_shared=32)
+    L = oracle.Layer(cfg.d, cfg.f, E, k, router, cfg.scaling, cfg.wkind, syn.gen_router_w(cfg),
+                     syn.gen_router_bias(cfg), n_group=G, topk_group=TG)
+    x = syn.gen_x(cfg, 0)
+    r = L.route(x)
+    per = E // G
+    for t in range(cfg.T):
+        lg = r["logits"][t]
+        key = lg if router == oracle.ROUTER_SOFTMAX else 1.0 / (1.0 + np.exp(-lg)) + L.router_bias.astype(np.float64)
+        gscore = [sum(sorted(key[g * per:(g + 1) * per])[-2:]) for g in range(G)]
+        best_groups = max(itertools.combinations(range(G), TG), key=lambda c: (sum(gscore[i] for i in c),
+                                                                              [-i for i in c]))
+        allowed = [e for g in best_groups for e in range(g * per, (g + 1) * per)]
+        best = max(itertools.combinations(allowed, k), key=lambda c: (sum(key[i] for i in c), [-i for i in c]))
+        assert sorted(r["idx"][t].tolist()) == sorted(best)
+        assert set(r["idx"][t].tolist()) <= set(allowed)
+
+
+def test_grouped_selection_reduces_to_plain_top_k():
+    cfg = small_config("glm_decode", T=20, d=64, E=32, k=4, f=32, f_shared=32)
+    args = (cfg.d, cfg.f, cfg.E, cfg.k, cfg.router, cfg.scaling, cfg.wkind, syn.gen_router_w(cfg),
+            syn.gen_router_bias(cfg))
+    x = syn.gen_x(cfg, 0)
+    plain = oracle.Layer(*args).route(x)
+    for G, TG in ((1, 1), (4, 4), (8, 8)):                 # one group, or every group kept
+        v = oracle.Layer(*args, n_group=G, topk_group=TG).route(x)
+        assert np.array_equal(v["idx"], plain["idx"]) and np.array_equal(v["w"], plain["w"])
+
+
+def test_top_p_golden():
+    g = _golden("router_variants.json")["top_p"]
+    for case in g["cases"]:
+        L, x = _router_with_logits(g["logits"], g["k"], top_p=case["p"])
+        r = L.route(x)
+        assert (r["idx"][0] >= 0).sum() == case["kept"], case
+        assert (r["idx"][0][case["kept"]:] == -1).all()
+        if "w" in case:
+            np.testing.assert_allclose(r["w"][0], case["w"], rtol=1e-15, atol=1e-300)
+        else:
+            L0, _ = _router_with_logits(g["logits"], g["k"])
+            assert np.array_equal(r["w"], L0.route(x)["w"])
+    tie = g["exact_tie"]
+    L, x = _router_with_logits(tie["logits"], tie["k"], top_p=tie["p"])
+    r = L.route(x)
+    assert (r["idx"][0] >= 0).sum() == tie["kept"] and r["w"][0].tolist() == tie["w"]
+
+
+@pytest.mark.parametrize("p", [0.3, 0.7, 0.9])
+def test_top_p_keeps_the_shortest_prefix_and_the_total(p):
+    cfg = small_config("glm_decode", T=40, d=64, E=32, k=8, f=32, f_shared=32)
+    args = (cfg.d, cfg.f, cfg.E, cfg.k, cfg.router, cfg.scaling, cfg.wkind, syn.gen_router_w(cfg),
+            syn.gen_router_bias(cfg))
+    x = syn.gen_x(cfg, 0)
+    plain = oracle.Layer(*args).route(x)
+    v = oracle.Layer(*args, top_p=p).route(x)
+    for t in range(cfg.T):
+        w0, i0 = plain["w"][t], plain["idx"][t]
+        m = int((v["idx"][t] >= 0).sum())
+        share = np.cumsum(w0) / w0.sum()
+        assert share[m - 1] >= p and (m == 1 or share[m - 2] < p)       # the shortest prefix
+        assert np.array_equal(v["idx"][t][:m], i0[:m]) and (v["idx"][t][m:] == -1).all()
+        np.testing.assert_allclose(v["w"][t][:m].sum(), cfg.scaling, rtol=1e-14)
+        np.testing.assert_allclose(v["w"][t][:m] / v["w"][t][0], w0[:m] / w0[0], rtol=1e-14)
+
+
+def test_top_p_forward_applies_only_the_kept_experts():
+    cfg = small_config("glm_decode", T=4, d=64, E=12, k=4, f=32, f_shared=48)
+    base = oracle_layer(cfg)
+    L = oracle.Layer(cfg.d, cfg.f, cfg.E, cfg.k, cfg.router, cfg.scaling, cfg.wkind, base.router_w,
+                     base.router_bias, experts=base.experts, shared=base.shared, f_shared=cfg.f_shared, top_p=0.5)
+    x = syn.gen_x(cfg, 0)
+    fw = L.forward(x)
+    assert (fw["idx"] < 0).any()                                          # some experts are dropped
+    for t in range(cfg.T):
+        kept = [(int(e), w) for e, w in zip(fw["idx"][t], fw["w"][t]) if e >= 0]
+        routed = sum(w * L.expert_ffn(e, x[t])["y"] for e, w in sorted(kept))
+        np.testing.assert_allclose(fw["out"][t], routed + L.expert_ffn("shared", x[t])["y"], rtol=1e-12, atol=1e-14)
+    u = L.forward(x, mode=oracle.MODE_UNION)
+    assert np.array_equal(u["out"], fw["out"])
