@@ -15,13 +15,19 @@ synthetic inputs of the pages' model shapes; no datasets or trained weights):
   granite      Granite-1B-a400m-like decode layer: T=1, d=1024, E=32, top-8 softmax, f=512 bf16
   tiny         T=4, d=256, E=8, top-2 softmax, f=128 int4
 
-Timing: CUDA events on the launching stream around every step; L2 is flushed (a 512 MiB
-write) between steps, outside the events.  Multi-GPU: one process per GPU, each a data-parallel
+The JSON line's top level is the headline workload (--workload, glm_decode by default); the
+other five workloads are measured in the same run and reported under "workloads", each with its
+own roofline, end-to-end figure and CPU baseline (--workloads none skips them).
+
+Timing: CUDA events on the launching stream around every step; between steps, outside the
+events, a read-only sweep of a 512 MiB buffer evicts L2 (it leaves no dirty lines behind, so no
+write-back lands inside the next step).  Multi-GPU: one process per GPU, each a data-parallel
 replica with its own token stream; value = all ranks' tokens / max over ranks of device time.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -47,8 +53,16 @@ WORKLOADS = {
     "glm_prefill": "GLM-5.2-like MoE layer prefill, T=2048, bf16 out",
     "granite": "Granite-1B-a400m-like MoE layer decode, T=1, d=1024, E=32, top-8 softmax, f=512 bf16",
     "tiny": "tiny MoE layer, T=4, d=256, E=8, top-2 softmax, f=128 int4",
+    "glm_decode_int8": "GLM-5.2-like MoE layer decode, T=1, experts in the int8 container (one code per byte)",
+    "glm_decode_int2": "GLM-5.2-like MoE layer decode, T=1, experts in the packed int2 container (four codes per byte)",
+    "glm_decode_variants": "GLM-5.2-like MoE layer decode, T=1, group-limited selection (8 groups, 4 kept) and "
+                           "adaptive expert top-p 0.7",
 }
-DEFAULT_STEPS = {"glm_decode": 2000, "glm_union2": 1000, "glm_union32": 200, "glm_prefill": 60, "granite": 2000,
+# layer options of workloads that use the router variants: (n_group, topk_group, top_p)
+ROUTER_VARIANTS = {"glm_decode_variants": (8, 4, 0.7)}
+WORKLOAD_ORDER = ["glm_decode", "glm_union2", "glm_union32", "glm_prefill", "glm_decode_variants", "granite", "tiny",
+                  "glm_decode_int8", "glm_decode_int2"]
+DEFAULT_STEPS = {"glm_decode_int8": 500, "glm_decode_int2": 500, "glm_decode_variants": 500, "glm_decode": 2000, "glm_union2": 1000, "glm_union32": 200, "glm_prefill": 60, "granite": 2000,
                  "tiny": 200}
 FLUSH_BYTES = 512 << 20
 # The Granite layer's 32 experts (100 MB of bf16) fit in L2, so its token stream is also timed
@@ -72,23 +86,45 @@ def parse():
                     help="single-token path: 2 one launch, 1 three kernels, 0 general kernels (default: the library's)")
     ap.add_argument("--experts", type=int, default=None,
                     help="override E (smaller device footprint for profiler captures; same per-token work)")
+    ap.add_argument("--workloads", default="all",
+                    help="workloads measured besides the headline one: all, none, or a comma-separated list")
     ap.add_argument("--warm-passes", default=None, choices=["none", "stream", "graph", "both"],
                     help="extra L2-warm passes (no flush between steps; not HBM figures): the steps as plain "
                          "stream launches, replayed from one CUDA graph, or both (default: both for granite)")
     a = ap.parse_args()
+    a.steps_given = a.steps
     if a.steps is None:
         a.steps = DEFAULT_STEPS[a.workload]
-    if a.warm_passes is None:
-        a.warm_passes = DEFAULT_WARM_PASSES.get(a.workload, "none")
     a.warmup = max(a.warmup, 3)
     return a
 
 
+# columns per byte of a weight row, per container (bf16 is 2 bytes per column, no scales)
+CODES_PER_BYTE = {syn.W_INT4: 2, syn.W_INT8: 1, syn.W_INT2: 4}
+
+
+def row_bytes(cfg, cols) -> int:
+    """Bytes of one weight row of `cols` columns, with its fp32 scale when the container has one."""
+    if cfg.wkind == syn.W_BF16:
+        return cols * 2
+    return cols // CODES_PER_BYTE[cfg.wkind] + 4
+
+
 def expert_bytes(cfg, f=None) -> int:
     f = cfg.f if f is None else f
-    if cfg.wkind == syn.W_INT4:
-        return 2 * f * (cfg.d // 2 + 4) + cfg.d * (f // 2 + 4)
-    return 2 * f * cfg.d * 2 + cfg.d * f * 2
+    return 2 * f * row_bytes(cfg, cfg.d) + cfg.d * row_bytes(cfg, f)
+
+
+def workload_config(name):
+    """The layer configuration of a workload: the five synthetic configurations, and the GLM decode
+    layer in the int8 and packed int2 containers."""
+    if name in syn.CONFIGS:
+        return syn.CONFIGS[name]
+    if name in ROUTER_VARIANTS:
+        return dataclasses.replace(syn.CONFIGS["glm_decode"], name=name)
+    base, kind = name.rsplit("_", 1)
+    return dataclasses.replace(syn.CONFIGS[base], name=name,
+                               wkind={"int8": syn.W_INT8, "int2": syn.W_INT2}[kind])
 
 
 # ------------------------------------------------------------------------------------------
@@ -101,17 +137,21 @@ def build_device_layer(cfg, seed, max_tokens, device):
     import quantized_expert_ffn_02_b200 as qe
 
     E, d, f = cfg.E, cfg.d, cfg.f
-    int4 = cfg.wkind == syn.W_INT4
+    int4 = cfg.wkind != syn.W_BF16       # a container of codes with per-row scales
     W = {}
+    if int4:
+        cpb = CODES_PER_BYTE[cfg.wkind]
+        dt = torch.int8 if cfg.wkind == syn.W_INT8 else torch.uint8
+        packer = {syn.W_INT4: qe.moe_pack_int4, syn.W_INT8: qe.moe_pack_int8, syn.W_INT2: qe.moe_pack_int2}[cfg.wkind]
 
     def mat(name, rows, cols):
         return syn.torch_normal_fp32(seed, name, rows * cols, syn.WEIGHT_STD, device).view(rows, cols)
 
     def alloc(prefix, n, f_):
         if int4:
-            W[prefix + "gate_up"] = torch.empty((n, 2 * f_, d // 2), dtype=torch.uint8, device=device)
+            W[prefix + "gate_up"] = torch.empty((n, 2 * f_, d // cpb), dtype=dt, device=device)
             W[prefix + "gate_up_scale"] = torch.empty((n, 2 * f_), dtype=torch.float32, device=device)
-            W[prefix + "down"] = torch.empty((n, d, f_ // 2), dtype=torch.uint8, device=device)
+            W[prefix + "down"] = torch.empty((n, d, f_ // cpb), dtype=dt, device=device)
             W[prefix + "down_scale"] = torch.empty((n, d), dtype=torch.float32, device=device)
         else:
             W[prefix + "gate_up"] = torch.empty((n, 2 * f_, d), dtype=torch.int16, device=device)
@@ -121,7 +161,7 @@ def build_device_layer(cfg, seed, max_tokens, device):
         for which, rows, cols in (("gate_up", 2 * f_, d), ("down", d, f_)):
             w = mat(syn.expert_tensor_name(e, which), rows, cols)
             if int4:
-                qe.moe_pack_int4(w, W[prefix + which][i], W[prefix + which + "_scale"][i])
+                packer(w, W[prefix + which][i], W[prefix + which + "_scale"][i])
             else:
                 W[prefix + which][i].copy_(w.to(torch.bfloat16).view(torch.int16))
 
@@ -138,9 +178,14 @@ def build_device_layer(cfg, seed, max_tokens, device):
     b = syn.gen_router_bias(cfg, seed)
     W["router_bias"] = None if b is None else torch.from_numpy(b).to(device)
     torch.cuda.synchronize()
-    layer = qe.MoELayer(d, f, E, cfg.k, max_tokens, cfg.router, cfg.wkind, W, n_shared=cfg.n_shared,
-                        f_shared=cfg.f_shared, routed_scaling_factor=cfg.scaling, out_bf16=cfg.out_bf16)
-    return layer, W
+    return layer_on(cfg, W, max_tokens), W
+
+
+def layer_on(cfg, W, max_tokens):
+    """A layer handle over already-resident weights (several handles may share one set)."""
+    import quantized_expert_ffn_02_b200 as qe
+    return qe.MoELayer(cfg.d, cfg.f, cfg.E, cfg.k, max_tokens, cfg.router, cfg.wkind, W, n_shared=cfg.n_shared,
+                       f_shared=cfg.f_shared, routed_scaling_factor=cfg.scaling, out_bf16=cfg.out_bf16)
 
 
 def make_batches(cfg, T, n, seed, token_offset, device):
@@ -248,9 +293,12 @@ class Clocks:
 def oracle_sample_layer(cfg, seed, x_bits):
     """Oracle layer holding the experts that the sample's tokens route to (host-drawn)."""
     import oracle
+    G, TG, p = ROUTER_VARIANTS.get(cfg.name, (1, 1, 0.0))
+    variants = {"n_group": G, "topk_group": TG, "top_p": p}
     router = oracle.Layer(cfg.d, cfg.f, cfg.E, cfg.k, cfg.router, cfg.scaling, cfg.wkind,
-                          syn.gen_router_w(cfg, seed), syn.gen_router_bias(cfg, seed), f_shared=cfg.f_shared or cfg.f)
-    need = sorted(set(router.route(x_bits)["idx"].reshape(-1).tolist()))
+                          syn.gen_router_w(cfg, seed), syn.gen_router_bias(cfg, seed), f_shared=cfg.f_shared or cfg.f,
+                          **variants)
+    need = sorted(e for e in set(router.route(x_bits)["idx"].reshape(-1).tolist()) if e >= 0)
 
     def host_expert(e):
         out = {}
@@ -258,6 +306,10 @@ def oracle_sample_layer(cfg, seed, x_bits):
             w = syn.gen_expert_fp32(cfg, e, which, seed)
             if cfg.wkind == syn.W_BF16:
                 out[which] = syn.fp32_to_bf16_bits(w)
+            elif cfg.wkind == syn.W_INT8:
+                out[which], out[which + "_scale"] = oracle.quantize_tier(w, 8)
+            elif cfg.wkind == syn.W_INT2:
+                out[which], out[which + "_scale"] = oracle.pack_int2(w)
             else:
                 out[which], out[which + "_scale"] = oracle.pack_int4(w)
         return out
@@ -265,7 +317,7 @@ def oracle_sample_layer(cfg, seed, x_bits):
     experts = {e: host_expert(e) for e in need}
     shared = host_expert("shared") if cfg.n_shared else None
     return oracle.Layer(cfg.d, cfg.f, cfg.E, cfg.k, cfg.router, cfg.scaling, cfg.wkind, router.router_w,
-                        router.router_bias, experts=experts, shared=shared, f_shared=cfg.f_shared or cfg.f)
+                        router.router_bias, experts=experts, shared=shared, f_shared=cfg.f_shared or cfg.f, **variants)
 
 
 def oracle_sample_tokens(cfg, name):
@@ -325,10 +377,9 @@ def kernel_work(cfg, T, n_unique):
     S = 1 if cfg.n_shared else 0
     slots = T * cfg.k + T * S
     fmax = max(cfg.f, cfg.f_shared if S else 0)
-    q = cfg.wkind == syn.W_INT4
     gu_rows = n_unique * 2 * cfg.f + S * 2 * cfg.f_shared
-    gu = gu_rows * ((cfg.d // 2 + 4) if q else cfg.d * 2) + T * cfg.d * 2 + slots * fmax * 2
-    f_of = lambda ff: (ff // 2 + 4) if q else ff * 2  # noqa: E731
+    gu = gu_rows * row_bytes(cfg, cfg.d) + T * cfg.d * 2 + slots * fmax * 2
+    f_of = lambda ff: row_bytes(cfg, ff)  # noqa: E731
     dn_w = n_unique * cfg.d * f_of(cfg.f) + S * cfg.d * f_of(cfg.f_shared) + slots * fmax * 2
     # the single-token kernel adds the slots itself and writes the output; the others write y per slot
     dn = dn_w + (T * cfg.d * 4 if T == 1 else slots * cfg.d * 4)
@@ -382,7 +433,7 @@ def run_reference(a, rank, world):
     """The oracle on host cores: each step one bounded oracle call of the workload."""
     if rank != 0:
         return
-    cfg = syn.CONFIGS[a.workload]
+    cfg = workload_config(a.workload)
     import oracle
     n_tok = oracle_sample_tokens(cfg, a.workload)
     x = syn.gen_x(cfg, a.seed, T=n_tok)
@@ -405,34 +456,24 @@ def run_reference(a, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def run_ours(a, rank, world, local_rank):
+def measure_workload(a, name, cfg, layer, dev, dist, world, rank, local_rank, flush, cpu_budget):
+    """Times one workload on an existing layer; returns its part of the JSON line."""
     import torch
-
-    import dataclasses
 
     import quantized_expert_ffn_02_b200 as qe
 
-    cfg = syn.CONFIGS[a.workload]
-    if a.experts:
-        cfg = dataclasses.replace(cfg, E=a.experts)
-    if a.tokens:
-        cfg = dataclasses.replace(cfg, T=a.tokens)
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     T = cfg.T
-    layer, W = build_device_layer(cfg, a.seed, T, dev)
     if a.t1_mode is not None:
         layer.set_single_token_mode(a.t1_mode)
+    if name in ROUTER_VARIANTS:
+        G, TG, p = ROUTER_VARIANTS[name]
+        layer.set_router_groups(G, TG)
+        layer.set_router_top_p(p)
     # every rank is an independent replica with its own tokens
     n_batches = a.warmup + a.steps if T <= 32 else 4
     token_base = replica_token_base(rank)
     xs = make_batches(cfg, T, n_batches, a.seed, token_base, dev)
     out = torch.empty((T, cfg.d), dtype=torch.int16 if cfg.out_bf16 else torch.float32, device=dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     # census of unique experts per batch (outside timing) for the algorithmic byte counts
@@ -441,7 +482,7 @@ def run_ours(a, rank, world, local_rank):
     wts = torch.empty((T, cfg.k), dtype=torch.float32, device=dev)
     for x in xs:
         layer.route(x, idx, wts)
-        uniq.append(len(torch.unique(idx).tolist()))
+        uniq.append(len([e for e in torch.unique(idx).tolist() if e >= 0]))     # -1: dropped by top-p
     torch.cuda.synchronize()
 
     def bx(i):
@@ -451,7 +492,7 @@ def run_ours(a, rank, world, local_rank):
         layer.forward(bx(i), out)
     torch.cuda.synchronize()
     if layer.last_error() != qe.MOE_OK:
-        raise RuntimeError("device status after warm-up: " + qe.status_str(layer.last_error()))
+        raise RuntimeError(f"{name}: device status after warm-up: " + qe.status_str(layer.last_error()))
     launches_per_step = layer.last_launches()
 
     def timed_pass(profile: bool):
@@ -461,7 +502,7 @@ def run_ours(a, rank, world, local_rank):
             dist.barrier()
         torch.cuda.synchronize()
         for i in range(a.steps):
-            flush.zero_()
+            flush()
             evs[i][0].record(stream)
             layer.forward(bx(a.warmup + i), out)
             evs[i][1].record(stream)
@@ -479,14 +520,15 @@ def run_ours(a, rank, world, local_rank):
     prof_ms = sum(timed_pass(True))
     prof = layer.profile_read()
     if layer.last_error() != qe.MOE_OK:
-        raise RuntimeError("device status after timing: " + qe.status_str(layer.last_error()))
+        raise RuntimeError(f"{name}: device status after timing: " + qe.status_str(layer.last_error()))
     total_ms = slowest_rank_ms(total_ms, dist, dev)
     value = job_tokens_per_s(world, a.steps, T, total_ms)
 
     # end to end: host buffers through the C ABI, copies inside the timed region.  Every step
     # copies its x in from pinned host memory and its output back out.  The calls are enqueued
-    # back to back (moe_forward_host_async) and the host waits once at the end; the form that
-    # waits after every step (moe_forward_host) is timed beside it.
+    # back to back (moe_forward_host_async) and the host waits once at the end, as a serving loop
+    # would; L2 is not flushed between these steps.  The form that waits after every step
+    # (moe_forward_host) is timed beside it.
     xh = [bx(a.warmup + i).cpu().pin_memory() for i in range(min(a.steps, len(xs)))]
     oh = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
     e2e_steps = a.steps
@@ -506,17 +548,18 @@ def run_ours(a, rank, world, local_rank):
         t1.record(stream)
         torch.cuda.synchronize()
         if layer.last_error() != qe.MOE_OK:
-            raise RuntimeError("device status after the end-to-end pass: " + qe.status_str(layer.last_error()))
+            raise RuntimeError(f"{name}: device status after the end-to-end pass: " +
+                               qe.status_str(layer.last_error()))
         return slowest_rank_ms(t0.elapsed_time(t1), dist, dev)
 
     sync_ms = e2e_pass(False)
     try:
         e2e_ms, e2e_api = e2e_pass(True), "moe_forward_host_async, one wait at the end"
-    except (RuntimeError, AttributeError) as exc:      # an older library without the call
-        e2e_ms, e2e_api = sync_ms, "moe_forward_host (the pipelined form failed: %s)" % str(exc).splitlines()[0][:120]
+    except AttributeError as exc:      # an older library without the call
+        e2e_ms, e2e_api = sync_ms, "moe_forward_host (no pipelined call: %s)" % str(exc).splitlines()[0][:120]
     e2e = {"value": job_tokens_per_s(world, e2e_steps, T, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": T * cfg.d * 2, "d2h_bytes_per_step": T * cfg.d * out.element_size(),
-           "api": e2e_api,
+           "api": e2e_api, "l2": "not flushed between steps (back-to-back serving loop)",
            "wait_every_step": {"value": job_tokens_per_s(world, e2e_steps, T, sync_ms), "unit": "tokens/s",
                                "api": "moe_forward_host"}}
 
@@ -546,15 +589,16 @@ def run_ours(a, rank, world, local_rank):
         if g is not None:
             g.reset()
         if layer.last_error() != qe.MOE_OK:
-            raise RuntimeError("device status after an L2-warm pass: " + qe.status_str(layer.last_error()))
+            raise RuntimeError(f"{name}: device status after an L2-warm pass: " + qe.status_str(layer.last_error()))
         return {"value": job_tokens_per_s(world, a.steps, T, ms), "unit": "tokens/s", "ms_per_step": ms / a.steps,
                 "steps": a.steps, "launch": "one CUDA graph" if graph else "stream launches",
                 "l2": "warm: no flush between steps, not an HBM figure"}
 
+    warm_mode = a.warm_passes if a.warm_passes is not None else DEFAULT_WARM_PASSES.get(name, "none")
     warm = {}
-    if a.warm_passes in ("stream", "both"):
+    if warm_mode in ("stream", "both"):
         warm["stream"] = warm_pass(False)
-    if a.warm_passes in ("graph", "both"):
+    if warm_mode in ("graph", "both"):
         try:
             warm["graph"] = warm_pass(True)
         except RuntimeError as exc:                # a capture the runtime refused: report it
@@ -588,13 +632,15 @@ def run_ours(a, rank, world, local_rank):
     step_bytes = statistics.mean(uniq[(a.warmup + i) % len(xs)] for i in range(a.steps)) * expert_bytes(cfg) + \
         (expert_bytes(cfg, cfg.f_shared) if cfg.n_shared else 0) + cfg.E * cfg.d * 4
     ms_per_step = total_ms / a.steps
-    line = {
+    res = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
-        "ms_per_step": ms_per_step, "step_ms_percentiles": step_percentiles(step_ms), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int4xbf16->f32" if cfg.wkind == syn.W_INT4 else "bf16->f32", "data": "synthetic",
-        "config": {"workload": a.workload, "desc": WORKLOADS[a.workload], "tokens_per_step": T,
+        "ms_per_step": ms_per_step, "step_ms_percentiles": step_percentiles(step_ms), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": {syn.W_INT4: "int4xbf16->f32", syn.W_INT8: "int8xbf16->f32", syn.W_INT2: "int2xbf16->f32"}.get(
+            cfg.wkind, "bf16->f32"), "data": "synthetic",
+        "config": {"workload": name, "desc": WORKLOADS[name], "tokens_per_step": T,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "flushed between steps (512 MiB write, outside the step events)",
+                   "l2": "evicted between steps by a read-only sweep of a 512 MiB buffer, outside the step events",
                    "weights": "seed 0, drawn on the device by the counter-based generator"},
         "roofline": roof,
         "step_hbm": {"gbs": step_bytes / (ms_per_step / 1e3) / 1e9, "frac": step_bytes / (ms_per_step / 1e3) / 1e9 / hbm,
@@ -605,13 +651,80 @@ def run_ours(a, rank, world, local_rank):
         "gpu_launches": launches_per_step * a.steps,
         "clocks": clk,
     }
+    if cfg.wkind == syn.W_INT4 and T >= 128 and "gemm_gateup" in prof:
+        flops = 2 * T * (cfg.k * 3 * cfg.d * cfg.f + (3 * cfg.d * cfg.f_shared if cfg.n_shared else 0))
+        res["step_tensor"] = {"tflops": flops / (ms_per_step / 1e3) / 1e12,
+                              "frac": flops / (ms_per_step / 1e3) / 1e12 / tf, "flops_per_step": flops,
+                              "peak": tf, "peak_kind": f"{peak_kind} bf16 dense (burst)"}
     if warm:
-        line["l2_warm"] = warm
+        res["l2_warm"] = warm
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg, a.workload, a.seed, a.cpu_seconds)
+        res["cpu_baseline"] = cpu_baseline(cfg, name, a.seed, cpu_budget)
+    return res
+
+
+def selected_workloads(a):
+    if a.workloads == "none":
+        extra = []
+    elif a.workloads == "all":
+        extra = [n for n in WORKLOAD_ORDER if n != a.workload]
+    else:
+        extra = [n.strip() for n in a.workloads.split(",") if n.strip() and n.strip() != a.workload]
+        for n in extra:
+            if n not in WORKLOADS:
+                raise SystemExit(f"unknown workload {n}")
+    return [a.workload] + extra
+
+
+def run_ours(a, rank, world, local_rank):
+    import torch
+
+    import dataclasses
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    flush_buf = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def flush():
+        flush_buf.sum()          # reads 512 MiB: every line of L2 is replaced by a clean one
+
+    names = selected_workloads(a)
+    # workloads over the same weights (the four int4 GLM workloads) share one resident copy of the
+    # experts (4.8 GB); each gets a layer handle with its own token limit and output type
+    def weight_key(n):
+        c = workload_config(n)
+        return (c.d, c.E, c.f, c.wkind, c.router)
+    results = {}
+    first_sharer = {n: next(m for m in WORKLOAD_ORDER if weight_key(m) == weight_key(n)) for n in names}
+    order = sorted(names, key=lambda n: (WORKLOAD_ORDER.index(first_sharer[n]), WORKLOAD_ORDER.index(n)))
+    held = (None, None)
+    for i, name in enumerate(order):
+        cfg = workload_config(name)
+        if a.experts:
+            cfg = dataclasses.replace(cfg, E=a.experts)
+        if a.tokens and name == a.workload:
+            cfg = dataclasses.replace(cfg, T=a.tokens)
+        if held[0] == weight_key(name):
+            layer = layer_on(cfg, held[1], cfg.T)
+        else:
+            held = (None, None)
+            torch.cuda.empty_cache()
+            layer, W = build_device_layer(cfg, a.seed, cfg.T, dev)
+            held = (weight_key(name), W)
+        budget = a.cpu_seconds if name == a.workload else a.cpu_seconds / 3
+        aw = a if a.steps_given is not None else argparse.Namespace(**{**vars(a), "steps": DEFAULT_STEPS[name]})
+        results[name] = measure_workload(aw, name, cfg, layer, dev, dist, world, rank, local_rank, flush, budget)
+        layer.close()
+    held = (None, None)
+    line = results.pop(a.workload)
+    if results:
+        line["workloads"] = results
     if rank == 0:
         print(json.dumps(line), flush=True)
-    layer.close()
     if dist:
         dist.barrier()
         dist.destroy_process_group()

@@ -28,9 +28,11 @@
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default stream).  Only
  *     the calls documented as synchronous wait for the device.
  *   - No C++ exception or CUDA error escapes: every failure is a moe_status.  Argument errors
- *     are returned before anything is enqueued.  Errors found by the device while running
- *     (a bounded wait that ran out, a value out of range) are latched in the layer's device
- *     status word and returned by moe_last_error().
+ *     are returned before anything is enqueued.  moe_route, moe_forward and moe_route_noalloc
+ *     first clear an error that an earlier, unrelated runtime call left pending (the CUDA
+ *     runtime's last-error state), so that they report only their own launches.  Errors found
+ *     by the device while running (a bounded wait that ran out, a value out of range) are
+ *     latched in the layer's device status word and returned by moe_last_error().
  *   - The library never allocates on the hot path: moe_route / moe_forward use the workspace
  *     that moe_layer_create allocated for `max_tokens` tokens.
  */
@@ -57,7 +59,12 @@ typedef enum {
 } moe_status;
 
 enum { MOE_ROUTER_SOFTMAX_TOPK = 0, MOE_ROUTER_SIGMOID_BIAS = 1 };
-enum { MOE_W_INT4_ROWSCALE = 0, MOE_W_BF16 = 1 };
+/* Weight containers (colibri README, "What's implemented": int8 / packed int4 / packed int2
+ * quantisation with per-row scales, dequant-on-use): packed int4 (two codes per byte), bf16,
+ * int8 (one code of the 8-bit tier per byte), packed int2 (four codes of the 2-bit tier per
+ * byte).  The int8 and int2 containers run on the general decode kernels at every batch size;
+ * the single-launch decode path and the tcgen05 grouped GEMMs take packed int4. */
+enum { MOE_W_INT4_ROWSCALE = 0, MOE_W_BF16 = 1, MOE_W_INT8_ROWSCALE = 2, MOE_W_INT2_ROWSCALE = 3 };
 
 typedef struct {
     int32_t d;                   /* hidden size; even, and a multiple of 64 */
@@ -83,6 +90,10 @@ typedef struct {
  *     gate_up        [E][2f][d/2] bytes     gate_up_scale [E][2f] fp32
  *     down           [E][d][f/2]  bytes     down_scale    [E][d]  fp32
  *   bf16 (MOE_W_BF16): gate_up [E][2f][d], down [E][d][f]; the scale pointers are ignored.
+ *   int8 (MOE_W_INT8_ROWSCALE): the output of moe_pack_int8 -- gate_up [E][2f][d] int8,
+ *     down [E][d][f] int8, scales as for int4.
+ *   int2 (MOE_W_INT2_ROWSCALE): the output of moe_pack_int2 -- gate_up [E][2f][d/4] bytes,
+ *     down [E][d][f/4] bytes, scales as for int4.
  *   shared_*: the same for the single shared expert (with f_shared in place of f), or NULL
  *   when n_shared == 0.
  *   router_w [E][d] fp32; router_bias [E] fp32 for the sigmoid router (NULL means zeros).
@@ -119,6 +130,21 @@ moe_status moe_pack_int4(const float *w, int64_t rows, int64_t cols, uint8_t *pa
                          moe_stream stream);
 
 /*
+ * moe_pack_int8 / moe_pack_int2 -- the 8-bit and 2-bit tiers of the same per-row rule (colibri
+ * README, "What's implemented": int8 / packed int4 / packed int2 quantisation, per-row scales):
+ * qmax = 2^(b-1) - 1 (127 or 1); scale = fp32(max|w| / qmax); q = clamp(round-half-even(fp32(w /
+ * scale)), -qmax - 1, qmax); a row of zeros has scale 0 and codes 0.
+ *   moe_pack_int8: q device [rows][cols] int8, one code per byte; cols > 0.
+ *   moe_pack_int2: packed device [rows][cols/4] bytes, column 4j + i of a row in bits 2i .. 2i+1 of
+ *                  byte j (a 2-bit two's-complement code); cols a multiple of 4.
+ *   w device [rows][cols] fp32; scales device [rows] fp32 (written).  Errors and synchronisation
+ *   as for moe_pack_int4 (non-finite input: MOE_ERR_RANGE, its codes written as 0).
+ */
+moe_status moe_pack_int8(const float *w, int64_t rows, int64_t cols, int8_t *q, float *scales, moe_stream stream);
+moe_status moe_pack_int2(const float *w, int64_t rows, int64_t cols, uint8_t *packed, float *scales,
+                         moe_stream stream);
+
+/*
  * moe_layer_create -- validate the configuration, borrow the weights, and allocate the
  * workspace for cfg->max_tokens tokens on the current CUDA device.  *out is set only on
  * success.  Errors: MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_OOM, MOE_ERR_CUDA.
@@ -128,8 +154,10 @@ moe_status moe_layer_create(const moe_config *cfg, const moe_weights *w, moe_lay
 /*
  * moe_route -- router and top-k only (step 1 above).
  *   x    device, [T][d] bf16
- *   idx  device, [T][k] int32 (written): chosen experts in rank order
- *   w    device, [T][k] fp32 (written): their gate weights (computed in fp64, rounded once)
+ *   idx  device, [T][k] int32 (written): chosen experts in rank order (-1 where adaptive top-p,
+ *        MOE_OPT_ROUTER_TOP_P, dropped one)
+ *   w    device, [T][k] fp32 (written): their gate weights (computed in fp64, rounded once; 0 for
+ *        a dropped expert)
  *   0 <= T <= max_tokens.  Asynchronous.  The logits are accumulated in fp64.
  */
 moe_status moe_route(moe_layer *layer, const uint16_t *x, int32_t T, int32_t *idx, float *w,
@@ -143,6 +171,23 @@ moe_status moe_route(moe_layer *layer, const uint16_t *x, int32_t T, int32_t *id
  *   one layer must not overlap on the device (they share its workspace).
  */
 moe_status moe_forward(moe_layer *layer, const uint16_t *x, int32_t T, void *out, moe_stream stream);
+
+/*
+ * moe_layer_set_expert -- point routed expert e (0 <= e < E) at weights anywhere in device memory:
+ * a ragged table of experts in place of one contiguous [E] array (iliria page, "What's
+ * implemented": grouped MoE over a ragged descriptor of expert slabs; colibri README, "The idea":
+ * experts streamed on demand).  gate_up, gate_up_scale, down, down_scale: device pointers in
+ * the layer's container format for ONE expert ([2f][...] rows, [2f] scales, [d][...] rows, [d]
+ * scales; the scale pointers are ignored for bf16 weights), 16-byte aligned, borrowed like the
+ * layer's other weights.  Asynchronous: the layer's device pointer table is updated on `stream`,
+ * in order with the forwards enqueued on that stream (order calls on other streams yourself).
+ * Once any expert has been re-pointed the tcgen05 grouped-GEMM path, whose tensor maps cover the
+ * contiguous arrays, is no longer used (MOE_OPT_PREFILL_AVAILABLE reads 0); every other path
+ * reads the table.  Errors: MOE_ERR_INVALID_ARG (index, NULL or misaligned pointer),
+ * MOE_ERR_CUDA.
+ */
+moe_status moe_layer_set_expert(moe_layer *layer, int32_t e, const void *gate_up, const float *gate_up_scale,
+                                const void *down, const float *down_scale, moe_stream stream);
 
 /*
  * moe_forward_host -- moe_forward on host buffers: copies x host->device, runs the layer,
@@ -202,8 +247,40 @@ void moe_layer_destroy(moe_layer *layer);
  *                               early with programmatic dependent launch and wait on the device
  *                               for their inputs; 0: ordinary stream order.  Same results.
  */
+/*   MOE_OPT_WAIT_LIMIT_US        time limit, in microseconds (100 .. 10,000,000; default 2,000,000), of
+ *                               every bounded device-side wait of the grouped-GEMM kernels.  When a
+ *                               wait runs out, the kernel latches MOE_ERR_TIMEOUT, lets the copies it
+ *                               issued land, frees its tensor memory and returns; moe_last_error
+ *                               reports it and the layer stays usable.  (The decode kernels keep a
+ *                               fixed 2 s limit.)
+ *   MOE_OPT_TEST_SKIP_GEMM_B_COPIES  test hook for that error path: 1 makes the grouped-GEMM kernels'
+ *                               activation-tile producer issue no copies, so the MMA warp's wait for
+ *                               them runs out after MOE_OPT_WAIT_LIMIT_US and the forward reports
+ *                               MOE_ERR_TIMEOUT (its output is then undefined); 0 (default) is normal
+ *                               operation.  Nothing faults or hangs: every waiter gives up within the
+ *                               limit.
+ */
+/*   MOE_OPT_ROUTER_GROUPS        group-limited selection (colibri README, "What's implemented": the
+ *                               DeepSeek-V3 router's noaux_tc): value = n_group + 65536 * topk_group.
+ *                               The E experts form n_group contiguous groups of E / n_group; a group's
+ *                               score is the sum of its two largest selection keys; only the
+ *                               topk_group best groups (equal scores: the lower group first) stay
+ *                               selectable, and the top-k runs over their experts.  Gate weights as
+ *                               without groups.  n_group = 1 (default) is the plain router;
+ *                               otherwise n_group <= 32, E % n_group == 0, 1 <= topk_group <= n_group
+ *                               and topk_group * E / n_group >= k.
+ *   MOE_OPT_ROUTER_TOP_P         adaptive expert top-p (colibri README, "Quick start": --topp), in
+ *                               millionths (0 .. 1,000,000; 0 and 1,000,000 = off, the default).  Of
+ *                               a token's k chosen experts, the shortest rank-order prefix whose gate
+ *                               weights reach p of the k weights' total is kept and rescaled to that
+ *                               total; the others are dropped: moe_route writes index -1 and weight
+ *                               0 for them, and moe_forward never reads their weights.
+ *   While either variant is on, T = 1 batches run on the general decode kernels (the single-token
+ *   paths take the plain router only).  moe_route_noalloc always uses the plain router.
+ */
 enum { MOE_OPT_PREFILL_MIN_TOKENS = 0, MOE_OPT_PREFILL_AVAILABLE = 1, MOE_OPT_SINGLE_TOKEN_KERNELS = 2,
-       MOE_OPT_PROGRAMMATIC_LAUNCH = 3 };
+       MOE_OPT_PROGRAMMATIC_LAUNCH = 3, MOE_OPT_WAIT_LIMIT_US = 4, MOE_OPT_TEST_SKIP_GEMM_B_COPIES = 5,
+       MOE_OPT_ROUTER_GROUPS = 6, MOE_OPT_ROUTER_TOP_P = 7 };
 moe_status moe_layer_set_option(moe_layer *layer, int32_t option, int64_t value);
 moe_status moe_layer_get_option(const moe_layer *layer, int32_t option, int64_t *value);
 
@@ -272,7 +349,9 @@ enum {
  * T*8 bytes of it; a larger request returns MOE_ERR_UNSUPPORTED (E = 256 allows T <= 510).
  * The first call on each device looks up that array's device address and sets the router
  * kernel's shared-memory limit (neither allocates); make that first call before any stream
- * capture.  Every call on a device shares the array and the array keeps the last call's
+ * capture.  The address is looked up once per device and kept until the process exits: it is
+ * not looked up again, so after cudaDeviceReset() on a device this entry point must not be
+ * called on that device again.  Every call on a device shares the array and the array keeps the last call's
  * contents (each call overwrites all it reads); calls that overlap on the GPU -- on different
  * streams, or from different host threads -- race on it.  Asynchronous; no allocation, no
  * synchronisation.

@@ -16,17 +16,18 @@ LIB_PATH = os.path.join(_HERE, "libmoe.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_CUDA, MOE_ERR_OOM, MOE_ERR_TIMEOUT, MOE_ERR_RANGE, MOE_ERR_UNSUPPORTED = range(7)
 MOE_ROUTER_SOFTMAX_TOPK, MOE_ROUTER_SIGMOID_BIAS = 0, 1
-MOE_W_INT4_ROWSCALE, MOE_W_BF16 = 0, 1
+MOE_W_INT4_ROWSCALE, MOE_W_BF16, MOE_W_INT8_ROWSCALE, MOE_W_INT2_ROWSCALE = 0, 1, 2, 3
 
 # Every symbol that include/moe.h declares.
 EXPORTS = (
-    "moe_pack_int4", "moe_layer_create", "moe_route", "moe_forward", "moe_forward_host", "moe_forward_host_async",
+    "moe_pack_int4", "moe_pack_int8", "moe_pack_int2", "moe_layer_create", "moe_route", "moe_forward", "moe_forward_host", "moe_forward_host_async",
     "moe_last_error",
     "moe_layer_destroy", "moe_layer_workspace_bytes", "moe_layer_last_launches", "moe_status_str",
     "moe_profile_enable", "moe_profile_read", "moe_kernel_name", "moe_route_noalloc",
-    "moe_layer_set_option", "moe_layer_get_option", "moe_layer_debug_read",
+    "moe_layer_set_option", "moe_layer_get_option", "moe_layer_debug_read", "moe_layer_set_expert",
 )
-MOE_OPT_PREFILL_MIN_TOKENS, MOE_OPT_PREFILL_AVAILABLE, MOE_OPT_SINGLE_TOKEN_KERNELS, MOE_OPT_PROGRAMMATIC_LAUNCH = 0, 1, 2, 3
+(MOE_OPT_PREFILL_MIN_TOKENS, MOE_OPT_PREFILL_AVAILABLE, MOE_OPT_SINGLE_TOKEN_KERNELS, MOE_OPT_PROGRAMMATIC_LAUNCH,
+ MOE_OPT_WAIT_LIMIT_US, MOE_OPT_TEST_SKIP_GEMM_B_COPIES, MOE_OPT_ROUTER_GROUPS, MOE_OPT_ROUTER_TOP_P) = range(8)
 DEBUG_ITEMS = {"h": 0, "y": 1, "idx": 2, "w": 3, "asc": 4, "ulist": 5, "cnt": 6, "xsum": 7, "trace": 8}
 KERNELS = ("router_logits", "topk", "bucket", "gateup", "down", "combine", "gather", "gemm_gateup", "gemm_down",
            "fused")
@@ -63,6 +64,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         L = ctypes.CDLL(path)
         P, I32, I64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
         L.moe_pack_int4.argtypes = [P, I64, I64, P, P, P]
+        L.moe_pack_int8.argtypes = [P, I64, I64, P, P, P]
+        L.moe_pack_int2.argtypes = [P, I64, I64, P, P, P]
         L.moe_layer_create.argtypes = [ctypes.POINTER(moe_config), ctypes.POINTER(moe_weights), ctypes.POINTER(P)]
         L.moe_route.argtypes = [P, P, I32, P, P, P]
         L.moe_forward.argtypes = [P, P, I32, P, P]
@@ -85,9 +88,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         L.moe_layer_set_option.argtypes = [P, I32, I64]
         L.moe_layer_get_option.argtypes = [P, I32, ctypes.POINTER(I64)]
         L.moe_layer_debug_read.argtypes = [P, I32, P, I64]
-        for n in ("moe_pack_int4", "moe_layer_create", "moe_route", "moe_forward", "moe_forward_host",
+        L.moe_layer_set_expert.argtypes = [P, I32, P, P, P, P, P]
+        for n in ("moe_pack_int4", "moe_pack_int8", "moe_pack_int2", "moe_layer_create", "moe_route", "moe_forward", "moe_forward_host",
                   "moe_forward_host_async", "moe_last_error", "moe_profile_enable", "moe_profile_read", "moe_route_noalloc",
-                  "moe_layer_set_option", "moe_layer_get_option", "moe_layer_debug_read"):
+                  "moe_layer_set_option", "moe_layer_get_option", "moe_layer_debug_read", "moe_layer_set_expert"):
             getattr(L, n).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -122,6 +126,18 @@ def moe_pack_int4(w, packed, scales, stream=None):
     rows, cols = w.shape
     _check(load().moe_pack_int4(_ptr(w), rows, cols, _ptr(packed), _ptr(scales), _stream(stream)),
            "moe_pack_int4")
+
+
+def moe_pack_int8(w, q, scales, stream=None):
+    """w fp32 [rows][cols] (CUDA) -> q int8 [rows][cols] (the 8-bit tier), scales fp32 [rows] (written)."""
+    rows, cols = w.shape
+    _check(load().moe_pack_int8(_ptr(w), rows, cols, _ptr(q), _ptr(scales), _stream(stream)), "moe_pack_int8")
+
+
+def moe_pack_int2(w, packed, scales, stream=None):
+    """w fp32 [rows][cols] (CUDA) -> packed uint8 [rows][cols/4] (the 2-bit tier), scales fp32 [rows]."""
+    rows, cols = w.shape
+    _check(load().moe_pack_int2(_ptr(w), rows, cols, _ptr(packed), _ptr(scales), _stream(stream)), "moe_pack_int2")
 
 
 def moe_layer_create(cfg: moe_config, weights: moe_weights) -> int:
@@ -197,6 +213,12 @@ def moe_layer_debug_read(layer: int, item: str, dst) -> None:
            "moe_layer_debug_read")
 
 
+def moe_layer_set_expert(layer: int, e: int, gate_up, gate_up_scale, down, down_scale, stream=None):
+    """Point routed expert e at one expert's device tensors (a ragged expert table; see moe.h)."""
+    _check(load().moe_layer_set_expert(layer, int(e), _ptr(gate_up), _ptr(gate_up_scale), _ptr(down),
+                                       _ptr(down_scale), _stream(stream)), "moe_layer_set_expert")
+
+
 def moe_route_noalloc(cfg: moe_config, router_w, router_bias, x, T: int, idx, w, stream=None):
     """Routing without any device allocation (for callers that may not allocate; see moe.h)."""
     _check(load().moe_route_noalloc(ctypes.byref(cfg), _ptr(router_w), _ptr(router_bias), _ptr(x), T, _ptr(idx),
@@ -255,6 +277,14 @@ class MoELayer:
 
     def debug_read(self, item: str, dst):
         moe_layer_debug_read(self.handle, item, dst)
+
+    def set_router_groups(self, n_group: int, topk_group: int):
+        """Group-limited selection (n_group = 1: the plain router)."""
+        moe_layer_set_option(self.handle, MOE_OPT_ROUTER_GROUPS, int(n_group) + (int(topk_group) << 16))
+
+    def set_router_top_p(self, p: float):
+        """Adaptive expert top-p (0 or 1: off)."""
+        moe_layer_set_option(self.handle, MOE_OPT_ROUTER_TOP_P, int(round(p * 1e6)))
 
     def set_prefill_min_tokens(self, n: int):
         moe_layer_set_option(self.handle, MOE_OPT_PREFILL_MIN_TOKENS, n)

@@ -5,7 +5,8 @@
 // (token, rank) entries routed to it.  The iliria page ("What's implemented": grouped CPU MoE,
 // a ragged descriptor over the expert slabs) keeps the same kind of ragged table.  Here:
 //   cnt[e]      entries routed to expert e
-//   off[e]      exclusive prefix sum of cnt (off[E] = T * k)
+//   off[e]      exclusive prefix sum of cnt (off[E] = the routed entries: T * k, fewer when
+//               adaptive top-p dropped some; a dropped entry has slot_of = -1)
 //   perm[p]     entry id t * k + rank for routed slot p; slots of one expert are contiguous
 //               and in ascending token order (a stable scatter)
 //   slot_of[i]  inverse of perm
@@ -37,7 +38,7 @@ bucket_kernel(const int32_t* __restrict__ idx, int T, int k, int E, int32_t* __r
     for (int t = t_begin; t < t_end; ++t) {
         if (lane < k) {
             const int e = idx[(size_t)t * k + lane];
-            hist[warp * E + e] += 1;
+            if (e >= 0) hist[warp * E + e] += 1;          // -1: dropped by adaptive top-p
         }
         __syncwarp();
     }
@@ -67,7 +68,7 @@ bucket_kernel(const int32_t* __restrict__ idx, int T, int k, int E, int32_t* __r
     }
     // scan[] is now inclusive; exclusive = inclusive - own
     if (threadIdx.x < E) off[threadIdx.x] = scan[threadIdx.x] - v;
-    if (threadIdx.x == 0) off[E] = T * k;
+    if (threadIdx.x == E - 1) off[E] = scan[E - 1];     // the routed slots (fewer than T k after top-p)
     // unique list: the same scan over the flags (cnt > 0)
     __syncthreads();
     const int excl = threadIdx.x < E ? scan[threadIdx.x] - v : 0;
@@ -90,9 +91,12 @@ bucket_kernel(const int32_t* __restrict__ idx, int T, int k, int E, int32_t* __r
     for (int t = t_begin; t < t_end; ++t) {
         if (lane < k) {
             const int e = idx[(size_t)t * k + lane];
-            const int p = scan[e] + hist[warp * E + e];
-            hist[warp * E + e] += 1;
-            perm[p] = t * k + lane;
+            int p = -1;
+            if (e >= 0) {
+                p = scan[e] + hist[warp * E + e];
+                hist[warp * E + e] += 1;
+                perm[p] = t * k + lane;
+            }
             slot_of[(size_t)t * k + lane] = p;
         }
         __syncwarp();

@@ -37,6 +37,29 @@ constexpr uint32_t kNib = 0x000F000Fu;
 constexpr uint32_t kBf16Magic = 0x43084308u;   // bf16 (136 + s) after the nibble flip
 constexpr uint32_t kF16Magic = 0x64086408u;    // fp16 (1032 + s) after the nibble flip
 constexpr float kBf16Offset = 136.0f;
+// int2 codes (four per byte, column 4j + i in bits 2i .. 2i+1): one LOP3 puts (n ^ 2) = s + 2 of
+// the codes of columns (i, i+8) of a 32-bit word at bits 0..1 of each 16-bit half:
+constexpr uint32_t kCrumb = 0x00030003u;
+constexpr uint32_t kBf16Magic2 = 0x43024302u;  // bf16 128 + (s + 2) = 130 + s
+constexpr uint32_t kF16Magic2 = 0x64026402u;   // fp16 1024 + (s + 2) = 1026 + s; minus 1026 is s
+constexpr float kBf16Offset2 = 130.0f;
+// int8 codes (one per byte): bytes 0 and 2 of a word, XOR 0x80, in the low mantissa bits of fp16
+// 1024 read 1024 + s + 128 = 1152 + s; minus 1152 is s.
+constexpr uint32_t kByte = 0x00FF00FFu;
+constexpr uint32_t kF16Magic8 = 0x64806480u;
+
+// Columns per 16-byte chunk of a weight row, and bytes per row of n columns, per weight kind.
+template <int WK> struct Kind;
+template <> struct Kind<MOE_W_INT4_ROWSCALE> { static constexpr int COLS = 32; __host__ __device__ static size_t bytes(int n) { return (size_t)n / 2; } };
+template <> struct Kind<MOE_W_BF16> { static constexpr int COLS = 8; __host__ __device__ static size_t bytes(int n) { return (size_t)n * 2; } };
+template <> struct Kind<MOE_W_INT8_ROWSCALE> { static constexpr int COLS = 16; __host__ __device__ static size_t bytes(int n) { return (size_t)n; } };
+template <> struct Kind<MOE_W_INT2_ROWSCALE> { static constexpr int COLS = 64; __host__ __device__ static size_t bytes(int n) { return (size_t)n / 4; } };
+
+// bf16 value number i (0..7) of an 8-column x vector
+__device__ __forceinline__ unsigned short xhalf(const uint4& v, int i) {
+    const uint32_t w = i < 2 ? v.x : i < 4 ? v.y : i < 6 ? v.z : v.w;
+    return (unsigned short)((i & 1) ? (w >> 16) : (w & 0xffffu));
+}
 
 struct Slots {
     int ntok;      // tokens in the bucket
@@ -67,9 +90,9 @@ gateup_kernel(const uint8_t* __restrict__ gate_up, const float* __restrict__ gu_
               const uint16_t* __restrict__ x, const double* __restrict__ xsum, int T, int k, int d, int f,
               int f_sh, int S, const int32_t* __restrict__ ulist, const int32_t* __restrict__ n_unique_p,
               const int32_t* __restrict__ cnt, const int32_t* __restrict__ off, const int32_t* __restrict__ perm,
-              uint16_t* __restrict__ h, int fmax, int* status) {
+              uint16_t* __restrict__ h, int fmax, int* status, const void* const* __restrict__ etab, int E) {
     constexpr int R = kGateUpRows;
-    constexpr int COLS = WK == MOE_W_INT4_ROWSCALE ? 32 : 8;     // columns per 16-byte chunk
+    constexpr int COLS = Kind<WK>::COLS;                          // columns per 16-byte chunk
     constexpr int XV = COLS / 8;                                  // 16-byte x vectors per chunk
     const int lane = threadIdx.x % kWarp;
     const int gwarp = (blockIdx.x * blockDim.x + threadIdx.x) / kWarp;
@@ -78,7 +101,7 @@ gateup_kernel(const uint8_t* __restrict__ gate_up, const float* __restrict__ gu_
     const int per_routed = f / R;
     const int n_tasks = n_unique * per_routed + (S ? f_sh / R : 0);
     const int nchunk = d / COLS;
-    const size_t rowbytes = WK == MOE_W_INT4_ROWSCALE ? (size_t)d / 2 : (size_t)d * 2;
+    const size_t rowbytes = Kind<WK>::bytes(d);
 
     for (int task = gwarp; task < n_tasks; task += nwarps) {
         const uint8_t* W;
@@ -89,8 +112,8 @@ gateup_kernel(const uint8_t* __restrict__ gate_up, const float* __restrict__ gu_
             const int e = ulist[task / per_routed];
             r0 = (task % per_routed) * R;
             fe = f;
-            W = gate_up + (size_t)e * 2 * f * rowbytes;
-            sc = gu_scale ? gu_scale + (size_t)e * 2 * f : nullptr;
+            W = ex_gate_up(etab, E, e);
+            sc = WK != MOE_W_BF16 ? ex_gu_scale(etab, E, e) : nullptr;
             b = Slots{cnt[e], off[e], false};
         } else {
             r0 = (task - n_unique * per_routed) * R;
@@ -169,6 +192,30 @@ gateup_kernel(const uint8_t* __restrict__ gate_up, const float* __restrict__ gu_
                                     a = fma_bf16(a6, x6, a);
                                     a = fma_bf16(a7, x7, a);
                                 }
+                            } else if (WK == MOE_W_INT2_ROWSCALE) {
+                                // word m: columns 16m .. 16m+15 (x vectors 2m and 2m+1)
+                                const uint32_t words[4] = {wv[rr].x, wv[rr].y, wv[rr].z, wv[rr].w};
+#pragma unroll
+                                for (int m = 0; m < 4; ++m) {
+#pragma unroll
+                                    for (int i = 0; i < 8; ++i) {
+                                        unsigned short lo, hi;
+                                        halves(lop_sel_xor(words[m] >> (2 * i), kCrumb, kBf16Magic2), lo, hi);
+                                        a = fma_bf16(lo, xhalf(xv[2 * m], i), a);
+                                        a = fma_bf16(hi, xhalf(xv[2 * m + 1], i), a);
+                                    }
+                                }
+                            } else if (WK == MOE_W_INT8_ROWSCALE) {
+                                // word m: columns 4m .. 4m+3; the codes convert exactly to fp32
+                                const uint32_t words[4] = {wv[rr].x, wv[rr].y, wv[rr].z, wv[rr].w};
+#pragma unroll
+                                for (int m = 0; m < 4; ++m) {
+#pragma unroll
+                                    for (int i = 0; i < 4; ++i) {
+                                        const float q = (float)((int)(words[m] << (24 - 8 * i)) >> 24);
+                                        a = fmaf(q, bf16_bits_to_f32(xhalf(xv[m >> 1], 4 * (m & 1) + i)), a);
+                                    }
+                                }
                             } else {
                                 const uint32_t ws[4] = {wv[rr].x, wv[rr].y, wv[rr].z, wv[rr].w};
                                 const uint32_t xs[4] = {xv[0].x, xv[0].y, xv[0].z, xv[0].w};
@@ -199,10 +246,12 @@ gateup_kernel(const uint8_t* __restrict__ gate_up, const float* __restrict__ gu_
                     for (int j = 0; j < TG; ++j) {
                         if (j < ng) {
                             float g = acc[rr][j], u = acc[R + rr][j];
-                            if (WK == MOE_W_INT4_ROWSCALE) {
-                                const float off136 = kBf16Offset * (float)xsum[tok[j]];
-                                g = sc[r] * (g - off136);
-                                u = sc[fe + r] * (u - off136);
+                            if (WK != MOE_W_BF16) {
+                                const float off = WK == MOE_W_INT4_ROWSCALE ? kBf16Offset * (float)xsum[tok[j]]
+                                                  : WK == MOE_W_INT2_ROWSCALE ? kBf16Offset2 * (float)xsum[tok[j]]
+                                                                              : 0.0f;
+                                g = sc[r] * (g - off);
+                                u = sc[fe + r] * (u - off);
                             }
                             const float hv = g / (1.0f + expf(-g)) * u;
                             const __half hh = __float2half_rn(hv);
@@ -226,9 +275,9 @@ down_kernel(const uint8_t* __restrict__ down, const float* __restrict__ dn_scale
             const uint16_t* __restrict__ h, int fmax, int T, int k, int d, int f, int f_sh, int S,
             const int32_t* __restrict__ ulist, const int32_t* __restrict__ n_unique_p,
             const int32_t* __restrict__ cnt, const int32_t* __restrict__ off, const int32_t* __restrict__ perm,
-            float* __restrict__ Y) {
+            float* __restrict__ Y, const void* const* __restrict__ etab, int E) {
     constexpr int R = kDownRows;
-    constexpr int COLS = WK == MOE_W_INT4_ROWSCALE ? 32 : 8;
+    constexpr int COLS = Kind<WK>::COLS;
     constexpr int HV = COLS / 8;      // 16-byte h vectors per chunk
     const int lane = threadIdx.x % kWarp;
     const int gwarp = (blockIdx.x * blockDim.x + threadIdx.x) / kWarp;
@@ -247,9 +296,8 @@ down_kernel(const uint8_t* __restrict__ down, const float* __restrict__ dn_scale
         if (u < n_unique) {
             const int e = ulist[u];
             fe = f;
-            const size_t rowbytes = WK == MOE_W_INT4_ROWSCALE ? (size_t)f / 2 : (size_t)f * 2;
-            W = down + (size_t)e * d * rowbytes;
-            sc = dn_scale ? dn_scale + (size_t)e * d : nullptr;
+            W = ex_down(etab, E, e);
+            sc = WK != MOE_W_BF16 ? ex_dn_scale(etab, E, e) : nullptr;
             b = Slots{cnt[e], off[e], false};
         } else {
             fe = f_sh;
@@ -257,7 +305,7 @@ down_kernel(const uint8_t* __restrict__ down, const float* __restrict__ dn_scale
             sc = sh_dn_scale;
             b = Slots{T, 0, true};
         }
-        const size_t rowbytes = WK == MOE_W_INT4_ROWSCALE ? (size_t)fe / 2 : (size_t)fe * 2;
+        const size_t rowbytes = Kind<WK>::bytes(fe);
         const int nchunk = fe / COLS;
         for (int g0 = 0; g0 < b.ntok; g0 += TG) {
             const int ng = min(TG, b.ntok - g0);
@@ -326,6 +374,32 @@ down_kernel(const uint8_t* __restrict__ down, const float* __restrict__ dn_scale
                                     a = fma_f16(s6, h6, a);
                                     a = fma_f16(s7, h7, a);
                                 }
+                            } else if (WK == MOE_W_INT2_ROWSCALE) {
+                                const uint32_t words[4] = {wv[rr].x, wv[rr].y, wv[rr].z, wv[rr].w};
+#pragma unroll
+                                for (int m = 0; m < 4; ++m) {
+#pragma unroll
+                                    for (int i = 0; i < 8; ++i) {
+                                        unsigned short lo, hi;
+                                        halves(hsub2_u32(lop_sel_xor(words[m] >> (2 * i), kCrumb, kF16Magic2), kF16Magic2),
+                                               lo, hi);
+                                        a = fma_f16(lo, xhalf(hv[2 * m], i), a);
+                                        a = fma_f16(hi, xhalf(hv[2 * m + 1], i), a);
+                                    }
+                                }
+                            } else if (WK == MOE_W_INT8_ROWSCALE) {
+                                const uint32_t words[4] = {wv[rr].x, wv[rr].y, wv[rr].z, wv[rr].w};
+#pragma unroll
+                                for (int m = 0; m < 4; ++m) {
+                                    unsigned short s0, s1, s2, s3;
+                                    halves(hsub2_u32(lop_sel_xor(words[m], kByte, kF16Magic8), kF16Magic8), s0, s2);
+                                    halves(hsub2_u32(lop_sel_xor(words[m] >> 8, kByte, kF16Magic8), kF16Magic8), s1, s3);
+                                    const int b = 4 * (m & 1);
+                                    a = fma_f16(s0, xhalf(hv[m >> 1], b), a);
+                                    a = fma_f16(s1, xhalf(hv[m >> 1], b + 1), a);
+                                    a = fma_f16(s2, xhalf(hv[m >> 1], b + 2), a);
+                                    a = fma_f16(s3, xhalf(hv[m >> 1], b + 3), a);
+                                }
                             } else {
                                 const uint32_t ws[4] = {wv[rr].x, wv[rr].y, wv[rr].z, wv[rr].w};
                                 const uint32_t hs[4] = {hv[0].x, hv[0].y, hv[0].z, hv[0].w};
@@ -349,7 +423,7 @@ down_kernel(const uint8_t* __restrict__ down, const float* __restrict__ dn_scale
             for (int rr = 0; rr < R; ++rr) {
                 if (lane == rr) {
                     const int jr = j0 + rr;
-                    const float s = WK == MOE_W_INT4_ROWSCALE ? sc[jr] : 1.0f;
+                    const float s = WK != MOE_W_BF16 ? sc[jr] : 1.0f;
 #pragma unroll
                     for (int j = 0; j < TG; ++j)
                         if (j < ng) Y[(size_t)slot[j] * d + jr] = s * acc[rr][j];
@@ -374,6 +448,7 @@ combine_kernel(const float* __restrict__ Y, const float* __restrict__ wts, const
         const int r = asc[(size_t)t * k + p];
         const float w = wts[(size_t)t * k + r];
         const int slot = slot_of[(size_t)t * k + r];
+        if (slot < 0) continue;                   // dropped by adaptive top-p
         const float4 y = reinterpret_cast<const float4*>(Y + (size_t)slot * d)[j4];
         acc.x = fmaf(w, y.x, acc.x);
         acc.y = fmaf(w, y.y, acc.y);
@@ -407,11 +482,12 @@ cudaError_t launch_experts_t(const LayerDims& L, const moe_weights& W, const uin
               (gateup_kernel<WK, TG><<<grid, kThreads, 0, ctx.s>>>(
                   (const uint8_t*)W.gate_up, W.gate_up_scale, (const uint8_t*)W.shared_gate_up, W.shared_gate_up_scale,
                   x, ws.xsum, T, L.k, L.d, L.f, L.f_shared, L.S, ws.ulist, ws.n_unique, ws.cnt, ws.off, ws.perm, ws.h,
-                  fmax, ws.status)));
+                  fmax, ws.status, ws.etab, L.E)));
     QE_LAUNCH(ctx, MOE_KERNEL_DOWN,
               (down_kernel<WK, TG><<<grid, kThreads, 0, ctx.s>>>(
                   (const uint8_t*)W.down, W.down_scale, (const uint8_t*)W.shared_down, W.shared_down_scale, ws.h, fmax,
-                  T, L.k, L.d, L.f, L.f_shared, L.S, ws.ulist, ws.n_unique, ws.cnt, ws.off, ws.perm, ws.Y)));
+                  T, L.k, L.d, L.f, L.f_shared, L.S, ws.ulist, ws.n_unique, ws.cnt, ws.off, ws.perm, ws.Y, ws.etab,
+                  L.E)));
     return cudaSuccess;
 }
 
@@ -428,6 +504,12 @@ cudaError_t launch_decode_experts(const LayerDims& L, const moe_weights& W, cons
     if (L.wkind == MOE_W_INT4_ROWSCALE)
         return T <= 4 ? launch_experts_t<MOE_W_INT4_ROWSCALE, 1>(L, W, x, T, ws, num_sms, ctx)
                       : launch_experts_t<MOE_W_INT4_ROWSCALE, 2>(L, W, x, T, ws, num_sms, ctx);
+    if (L.wkind == MOE_W_INT8_ROWSCALE)
+        return T <= 4 ? launch_experts_t<MOE_W_INT8_ROWSCALE, 1>(L, W, x, T, ws, num_sms, ctx)
+                      : launch_experts_t<MOE_W_INT8_ROWSCALE, 2>(L, W, x, T, ws, num_sms, ctx);
+    if (L.wkind == MOE_W_INT2_ROWSCALE)
+        return T <= 4 ? launch_experts_t<MOE_W_INT2_ROWSCALE, 1>(L, W, x, T, ws, num_sms, ctx)
+                      : launch_experts_t<MOE_W_INT2_ROWSCALE, 2>(L, W, x, T, ws, num_sms, ctx);
     return T <= 4 ? launch_experts_t<MOE_W_BF16, 1>(L, W, x, T, ws, num_sms, ctx)
                   : launch_experts_t<MOE_W_BF16, 2>(L, W, x, T, ws, num_sms, ctx);
 }

@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kGuMaxWarps * kWarp, 1)
 gateup_t1_kernel(const uint8_t* __restrict__ gate_up, const float* __restrict__ gu_scale,
                  const uint8_t* __restrict__ sh_gate_up, const float* __restrict__ sh_gu_scale,
                  const uint16_t* __restrict__ x, int k, int d, int f, int f_sh, int S, const int32_t* ulist,
-                 uint16_t* __restrict__ h, int fmax, int* status) {
+                 uint16_t* __restrict__ h, int fmax, int* status, const void* const* __restrict__ etab, int E) {
     // [warps][kGuStages][gate row | up row | 16 B holding the gate scale | 16 B holding the up scale]
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bars[kGuMaxWarps][kGuStages];
@@ -103,8 +103,8 @@ gateup_t1_kernel(const uint8_t* __restrict__ gate_up, const float* __restrict__ 
             const int t2 = t - n_shared_tasks;
             const int u = t2 / f, r = t2 % f;
             const int e = s_ulist[warp][u];
-            tk.gate = gate_up + ((size_t)e * 2 * f + r) * rowbytes;
-            tk.sc = gu_scale + (size_t)e * 2 * f + r;
+            tk.gate = ex_gate_up(etab, E, e) + (size_t)r * rowbytes;
+            tk.sc = ex_gu_scale(etab, E, e) + r;
             tk.r = r;
             tk.fe = f;
             tk.slot = u;
@@ -214,7 +214,8 @@ __global__ void __launch_bounds__(kDnMaxSlots * kDnSlotWarps * kWarp, 1)
 down_t1_kernel(const uint8_t* __restrict__ down, const float* __restrict__ dn_scale,
                const uint8_t* __restrict__ sh_down, const float* __restrict__ sh_dn_scale, const uint16_t* h,
                int fmax, int k, int d, int f, int S, const int32_t* ulist, const float* wts, const int32_t* asc,
-               void* __restrict__ out, int out_bf16, int rj, int* status) {
+               void* __restrict__ out, int out_bf16, int rj, int* status, const void* const* __restrict__ etab,
+               int E) {
     extern __shared__ __align__(128) uint8_t smem[];          // [warps][kDnStages][kDnRows * rowbytes]
     __shared__ __align__(8) uint64_t bars[kDnMaxSlots * kDnSlotWarps][kDnStages];
     __shared__ float ys[kDnMaxSlots][kDnRowsMax];
@@ -234,8 +235,8 @@ down_t1_kernel(const uint8_t* __restrict__ down, const float* __restrict__ dn_sc
     const uint32_t ring = saddr(smem) + (uint32_t)warp * kDnStages * stage_bytes;
     // routing is final when this grid starts (the gate/up kernel triggered after its own wait)
     const int e = shared ? -1 : __ldcg(ulist + u);
-    const uint8_t* W = shared ? sh_down : down + (size_t)e * d * rowbytes;
-    const float* sc = shared ? sh_dn_scale : dn_scale + (size_t)e * d;
+    const uint8_t* W = shared ? sh_down : ex_down(etab, E, e);
+    const float* sc = shared ? sh_dn_scale : ex_dn_scale(etab, E, e);
     if (u < k && half == 0 && lane == 0) gate_w[u] = __ldcg(wts + __ldcg(asc + u));
     if (lane == 0) {
         for (int s = 0; s < kDnStages; ++s) bar_init(saddr(&bars[warp][s]), 1);
@@ -364,7 +365,7 @@ cudaError_t launch_decode_t1(const LayerDims& L, const moe_weights& W, const uin
         e = launch_pdl(L.pdl != 0, gateup_t1_kernel<N>, dim3(num_sms), dim3(guw * kWarp), gu_smem, ctx.s,              \
                        (const uint8_t*)W.gate_up, W.gate_up_scale, (const uint8_t*)W.shared_gate_up,                  \
                        W.shared_gate_up_scale, x, L.k, L.d, L.f, L.f_shared, L.S, (const int32_t*)ws.ulist, ws.h,     \
-                       fmax, ws.status);                                                                              \
+                       fmax, ws.status, (const void* const*)ws.etab, L.E);                                            \
         break;
     switch (nchx) {
         QE_GU(1) QE_GU(2) QE_GU(3) QE_GU(4) QE_GU(5) QE_GU(6) QE_GU(7) QE_GU(8)
@@ -385,7 +386,7 @@ cudaError_t launch_decode_t1(const LayerDims& L, const moe_weights& W, const uin
         e = launch_pdl(L.pdl != 0, down_t1_kernel<N>, dim3(grid), dim3(threads), dsm, ctx.s, (const uint8_t*)W.down,   \
                        W.down_scale, (const uint8_t*)W.shared_down, W.shared_down_scale, (const uint16_t*)ws.h, fmax, \
                        L.k, L.d, L.f, L.S, (const int32_t*)ws.ulist, (const float*)ws.wts, (const int32_t*)ws.asc,    \
-                       out, L.out_bf16, rj, ws.status);                                                              \
+                       out, L.out_bf16, rj, ws.status, (const void* const*)ws.etab, L.E);                             \
         break;
     switch (nchf) {
         QE_DN(1) QE_DN(2) QE_DN(3) QE_DN(4)

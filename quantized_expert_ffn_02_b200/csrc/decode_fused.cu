@@ -3,21 +3,21 @@
 // For one token the layer reads each weight byte once, so its time is the time to stream the
 // router matrix and k + 1 experts from HBM.  Separate kernels for the router, gate/up and down
 // each pay the ramp of a fresh grid and leave HBM idle while the previous grid drains; here one
-// persistent CTA per SM (16 warps) runs the steps back to back and keeps its copies in flight
-// across the joins.  Shared memory holds x, rearranged once per CTA so that a lane's 32-column
-// chunk loads without bank conflicts, and one ring of two TMA stages per warp (a gate row, the
-// matching up row and two 16-byte slivers holding their scales).
+// persistent CTA per SM (8 warps) runs the steps back to back and keeps its copies in flight
+// across the joins.  Each warp streams its weight rows through a private ring of TMA bulk copies
+// (a gate row, the matching up row and two 16-byte slivers holding their scales per stage).
 //
-//   A  router + shared expert.  One bulk copy brings x in; each warp's first router piece (one
-//      expert x 1024 columns, coalesced loads) is in flight meanwhile.  The warps rearrange x,
-//      sum it, queue their shared-expert row pairs (they need no routing), compute their router
-//      pieces in fp64 and store them.  The CTA arrives on grid barrier 0, and the warps reduce
-//      their shared rows while the other CTAs arrive.
+//   A  router + shared expert.  The warps queue their shared-expert row pairs (they need no
+//      routing) at once; one bulk copy brings x in while each warp's first router piece (one
+//      expert x 1024 columns, coalesced loads) is in flight.  The warps compute their router
+//      pieces in fp64 and store them, turn x into their fp16 operand registers (below), and the
+//      CTA arrives on grid barrier 0; the warps reduce their shared rows while the others arrive.
 //   B  selection, by the whole CTA: one bulk copy gathers every piece; thread e sums expert e's
 //      pieces (the same order in every CTA, so every CTA selects the same experts) and forms an
 //      order-preserving integer key; the k best of each warp's 32 experts become candidates, and
 //      each candidate's rank among the candidates is its overall rank.  The k experts (ascending)
-//      and their gate weights go to shared memory.
+//      and their gate weights go to shared memory, and the CTA asks L2 to prefetch the down rows
+//      it will read in D (read once, so the gate/up stream is marked evict-first).
 //   C  routed gate/up: row pairs of the k experts, strided over every warp of the grid;
 //      h = SiLU(gate) * up in fp16 (global, L2), the SiLU of 32 row pairs at a time.  A warp that
 //      has finished its row pairs queues its first down rows (they do not depend on h), then the
@@ -26,10 +26,24 @@
 //      routed experts in ascending index order, then the shared expert); its warps split the
 //      (slot, row) list, and the CTA adds the slots with their gate weights and stores y.
 //
-// Dequantisation: gate/up as bf16 136 + s (one LOP3 per two codes) with the offset removed
-// through the sum of x; down as fp16 3/2 + s/16 (one shift and one LOP3 per two codes) with the
-// offset removed through the sum of h.  Products are exact, sums fp32, h is rounded to fp16; the
-// router logits accumulate in fp64.
+// The dot products run on the tensor cores (mma.sync m16n8k16, fp16 operands, fp32
+// accumulation) -- not to reach tensor-core throughput, which a matrix-vector product cannot use,
+// but because the same sums on the FP32 pipe cost about two instructions per weight and lane and
+// bound the kernel by instruction issue instead of HBM.  One MMA takes the 16 rows
+// {8 K-segments of the gate row, the same 8 segments of the up row} against B = the 8 matching
+// segments of x, one per column; the diagonal of the 8 x 8 product blocks is the two dot products
+// (the off-diagonal terms are discarded).  Lane (g, c) of the warp feeds segment g, so it only
+// ever touches x and weights of its own segment, at the K positions of its own quarter.
+//
+// Dequantisation: a code s = n - 16 [n >= 8] is stored as the nibble n; n ^ 8 = s + 8.  One LOP3
+// builds the pair (n_i ^ 8, n_{i+4} ^ 8) at fp16 mantissa bits 0..3 with a zero exponent -- the
+// exact fp16 value (s + 8) 2^-24 -- or at bits 4..7, the exact value (s + 8) 2^-20; one shift by
+// 8 bits reaches the other two nibble pairs, so 8 codes cost one shift and four LOP3s.  The x
+// entries that meet the 2^-20 codes are stored scaled by 2^-4, so every product is
+// (s + 8) x 2^-24, exact, and the fp32 sums give sum s x = 2^24 D - 8 sum x.  x enters as fp16
+// x 2^sigma, with sigma a per-token power of two that puts max|x| in [2^14, 2^15): every bf16
+// value in that range converts exactly.  h (fp16 already) is scaled the same way per slot.  The
+// router logits accumulate in fp64 on the FP64 pipe.
 //
 // Phase timestamps (%globaltimer, thread 0 of each CTA) go to the workspace for the layer's
 // debug read.
@@ -52,12 +66,14 @@ namespace {
 
 using namespace dec;
 
-constexpr int kFzMaxWarps = 16;
-constexpr int kFzStages = 2;
+constexpr int kFzWarps = 8;
+constexpr int kFzThreads = kFzWarps * kWarp;
+constexpr int kFzMaxStages = 4;
 constexpr int kFzMaxSlots = 10;       // k routed experts + the shared one
 constexpr int kFzMaxPer = 8;          // experts per lane in the selection: E <= 256
 constexpr int kFzRowsMax = 64;        // output rows per CTA
 constexpr int kFzDnRowsMax = 8;       // down rows per stage
+constexpr int kFzScRegs = 3;          // down-row scales per lane: up to 96 (slot, row) items per warp
 constexpr size_t kSmemLimit = 227 * 1024;
 constexpr int kStaticReserve = 5120;  // static shared memory of the kernel, rounded up
 
@@ -65,14 +81,11 @@ struct FusedArgs {
     const float* router_w;            // [E][d] fp32
     const float* bias;                // [E] selection bias (sigmoid router) or null
     const uint16_t* x;                // [d] bf16
-    const uint8_t* gate_up;           // [E][2f][d/2]
-    const float* gu_scale;            // [E][2f]
     const uint8_t* sh_gate_up;        // [2f][d/2]
     const float* sh_gu_scale;         // [2f]
-    const uint8_t* down;              // [E][d][f/2]
-    const float* dn_scale;            // [E][d]
     const uint8_t* sh_down;           // [d][f/2]
     const float* sh_dn_scale;         // [d]
+    const void* const* etab;          // [4][E] the routed experts' gate/up, its scales, down, its scales
     double* rpart;                    // [E][d/1024] pieces of the router logits
     uint16_t* h;                      // [k+1][f] fp16
     void* out;                        // [d] fp32 or bf16
@@ -83,7 +96,7 @@ struct FusedArgs {
     int32_t* n_unique;
     double* xsum;
     unsigned long long* bar;          // grid-barrier arrivals (never reset between launches)
-    unsigned long long* trace;        // [CTA][8] %globaltimer at the phase boundaries
+    unsigned long long* trace;        // [CTA][16] %globaltimer at the phase boundaries
     int* status;
     int d, f, E, k, S, router, out_bf16, dn_rows;
     float scaling;
@@ -114,6 +127,21 @@ __device__ __forceinline__ float4 ld_stream16f(const float* p) {
     const uint4 v = ld_stream16(p);
     return make_float4(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z), __uint_as_float(v.w));
 }
+// L2 cache policies: streamed weight rows are read once (evict first); the down rows prefetched
+// for phase D should outlive them (normal priority).
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// Bulk copy global -> shared with an L2 cache policy, completion counted on `bar`.
+__device__ __forceinline__ void bulk_g2s_hint(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
+                                              uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+        : "memory");
+}
 // Start an L2 prefetch of [p, p + bytes) (16-byte aligned, size a multiple of 16).
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
@@ -141,75 +169,181 @@ __device__ __forceinline__ double router_piece(const float4 (&rw)[8], uint32_t x
     return a;
 }
 
-// x of one lane's chunk c (32 columns) from the pre-paired copy in shared memory: four 16-byte
-// rows, the pairs (column 8m + i, column 8m + i + 4) for m = 0..3, i = 0..3.
-__device__ __forceinline__ void load_xq(uint32_t xp_s, int nchunks, int c, uint32_t (&xq)[16]) {
+// ---------------------------------------------------------------------------------------
+// The tensor-core dot products
+// ---------------------------------------------------------------------------------------
+// D += A B for one m16n8k16 tile, fp16 operands, fp32 accumulators.  Fragments (lane = 4 g + c):
+// a0 = A[g][2c, 2c+1], a1 = A[g+8][2c, 2c+1], a2 = A[g][2c+8, 2c+9], a3 = A[g+8][2c+8, 2c+9];
+// b0 = B[2c, 2c+1][g], b1 = B[2c+8, 2c+9][g]; d = D[g][2c, 2c+1], D[g+8][2c, 2c+1].
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// Codes of columns (i, i+4) of a 32-bit word (nibble i = column i) as the fp16 pair
+// ((s_i + 8) 2^-24, (s_{i+4} + 8) 2^-24) for i = 0 (nib_lo) or (s + 8) 2^-20 for i = 1 (nib_hi);
+// of w >> 8, the same for i = 2 and 3.
+__device__ __forceinline__ uint32_t nib_lo(uint32_t w) { return lop_sel_xor(w, 0x000F000Fu, 0x00080008u); }
+__device__ __forceinline__ uint32_t nib_hi(uint32_t w) { return lop_sel_xor(w, 0x00F000F0u, 0x00800080u); }
+
+// The 16-byte group a lane reads at step j of a row: its groups are visited from a lane-dependent
+// start so that the 8 lanes of each shared-memory phase hit 8 different bank quads (checked for
+// every width the kernel takes).
+template <int NDK>
+__device__ __forceinline__ int gu_rot(int lane) {
+    const int g = lane >> 2, c = lane & 3;
+    if (NDK % 2) return 0;
+    if (NDK == 4) return (c >> 1) + 2 * (g & 1);
+    if (NDK == 8) return (g & 1) + 2 * c;
+    return g & 1;
+}
+template <int NF>
+__device__ __forceinline__ int dn_rot(int lane) {
+    return NF == 2 ? ((lane >> 2) & 1) : 0;
+}
+
+// 8 bf16 (or fp16) values of one 8-column group, as the four operand pairs of that group:
+// (col 0, col 4), (col 1, col 5) x 2^-4, (col 2, col 6), (col 3, col 7) x 2^-4, each scaled by
+// 2^e (fp32 arithmetic, then one rounding to fp16; exact for values in fp16's normal range).
+__device__ __forceinline__ void pairs_from_bf16(uint4 v, float s, float s16, uint32_t* p, float& sum) {
+    const float c0 = __uint_as_float(v.x << 16), c1 = __uint_as_float(v.x & 0xffff0000u);
+    const float c2 = __uint_as_float(v.y << 16), c3 = __uint_as_float(v.y & 0xffff0000u);
+    const float c4 = __uint_as_float(v.z << 16), c5 = __uint_as_float(v.z & 0xffff0000u);
+    const float c6 = __uint_as_float(v.w << 16), c7 = __uint_as_float(v.w & 0xffff0000u);
+    const __half2 p0 = __floats2half2_rn(c0 * s, c4 * s), p1 = __floats2half2_rn(c1 * s16, c5 * s16);
+    const __half2 p2 = __floats2half2_rn(c2 * s, c6 * s), p3 = __floats2half2_rn(c3 * s16, c7 * s16);
+    p[0] = *reinterpret_cast<const uint32_t*>(&p0);
+    p[1] = *reinterpret_cast<const uint32_t*>(&p1);
+    p[2] = *reinterpret_cast<const uint32_t*>(&p2);
+    p[3] = *reinterpret_cast<const uint32_t*>(&p3);
+    // the sum of the scaled values the MMA sees at the unscaled positions (fp16-rounded)
+    const float2 f0 = __half22float2(p0), f2 = __half22float2(p2);
+    const float2 f1 = __half22float2(p1), f3 = __half22float2(p3);
+    sum += (f0.x + f0.y) + (f2.x + f2.y) + 16.0f * ((f1.x + f1.y) + (f3.x + f3.y));
+}
+__device__ __forceinline__ void pairs_from_f16(uint4 v, float s, float s16, uint32_t* p, float& sum) {
+    const uint32_t q[4] = {__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632),
+                           __byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632)};
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const uint4 v = lds16(xp_s + (uint32_t)(m * nchunks + c) * 16u);
-        xq[4 * m] = v.x;
-        xq[4 * m + 1] = v.y;
-        xq[4 * m + 2] = v.z;
-        xq[4 * m + 3] = v.w;
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&q[i]));
+        const float m = (i & 1) ? s16 : s;
+        const __half2 r = __floats2half2_rn(f.x * m, f.y * m);
+        p[i] = *reinterpret_cast<const uint32_t*>(&r);
+        const float2 b = __half22float2(r);
+        sum += (i & 1) ? 16.0f * (b.x + b.y) : (b.x + b.y);
     }
 }
-
-// Dot products of one gate row and one up row (stage at shared address st) with x; x comes from
-// the pre-paired shared copy, so the loop over the lane's chunks stays rolled (a small loop body
-// keeps the instruction cache warm).
-__device__ __forceinline__ float2 gu_dot(uint32_t st, uint32_t gu_row, int lane, uint32_t xp_s, int nchunks) {
-    // two accumulators per row (even and odd words) halve the chains of dependent FMAs
-    float ag0 = 0.0f, ag1 = 0.0f, au0 = 0.0f, au1 = 0.0f;
-#pragma unroll 2
-    for (int c = lane; c < nchunks; c += kWarp) {
-        uint32_t xq[16];
-        load_xq(xp_s, nchunks, c, xq);
-        const uint4 Gv = lds16(st + (uint32_t)c * 16), Uv = lds16(st + gu_row + (uint32_t)c * 16);
-        ag0 = dot_word_bf16(Gv.x, &xq[0], ag0);
-        au0 = dot_word_bf16(Uv.x, &xq[0], au0);
-        ag1 = dot_word_bf16(Gv.y, &xq[4], ag1);
-        au1 = dot_word_bf16(Uv.y, &xq[4], au1);
-        ag0 = dot_word_bf16(Gv.z, &xq[8], ag0);
-        au0 = dot_word_bf16(Uv.z, &xq[8], au0);
-        ag1 = dot_word_bf16(Gv.w, &xq[12], ag1);
-        au1 = dot_word_bf16(Uv.w, &xq[12], au1);
-    }
-    return make_float2(ag0 + ag1, au0 + au1);
+// 2^e as a float for |e| <= 126.
+__device__ __forceinline__ float exp2i(int e) { return __uint_as_float((uint32_t)(127 + e) << 23); }
+// The power of two that moves max|v| (v > 0, finite) into [2^14, 2^15), clamped to [-100, 100];
+// 0 for v == 0.
+__device__ __forceinline__ int scale_exp(float vmax) {
+    if (!(vmax > 0.0f) || !isfinite(vmax)) return 0;
+    const int e = (int)((__float_as_uint(vmax) >> 23) & 0xff) - 127;   // floor(log2 vmax), vmax normal in fp32
+    return max(-100, min(100, 14 - e));
 }
 
-// NCF = f / 1024 (h chunks per lane in the down phase).
-template <int NCF>
-__global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(const FusedArgs a) {
-    // [x pre-paired: 2d bytes][kFzStages][warps][stage]: stage s of every warp is one region
+// Diagonal of the two 8 x 8 blocks held by the warp's D fragments (four accumulator chains):
+// this lane's part of (rows 0..7 . columns) and (rows 8..15 . columns); 0 for lanes that hold no
+// diagonal entry.
+__device__ __forceinline__ float2 diag_part(const float (&acc)[4][4], int lane) {
+    const int g = lane >> 2, c = lane & 3;
+    if (c != (g >> 1)) return make_float2(0.0f, 0.0f);
+    const float e0 = (acc[0][0] + acc[1][0]) + (acc[2][0] + acc[3][0]);
+    const float e1 = (acc[0][1] + acc[1][1]) + (acc[2][1] + acc[3][1]);
+    const float e2 = (acc[0][2] + acc[1][2]) + (acc[2][2] + acc[3][2]);
+    const float e3 = (acc[0][3] + acc[1][3]) + (acc[2][3] + acc[3][3]);
+    return (g & 1) ? make_float2(e1, e3) : make_float2(e0, e2);
+}
+
+// Gate row . x and up row . x for the row pair of stage st (2^24 times the sums of (s + 8) x~;
+// this lane's part, see diag_part).  xr holds this lane's x~ pairs, group by group in its visiting
+// order; lane_off is the byte offset of its segment quarter within a row.
+template <int NDK>
+__device__ __forceinline__ float2 gu_mma(uint32_t st, uint32_t gu_row, uint32_t lane_off, int rot,
+                                         const uint32_t (&xr)[NDK][16], int lane) {
+    float acc[4][4] = {};          // four independent accumulator chains (one per word of a group)
+#pragma unroll
+    for (int j = 0; j < NDK; ++j) {
+        int q = j + rot;
+        if (q >= NDK) q -= NDK;
+        const uint32_t off = lane_off + 16u * (uint32_t)q;
+        const uint4 G = lds16(st + off), U = lds16(st + gu_row + off);
+        const uint32_t gw[4] = {G.x, G.y, G.z, G.w}, uw[4] = {U.x, U.y, U.z, U.w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            mma16816(acc[w], nib_lo(gw[w]), nib_lo(uw[w]), nib_hi(gw[w]), nib_hi(uw[w]), xr[j][4 * w],
+                     xr[j][4 * w + 1]);
+            const uint32_t g8 = gw[w] >> 8, u8 = uw[w] >> 8;
+            mma16816(acc[w], nib_lo(g8), nib_lo(u8), nib_hi(g8), nib_hi(u8), xr[j][4 * w + 2], xr[j][4 * w + 3]);
+        }
+    }
+    return diag_part(acc, lane);
+}
+
+// Down rows A and B (shared addresses) . h~ of their slot: this lane's parts of 2^24 times the
+// sums of (s + 8) h~ (see diag_part); B may equal A.
+template <int NF>
+__device__ __forceinline__ float2 dn_mma(uint32_t rowA, uint32_t rowB, uint32_t lane_off, int rot,
+                                         const uint32_t (&hr)[NF][16], int lane) {
+    float acc[4][4] = {};
+#pragma unroll
+    for (int j = 0; j < NF; ++j) {
+        int q = j + rot;
+        if (q >= NF) q -= NF;
+        const uint32_t off = lane_off + 16u * (uint32_t)q;
+        const uint4 A = lds16(rowA + off), B = lds16(rowB + off);
+        const uint32_t aw[4] = {A.x, A.y, A.z, A.w}, bw[4] = {B.x, B.y, B.z, B.w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            mma16816(acc[w], nib_lo(aw[w]), nib_lo(bw[w]), nib_hi(aw[w]), nib_hi(bw[w]), hr[j][4 * w],
+                     hr[j][4 * w + 1]);
+            const uint32_t a8 = aw[w] >> 8, b8 = bw[w] >> 8;
+            mma16816(acc[w], nib_lo(a8), nib_lo(b8), nib_hi(a8), nib_hi(b8), hr[j][4 * w + 2], hr[j][4 * w + 3]);
+        }
+    }
+    return diag_part(acc, lane);
+}
+
+// NDK = d / 1024, NF = f / 1024.
+template <int NDK, int NF>
+__global__ void __launch_bounds__(kFzThreads, 1) decode_fused_kernel(const FusedArgs a) {
+    // [kFzMaxStages][warps][stage]: stage s of every warp is one region; x (plain bf16, 2d bytes)
+    // lands in the last stage's region during phase A
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ __align__(8) uint64_t bars[kFzMaxWarps][kFzStages];
-    __shared__ int4 s_desc[kFzMaxWarps][kFzStages];       // gate/up stage: slot, row, scale slots
+    __shared__ __align__(8) uint64_t bars[kFzWarps][kFzMaxStages];
+    __shared__ int4 s_desc[kFzWarps][kFzMaxStages];       // gate/up stage: slot, row, scale slots
     __shared__ __align__(8) uint64_t s_xbar;              // x -> shared memory
     __shared__ __align__(8) uint64_t s_rbar;              // the router pieces -> shared memory
     __shared__ float ys[kFzMaxSlots][kFzRowsMax];
     __shared__ int s_e[kFzMaxSlots];                       // routed experts, ascending
+    __shared__ const uint8_t* s_gu[kFzMaxSlots];           // their weights (the layer's pointer table)
+    __shared__ const float* s_gus[kFzMaxSlots];
+    __shared__ const uint8_t* s_dn[kFzMaxSlots];
+    __shared__ const float* s_dns[kFzMaxSlots];
     __shared__ float s_w[kFzMaxSlots];                     // their gate weights
     __shared__ int sel_e[kFzMaxSlots];                     // rank order
     __shared__ int cand_e[kFzMaxPer * kFzMaxSlots];       // selection candidates, k per warp
     __shared__ uint2 cand_k[kFzMaxPer * kFzMaxSlots];     // and their keys
     __shared__ double sel_l[kFzMaxSlots];
     __shared__ unsigned long long s_base;                 // arrivals before this launch
-    __shared__ double s_xpart[kFzMaxWarps];                // sum of x per warp slice
     __shared__ int s_ok;
 
+    constexpr int d = 1024 * NDK, f = 1024 * NF;
     const int tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
-    const int nwc = blockDim.x / kWarp;
-    const int gw = blockIdx.x * nwc + warp, nw = gridDim.x * nwc;
     const int G = gridDim.x;
-    const int d = a.d, f = a.f, k = a.k, E = a.E;
-    const int nchunks = d / 32, nch = d / 1024;
-    const uint32_t gu_row = (uint32_t)d / 2, dn_row_b = (uint32_t)f / 2;
-    const uint32_t stage_bytes = 2 * gu_row + 32;
-    const uint32_t xp_s = saddr(smem);                     // x, pre-paired
-    uint8_t* const rings = smem + 2 * d;
-    const uint32_t rings_s = xp_s + 2u * d;
-    auto st_s = [&](int s) { return rings_s + ((uint32_t)s * nwc + warp) * stage_bytes; };
-    auto st_g = [&](int s) { return rings + ((size_t)s * nwc + warp) * stage_bytes; };
+    const int gw = warp * G + blockIdx.x, nw = G * kFzWarps;   // warp-major: low numbers on every SM
+    const int k = a.k, E = a.E;
+    constexpr int nst = NDK <= 6 ? kFzMaxStages : kFzMaxStages - 1;   // ring stages per warp
+    constexpr int nch = NDK;                               // 1024-column router pieces per expert
+    constexpr uint32_t gu_row = d / 2, dn_row_b = f / 2;
+    constexpr uint32_t stage_bytes = 2 * gu_row + 32;
+    const uint32_t rings_s = saddr(smem);
+    auto st_s = [&](int s) { return rings_s + ((uint32_t)s * kFzWarps + warp) * stage_bytes; };
+    auto st_g = [&](int s) { return smem + ((size_t)s * kFzWarps + warp) * stage_bytes; };
+    const uint32_t xraw_s = rings_s + (uint32_t)(nst - 1) * kFzWarps * stage_bytes;
     const int n_sh = a.S ? f : 0;                          // shared row pairs
     const int n_tasks = n_sh + k * f;
     auto count_of = [&](int lo, int hi) {                  // my tasks among [lo, hi)
@@ -223,7 +357,13 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
     const int j0 = (int)((int64_t)blockIdx.x * d / G), rj = (int)((int64_t)(blockIdx.x + 1) * d / G) - j0;
     const int nslots = k + a.S;
     const int n_items = nslots * rj;
-    const int it0 = (int)((int64_t)warp * n_items / nwc), it1 = (int)((int64_t)(warp + 1) * n_items / nwc);
+    const int it0 = (int)((int64_t)warp * n_items / kFzWarps), it1 = (int)((int64_t)(warp + 1) * n_items / kFzWarps);
+    // the lane's segment (g) and quarter (c): byte offsets within a gate/up row and a down row
+    const int lg = lane >> 2, lc = lane & 3;
+    const uint32_t gu_lane_off = (uint32_t)lg * (d / 16) + (uint32_t)lc * (16 * NDK);
+    const uint32_t dn_lane_off = (uint32_t)lg * (f / 16) + (uint32_t)lc * (16 * NF);
+    const int grot = gu_rot<NDK>(lane), drot = dn_rot<NF>(lane);
+    const uint64_t pol_first = policy_evict_first();
 
     unsigned long long* trace = a.trace + (size_t)blockIdx.x * kTraceStamps;
     auto stamp = [&](int i) {
@@ -231,7 +371,7 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
     };
     stamp(0);
     if (lane == 0) {
-        for (int s = 0; s < kFzStages; ++s) bar_init(saddr(&bars[warp][s]), 1);
+        for (int s = 0; s < nst; ++s) bar_init(saddr(&bars[warp][s]), 1);
         if (warp == 0) {
             bar_init(saddr(&s_xbar), 1);
             bar_init(saddr(&s_rbar), 1);
@@ -239,14 +379,12 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
-    // x (2d bytes) into the last stage's region, once per CTA
-    const uint32_t xraw_s = st_s(kFzStages - 1) - (uint32_t)warp * stage_bytes;
     if (tid == 0) {
         bar_expect_tx(saddr(&s_xbar), 2u * d);
         bulk_g2s(xraw_s, a.x, 2u * d, saddr(&s_xbar));
     }
 
-    // ---- the ring: use q of this warp goes to stage q % kFzStages
+    // ---- the ring: use q of this warp goes to stage q % nst
     //      q < my_tasks: gate/up row pair (task q); q >= my_tasks: down stage (lane 0's cursor)
     int issued = 0;               // lane 0: next use to issue
     int n_dn = 0;                 // this warp's down stages
@@ -256,8 +394,9 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
     int dn_u = it0 / max(rj, 1), dn_row = it0 - dn_u * rj, dn_it = it0;
     auto dn_count = [&](int it, int row) { return min(min(a.dn_rows, it1 - it), rj - row); };
     auto issue = [&](int q) {
-        const uint32_t bar = saddr(&bars[warp][q % kFzStages]);
-        const uint32_t dst = st_s(q % kFzStages);
+        const int sidx = q % nst;
+        const uint32_t bar = saddr(&bars[warp][sidx]);
+        const uint32_t dst = st_s(sidx);
         if (q < my_tasks) {
             const int t = gw + q * nw;
             const uint8_t* rows;
@@ -275,22 +414,20 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
                 }
                 r = gu_r;
                 slot = gu_u;
-                const size_t row = (size_t)s_e[gu_u] * 2 * f + gu_r;
-                rows = a.gate_up + row * gu_row;
-                sc = a.gu_scale + row;
+                rows = s_gu[gu_u] + (size_t)gu_r * gu_row;
+                sc = s_gus[gu_u] + gu_r;
                 for (gu_r += nw; gu_r >= f; gu_r -= f) ++gu_u;
             }
             // the consumer finds its row and, in the two 16-byte slivers, its two scales
-            s_desc[warp][q % kFzStages] = make_int4(slot, r, (int)(((uintptr_t)sc >> 2) & 3),
-                                                    4 + (int)(((uintptr_t)(sc + f) >> 2) & 3));
+            s_desc[warp][sidx] = make_int4(slot, r, (int)(((uintptr_t)sc >> 2) & 3), 4 + (int)(((uintptr_t)(sc + f) >> 2) & 3));
             bar_expect_tx(bar, stage_bytes);
-            bulk_g2s(dst, rows, gu_row, bar);
-            bulk_g2s(dst + gu_row, rows + (size_t)f * gu_row, gu_row, bar);
+            bulk_g2s_hint(dst, rows, gu_row, bar, pol_first);
+            bulk_g2s_hint(dst + gu_row, rows + (size_t)f * gu_row, gu_row, bar, pol_first);
             bulk_g2s(dst + 2 * gu_row, sliver(sc), 16, bar);
             bulk_g2s(dst + 2 * gu_row + 16, sliver(sc + f), 16, bar);
         } else {
             const int n = dn_count(dn_it, dn_row);
-            const uint8_t* W = dn_u < k ? a.down + (size_t)s_e[dn_u] * d * dn_row_b : a.sh_down;
+            const uint8_t* W = dn_u < k ? s_dn[dn_u] : a.sh_down;
             bar_expect_tx(bar, (uint32_t)n * dn_row_b);
             bulk_g2s(dst, W + (size_t)(j0 + dn_row) * dn_row_b, (uint32_t)n * dn_row_b, bar);
             dn_it += n;
@@ -302,68 +439,114 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
         }
     };
     auto wait_use = [&](int q) {
-        const bool ok = bar_wait(saddr(&bars[warp][q % kFzStages]), (uint32_t)(q / kFzStages) & 1u);
+        const bool ok = bar_wait(saddr(&bars[warp][q % nst]), (uint32_t)(q / nst) & 1u);
         __syncwarp();                                      // lane 0's stage descriptor is visible
         return __all_sync(0xffffffffu, ok);
     };
     auto drain = [&](int from) {      // lane 0: let every copy still in flight land
         if (lane == 0)
-            for (int q = from; q < issued; ++q)
-                bar_wait(saddr(&bars[warp][q % kFzStages]), (uint32_t)(q / kFzStages) & 1u);
+            for (int q2 = from; q2 < issued; ++q2)
+                bar_wait(saddr(&bars[warp][q2 % nst]), (uint32_t)(q2 / nst) & 1u);
     };
 
-    // ---- A: x (one bulk copy per CTA) and this warp's first router piece, both ahead of the
-    //      stream of expert rows, so that the router's inputs are not queued behind it
+    // ---- A: the shared expert's row pairs need no routing: queue them into every stage but the
+    //      last (which takes x), then this warp's first router piece, then wait for x
+    int limit = my_sh;            // lane 0: uses that may be issued so far
+    if (lane == 0)
+        while (issued < my_sh && issued < nst - 1) issue(issued++);
     const int n_units = E * nch;
-    // this warp's first router piece: its loads (coalesced, 512 bytes per instruction) are in
-    // flight while x lands and is rearranged
-    float4 rw[8];
+    // this warp's first two router pieces: every load of both in flight at once while x lands
+    float4 rw[8], rw2[8];
+    const int u2 = gw + nw;
     if (gw < n_units) {
         const int e = gw / nch, p = gw - e * nch;
         load_router_piece(a.router_w + (size_t)e * d + 1024 * p, lane, rw);
     }
+    if (u2 < n_units) {
+        const int e = u2 / nch, p = u2 - e * nch;
+        load_router_piece(a.router_w + (size_t)e * d + 1024 * p, lane, rw2);
+    }
+    // the shared expert's down rows of this CTA are read last: start pulling them into L2
+    if (a.S && tid == kWarp && rj > 0) prefetch_l2(a.sh_down + (size_t)j0 * dn_row_b, (uint32_t)rj * dn_row_b);
     bool ok = __all_sync(0xffffffffu, bar_wait(saddr(&s_xbar), 0u));
     stamp(11);
-    // x pre-paired into its own region (group g = columns 8g .. 8g + 7 goes to row g % 4 of chunk
-    // g / 4), and the sum of x: thread i adds groups i, i + threads, ... (fp32), each warp's
-    // total goes to shared memory (fp64).
+    // x as the lanes' fp16 MMA operand, once per CTA while the router loads are in flight: sigma
+    // from max|x|, then thread t converts the 8-column groups t, t + threads, ... into the lane
+    // blocks (lane L's block holds its groups in its visiting order; blocks are padded by 16 bytes
+    // so that the lanes' 16-byte loads meet no bank conflict).  The sum of x~ (fp64) is reduced
+    // in a fixed order, so every CTA gets the same value.
+    constexpr uint32_t kLaneBlk = 64 * NDK + 16;
+    const uint32_t xt_s = xraw_s + 2u * d;
+    __shared__ float s_redf[kFzWarps];
+    __shared__ double s_redd[kFzWarps];
+    int sig;
+    double xs;                    // sum of x~ = x 2^sigma over the whole row
     {
-        float xsl = 0.0f;
-        for (int g = tid; g < d / 8; g += blockDim.x) {
-            const uint4 v = lds16(xraw_s + (uint32_t)g * 16u);
-            uint32_t p[4];
-            pair_cols(v, p);
-            sts16(xp_s + (uint32_t)((g & 3) * nchunks + (g >> 2)) * 16u, make_uint4(p[0], p[1], p[2], p[3]));
+        float m = 0.0f;
+        for (int g = tid; g < d / 8; g += kFzThreads) {
+            const uint4 v = lds16(xraw_s + 16u * (uint32_t)g);
             const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) xsl += __uint_as_float(ws[i] << 16) + __uint_as_float(ws[i] & 0xffff0000u);
+            for (int i = 0; i < 4; ++i)
+                m = fmaxf(m, fmaxf(fabsf(__uint_as_float(ws[i] << 16)), fabsf(__uint_as_float(ws[i] & 0xffff0000u))));
         }
-        const double wsum = warp_sum_d((double)xsl);
-        if (lane == 0) s_xpart[warp] = wsum;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) s_redf[warp] = m;
+        __syncthreads();
+        m = 0.0f;
+        for (int w = 0; w < kFzWarps; ++w) m = fmaxf(m, s_redf[w]);
+        sig = scale_exp(m);
+        const float s1 = exp2i(sig), s16 = exp2i(sig - 4);
+        float part = 0.0f;
+        for (int g = tid; g < d / 8; g += kFzThreads) {
+            uint32_t pr[4];
+            pairs_from_bf16(lds16(xraw_s + 16u * (uint32_t)g), s1, s16, pr, part);
+            // group g belongs to lane L = 4 seg + quarter, as word w of its group q
+            const int seg = g / (d / 64), rem = g - seg * (d / 64);
+            const int cq = rem / (4 * NDK), rem2 = rem - cq * (4 * NDK);
+            const int q = rem2 >> 2, w = rem2 & 3, L = 4 * seg + cq;
+            int j = q - gu_rot<NDK>(L);
+            if (j < 0) j += NDK;
+            sts16(xt_s + (uint32_t)L * kLaneBlk + (uint32_t)(4 * j + w) * 16u, make_uint4(pr[0], pr[1], pr[2], pr[3]));
+        }
+        const double pd = warp_sum_d((double)part);
+        if (lane == 0) s_redd[warp] = pd;
+        __syncthreads();
+        xs = 0.0;
+        for (int w = 0; w < kFzWarps; ++w) xs += s_redd[w];
     }
+    // router pieces: unit u = (expert u / nch, columns [1024 p, 1024 p + 1024), p = u % nch)
+    auto piece = [&](int u, const float4 (&wv)[8]) {
+        const int p = u % nch;
+        const double v = warp_sum_d(router_piece(wv, xraw_s + 2048u * p, lane));
+        if (lane == 0) __stcg(a.rpart + u, v);
+    };
+    if (gw < n_units) piece(gw, rw);
+    if (u2 < n_units) piece(u2, rw2);
+    for (int u = gw + 2 * nw; u < n_units; u += nw) {
+        const int e = u / nch, p = u - e * nch;
+        load_router_piece(a.router_w + (size_t)e * d + 1024 * p, lane, rw);
+        piece(u, rw);
+    }
+    stamp(1);
+    // this lane's x~ registers, from its block
+    uint32_t xr[NDK][16];
+#pragma unroll
+    for (int j = 0; j < NDK; ++j)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const uint4 v = lds16(xt_s + (uint32_t)lane * kLaneBlk + (uint32_t)(4 * j + w) * 16u);
+            xr[j][4 * w] = v.x;
+            xr[j][4 * w + 1] = v.y;
+            xr[j][4 * w + 2] = v.z;
+            xr[j][4 * w + 3] = v.w;
+        }
+    const float xoff = 8.0f * (float)xs;                   // 8 sum x~
+    const float xunscale = exp2i(-sig) * 16777216.0f;      // 2^(24 - sigma)
     // this thread's selection bias
     const float my_bias = a.bias && tid < E ? a.bias[tid] : 0.0f;
-    __syncthreads();                                       // x is pre-paired
-    stamp(1);
-    // the shared expert's rows need no routing: queue them now (all stages but the last, which
-    // keeps x in plain order for the router pieces)
-    if (lane == 0)
-        while (issued < my_sh && issued < kFzStages - 1) issue(issued++);
-    // the shared expert's down rows of this CTA are read last: start pulling them into L2
-    if (a.S && tid == kWarp && rj > 0)
-        prefetch_l2(a.sh_down + (size_t)j0 * dn_row_b, (uint32_t)rj * dn_row_b);
-    double xs = 0.0;                                       // sum of x, the same order in every warp
-    for (int w = 0; w < nwc; ++w) xs += s_xpart[w];
-    const float off136 = 136.0f * (float)xs;
-
-    // router pieces: unit u = (expert u / nch, columns [1024 p, 1024 p + 1024), p = u % nch)
-    for (int u = gw; u < n_units; u += nw) {
-        const int e = u / nch, p = u - e * nch;
-        if (u != gw) load_router_piece(a.router_w + (size_t)e * d + 1024 * p, lane, rw);
-        const double v = warp_sum_d(router_piece(rw, xraw_s + 2048u * p, lane));
-        if (lane == 0) __stcg(a.rpart + u, v);
-    }
-    __syncthreads();                                       // the last stage is free
+    __syncthreads();                                       // the last stage (x) is free
     if (tid == 0) {                                        // barrier 0: every piece is stored
         const unsigned long long old = arrive(a.bar);
         s_base = old - old % (2ull * G);
@@ -372,7 +555,6 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
 
     // ---- one gate/up row pair: stage of use q.  Lane n of the warp keeps the n-th pending result
     //      (g, u, index into h); every 32 row pairs, and at the end, all lanes finish theirs at once.
-    int limit = my_sh;            // lane 0: uses that may be issued so far
     int n_pend = 0;
     float p_g = 0.0f, p_u = 0.0f;
     int p_h = 0;
@@ -385,18 +567,18 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
         }
         n_pend = 0;
     };
-    auto gate_up_use = [&](int q, float2 acc) {
-        const int s = q % kFzStages;
+    auto gate_up_use = [&](int q, float2 part) {
+        const int s = q % nst;
         const int4 dsc = s_desc[warp][s];
         const float* scs = reinterpret_cast<const float*>(st_g(s) + 2 * gu_row);
         const float sg = scs[dsc.z], su = scs[dsc.w];
         __syncwarp();                                      // the stage is free again
         if (lane == 0)
-            while (issued < limit && issued < q + 1 + kFzStages) issue(issued++);
-        const float ag = warp_sum(acc.x), au = warp_sum(acc.y);
+            while (issued < limit && issued < q + 1 + nst) issue(issued++);
+        const float ag = warp_sum(part.x), au = warp_sum(part.y);
         if (lane == n_pend) {
-            p_g = sg * (ag - off136);
-            p_u = su * (au - off136);
+            p_g = sg * fmaf(ag, xunscale, -xoff * exp2i(-sig));
+            p_u = su * fmaf(au, xunscale, -xoff * exp2i(-sig));
             p_h = dsc.x * f + dsc.y;
         }
         if (++n_pend == kWarp) flush();
@@ -405,9 +587,9 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
     int q = 0;                    // next use to consume
     for (; ok && q < my_sh; ++q) {                         // the shared expert's row pairs
         if (lane == 0)
-            while (issued < limit && issued < q + kFzStages) issue(issued++);
+            while (issued < limit && issued < q + nst) issue(issued++);
         if (!wait_use(q)) { ok = false; break; }
-        gate_up_use(q, gu_dot(st_s(q % kFzStages), gu_row, lane, xp_s, nchunks));
+        gate_up_use(q, gu_mma<NDK>(st_s(q % nst), gu_row, gu_lane_off, grot, xr, lane));
     }
 
     // ---- B: selection by the whole CTA once every piece of the logits is stored.  The rings are
@@ -415,6 +597,7 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
     __syncthreads();
     stamp(3);
     const uint32_t rbytes = ((uint32_t)n_units * 8u + 15u) & ~15u;
+    uint8_t* const rings = smem;
     uint2* keys = reinterpret_cast<uint2*>(rings + rbytes);    // keys, order-preserving integers
     double* lgs = reinterpret_cast<double*>(keys + E);
     if (tid == 0) {
@@ -499,16 +682,22 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
             if (lane < k) {
                 s_e[pk.pos] = pk.e;
                 s_w[pk.pos] = pk.w;
+                s_gu[pk.pos] = ex_gate_up(a.etab, E, pk.e);
+                s_gus[pk.pos] = ex_gu_scale(a.etab, E, pk.e);
+                s_dn[pk.pos] = ex_down(a.etab, E, pk.e);
+                s_dns[pk.pos] = ex_dn_scale(a.etab, E, pk.e);
                 if (blockIdx.x == 0) {
                     a.idx[lane] = pk.e;
                     a.wts[lane] = pk.w;
                     a.asc[pk.pos] = lane;
                     a.ulist[pk.pos] = pk.e;
                 }
+                // this CTA's down rows of the routed expert: into L2 while gate/up streams
+                if (rj > 0) prefetch_l2(ex_down(a.etab, E, pk.e) + (size_t)j0 * dn_row_b, (uint32_t)rj * dn_row_b);
             }
             if (blockIdx.x == 0 && lane == 0) {
                 *a.n_unique = k;
-                *a.xsum = xs;
+                *a.xsum = xs * (double)exp2i(-sig);
             }
         }
     }
@@ -520,6 +709,19 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
     stamp(6);
     const bool routed = sel;
 
+    // the scales of this warp's down items (slot, row), lane i holding item it0 + 32 r + i
+    float dsc_r[kFzScRegs];
+#pragma unroll
+    for (int r = 0; r < kFzScRegs; ++r) {
+        const int it = it0 + kWarp * r + lane;
+        float v = 0.0f;
+        if (routed && it < it1) {
+            const int u = it / rj, row = it - u * rj;
+            v = __ldg((u < k ? s_dns[u] : a.sh_dn_scale) + j0 + row);
+        }
+        dsc_r[r] = v;
+    }
+
     // ---- C: the routed row pairs; then the first down stages (independent of h)
     for (int it = it0, row = it0 - (it0 / max(rj, 1)) * rj; it < it1; ++n_dn) {
         const int n = dn_count(it, row);
@@ -530,12 +732,12 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
         limit = my_tasks + n_dn;
         for (; q < my_tasks; ++q) {
             if (lane == 0)
-                while (issued < limit && issued < q + kFzStages) issue(issued++);
+                while (issued < limit && issued < q + nst) issue(issued++);
             if (!wait_use(q)) { ok = false; break; }
-            gate_up_use(q, gu_dot(st_s(q % kFzStages), gu_row, lane, xp_s, nchunks));
+            gate_up_use(q, gu_mma<NDK>(st_s(q % nst), gu_row, gu_lane_off, grot, xr, lane));
         }
         if (ok && lane == 0)
-            while (issued < limit && issued < q + kFzStages) issue(issued++);
+            while (issued < limit && issued < q + nst) issue(issued++);
     }
     flush();
 
@@ -551,57 +753,71 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
     stamp(8);
     __syncthreads();
 
-    // ---- D: down rows of this CTA's output block, slot by slot
+    // ---- D: down rows of this CTA's output block, slot by slot, two rows per MMA
     if (ok && s_ok) {
-        uint32_t hr[NCF][16];
-        float hs = 0.0f;                                   // sum of this slot's h
+        uint32_t hr[NF][16];
+        float hoff = 0.0f, hun = 0.0f;                     // 8 sum h~, 2^(24 - tau) of the current slot
         int cu = it0 / max(rj, 1), crow = it0 - cu * rj, hu = -1;
         for (int it = it0; it < it1; ++q) {
             const int n = dn_count(it, crow);
-            const float* scp = (cu < k ? a.dn_scale + (size_t)s_e[cu] * d : a.sh_dn_scale) + j0 + crow;
-            const float my_sc = lane < n ? __ldg(scp + lane) : 0.0f;
             if (cu != hu) {                                // this slot's h (written by other CTAs)
-                float hl = 0.0f;
+                uint4 hv[NF][4];
+                float m = 0.0f;
 #pragma unroll
-                for (int j = 0; j < NCF; ++j) {
-                    const int c = lane + kWarp * j;
+                for (int j = 0; j < NF; ++j) {
+                    int qq = j + drot;
+                    if (qq >= NF) qq -= NF;
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        const uint4 v = ld_cg16(a.h + (size_t)cu * f + (size_t)c * 32 + 8 * m);
-                        pair_cols(v, &hr[j][4 * m]);
-                        const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
+                    for (int w = 0; w < 4; ++w) {
+                        hv[j][w] = ld_cg16(a.h + (size_t)cu * f + 8 * (lg * (f / 64) + lc * 4 * NF + 4 * qq + w));
+                        const uint32_t ws[4] = {hv[j][w].x, hv[j][w].y, hv[j][w].z, hv[j][w].w};
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&ws[i]));
-                            hl += hf.x + hf.y;
+                            m = fmaxf(m, fmaxf(fabsf(hf.x), fabsf(hf.y)));
                         }
                     }
                 }
-                hs = warp_sum(hl);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                const int tau = scale_exp(m);
+                const float s1 = exp2i(tau), s16 = exp2i(tau - 4);
+                float part = 0.0f;
+#pragma unroll
+                for (int j = 0; j < NF; ++j)
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) pairs_from_f16(hv[j][w], s1, s16, &hr[j][4 * w], part);
+                hoff = 8.0f * warp_sum(part);
+                hun = exp2i(-tau) * 16777216.0f;
                 hu = cu;
             }
             if (lane == 0)
-                while (issued < limit && issued < q + kFzStages) issue(issued++);
+                while (issued < limit && issued < q + nst) issue(issued++);
             if (!wait_use(q)) { ok = false; break; }
-            const uint32_t st = st_s(q % kFzStages);
+            const uint32_t st = st_s(q % nst);
 #pragma unroll 1
-            for (int rr = 0; rr < n; ++rr) {
-                float v0 = 0.0f, v1 = 0.0f;
-#pragma unroll
-                for (int j = 0; j < NCF; ++j) {
-                    const uint4 wv = lds16(st + (uint32_t)rr * dn_row_b + (uint32_t)(lane + kWarp * j) * 16);
-                    v0 = dot_word_f16top(wv.x, &hr[j][0], v0);
-                    v1 = dot_word_f16top(wv.y, &hr[j][4], v1);
-                    v0 = dot_word_f16top(wv.z, &hr[j][8], v0);
-                    v1 = dot_word_f16top(wv.w, &hr[j][12], v1);
+            for (int rr = 0; rr < n; rr += 2) {
+                const uint32_t rowA = st + (uint32_t)rr * dn_row_b;
+                const uint32_t rowB = rr + 1 < n ? rowA + dn_row_b : rowA;
+                const float2 pr = dn_mma<NF>(rowA, rowB, dn_lane_off, drot, hr, lane);
+                const float vA = warp_sum(pr.x), vB = warp_sum(pr.y);
+                const int iA = it + rr - it0, iB = iA + 1;
+                const float sA = __shfl_sync(0xffffffffu, dsc_r[0], iA & 31);
+                const float sA1 = __shfl_sync(0xffffffffu, dsc_r[1], iA & 31);
+                const float sA2 = __shfl_sync(0xffffffffu, dsc_r[2], iA & 31);
+                const float sB = __shfl_sync(0xffffffffu, dsc_r[0], iB & 31);
+                const float sB1 = __shfl_sync(0xffffffffu, dsc_r[1], iB & 31);
+                const float sB2 = __shfl_sync(0xffffffffu, dsc_r[2], iB & 31);
+                const float scA = iA < 32 ? sA : iA < 64 ? sA1 : sA2;
+                const float scB = iB < 32 ? sB : iB < 64 ? sB1 : sB2;
+                if (lane == 0) {
+                    ys[cu][crow + rr] = scA * fmaf(vA, hun, -hoff * hun * (1.0f / 16777216.0f));
+                    if (rr + 1 < n) ys[cu][crow + rr + 1] = scB * fmaf(vB, hun, -hoff * hun * (1.0f / 16777216.0f));
                 }
-                const float v = warp_sum(v0 + v1);         // sum (3/2 + s/16) h
-                const float srow = __shfl_sync(0xffffffffu, my_sc, rr);
-                if (lane == 0) ys[cu][crow + rr] = srow * fmaf(16.0f, v, -24.0f * hs);
             }
             __syncwarp();
             if (lane == 0)
-                while (issued < limit && issued < q + 1 + kFzStages) issue(issued++);
+                while (issued < limit && issued < q + 1 + nst) issue(issued++);
             it += n;
             crow += n;
             if (crow == rj) {
@@ -631,20 +847,30 @@ __global__ void __launch_bounds__(kFzMaxWarps * kWarp, 1) decode_fused_kernel(co
 }
 
 size_t fz_stage_bytes(const LayerDims& L) { return (size_t)L.d + 32; }
-int fz_warps(const LayerDims& L) {
-    const int w = (int)((kSmemLimit - kStaticReserve - 2 * (size_t)L.d) / ((size_t)kFzStages * fz_stage_bytes(L)));
-    return w > kFzMaxWarps ? kFzMaxWarps : w;
-}
-size_t fz_dyn_smem(const LayerDims& L) {
-    return 2 * (size_t)L.d + (size_t)fz_warps(L) * kFzStages * fz_stage_bytes(L);
-}
+// Ring stages per warp (the kernel's constant for its d): 4 up to d = 6144, 3 above.
+int fz_stages(const LayerDims& L) { return L.d / 1024 <= 6 ? kFzMaxStages : kFzMaxStages - 1; }
+size_t fz_dyn_smem(const LayerDims& L) { return (size_t)fz_stages(L) * kFzWarps * fz_stage_bytes(L); }
 int fz_dn_rows(const LayerDims& L) {
     const int r = (int)(fz_stage_bytes(L) / (size_t)(L.f / 2));
     return r > kFzDnRowsMax ? kFzDnRowsMax : r;
 }
 
+template <int NDK>
+const void* fz_pick_f(int nf) {
+    return nf == 1 ? (const void*)decode_fused_kernel<NDK, 1> : (const void*)decode_fused_kernel<NDK, 2>;
+}
 const void* fz_pick(const LayerDims& L) {
-    return L.f / 1024 == 1 ? (const void*)decode_fused_kernel<1> : (const void*)decode_fused_kernel<2>;
+    const int nf = L.f / 1024;
+    switch (L.d / 1024) {
+        case 1: return fz_pick_f<1>(nf);
+        case 2: return fz_pick_f<2>(nf);
+        case 3: return fz_pick_f<3>(nf);
+        case 4: return fz_pick_f<4>(nf);
+        case 5: return fz_pick_f<5>(nf);
+        case 6: return fz_pick_f<6>(nf);
+        case 7: return fz_pick_f<7>(nf);
+        default: return fz_pick_f<8>(nf);
+    }
 }
 
 }  // namespace
@@ -652,18 +878,21 @@ const void* fz_pick(const LayerDims& L) {
 bool decode_fused_shape_ok(const LayerDims& L) {
     if (!(L.wkind == MOE_W_INT4_ROWSCALE && L.d % 1024 == 0 && L.d / 1024 >= 1 && L.d / 1024 <= 8 &&
           (L.f == 1024 || L.f == 2048) && (!L.S || L.f_shared == L.f) && L.k + L.S <= kFzMaxSlots &&
-          L.E <= kWarp * kFzMaxPer && L.k <= L.E && fz_warps(L) >= 4 && fz_dn_rows(L) >= 1))
+          L.E <= kWarp * kFzMaxPer && L.k <= L.E && fz_dn_rows(L) >= 1 &&
+          fz_dyn_smem(L) + kStaticReserve <= kSmemLimit))
         return false;
     // the selection keeps the router pieces, keys and logits in the (idle) rings; E <= threads
-    const size_t dyn = (size_t)fz_warps(L) * kFzStages * fz_stage_bytes(L);   // the rings
     const size_t sel_bytes = ((size_t)L.E * (L.d / 1024) * 8 + 15) / 16 * 16 + 16 * (size_t)L.E;
-    return sel_bytes <= dyn && L.E <= fz_warps(L) * kWarp;
+    return sel_bytes <= fz_dyn_smem(L) && L.E <= kFzThreads;
 }
 
 cudaError_t prepare_decode_fused(const LayerDims& L, int num_sms, bool* usable) {
     *usable = false;
     if (!decode_fused_shape_ok(L) || (L.d + num_sms - 1) / num_sms > kFzRowsMax || num_sms > kTraceCtas)
         return cudaSuccess;
+    // the down items of one warp must fit the scale registers
+    const int rows = (L.d + num_sms - 1) / num_sms;
+    if ((L.k + L.S) * rows > kFzWarps * kWarp * kFzScRegs - kFzWarps) return cudaSuccess;
     int dev = 0, coop = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
@@ -677,7 +906,7 @@ cudaError_t prepare_decode_fused(const LayerDims& L, int num_sms, bool* usable) 
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(kSmemLimit - fa.sharedSizeBytes));
     if (e != cudaSuccess) return e;
     int blocks = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, fn, fz_warps(L) * kWarp, dyn);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, fn, kFzThreads, dyn);
     if (e != cudaSuccess) return e;
     *usable = blocks >= 1;
     return cudaSuccess;
@@ -691,14 +920,11 @@ cudaError_t launch_decode_fused(const LayerDims& L, const moe_weights& W, const 
     a.router_w = W.router_w;
     a.bias = L.router == MOE_ROUTER_SIGMOID_BIAS ? W.router_bias : nullptr;
     a.x = x;
-    a.gate_up = (const uint8_t*)W.gate_up;
-    a.gu_scale = W.gate_up_scale;
     a.sh_gate_up = (const uint8_t*)W.shared_gate_up;
     a.sh_gu_scale = W.shared_gate_up_scale;
-    a.down = (const uint8_t*)W.down;
-    a.dn_scale = W.down_scale;
     a.sh_down = (const uint8_t*)W.shared_down;
     a.sh_dn_scale = W.shared_down_scale;
+    a.etab = (const void* const*)ws.etab;
     a.rpart = ws.rpart;
     a.h = ws.h;
     a.out = out;
@@ -720,10 +946,9 @@ cudaError_t launch_decode_fused(const LayerDims& L, const moe_weights& W, const 
     a.out_bf16 = L.out_bf16;
     a.dn_rows = fz_dn_rows(L);
     a.scaling = L.scaling;
-    const int warps = fz_warps(L);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)num_sms);
-    cfg.blockDim = dim3((unsigned)(warps * kWarp));
+    cfg.blockDim = dim3((unsigned)kFzThreads);
     cfg.dynamicSmemBytes = fz_dyn_smem(L);
     cfg.stream = ctx.s;
     cudaLaunchAttribute attr[1];

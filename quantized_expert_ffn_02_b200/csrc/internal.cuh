@@ -116,6 +116,10 @@ struct Workspace {
     float* xsum_slot;      // [slots]: sum of x of each slot's token (gate/up GEMM epilogue)
     uint32_t* counter;     // [1]: blocks done in the fused small-batch router (reset to 0 by the last)
     // single-launch decode path
+    // the routed experts' weights, one pointer each: [0, E) gate/up rows, [E, 2E) gate/up scales,
+    // [2E, 3E) down rows, [3E, 4E) down scales.  Filled from the contiguous [E] arrays at layer
+    // creation; moe_layer_set_expert re-points one expert (a non-contiguous expert slab).
+    const void** etab;
     double* rpart;         // [E][d / 1024]: pieces of the router logits
     unsigned long long* gbar;  // [1]: grid-barrier arrivals (only grows)
     unsigned long long* trace; // [kTraceCtas][kTraceStamps]: phase timestamps of that path
@@ -123,10 +127,40 @@ struct Workspace {
 constexpr int kTraceCtas = 1024;
 constexpr int kTraceStamps = 16;
 
+// Router variants (colibri README: the DeepSeek-V3 router's noaux_tc, and the --topp adaptive
+// expert top-p knob): group-limited selection when n_group > 1 -- the E experts form n_group
+// contiguous groups, a group's score is the sum of its two largest keys, and only the topk_group
+// best groups (equal scores: the lower group first) stay selectable -- and, for top_p in (0, 1),
+// the shortest rank-order prefix whose weights reach top_p of the k weights' total, rescaled to
+// that total, the rest dropped (index -1, weight 0).  The defaults are the plain router.
+struct RouterOpts {
+    int n_group = 1, topk_group = 1;
+    double top_p = 0.0;
+    bool active() const { return n_group > 1 || (top_p > 0.0 && top_p < 1.0); }
+};
+
+// Routed expert e's weights through the layer's pointer table ([4][E]; no kernel writes it while
+// another reads it, so it goes through the read-only cache).
+__device__ __forceinline__ const uint8_t* ex_gate_up(const void* const* t, int E, int e) {
+    return reinterpret_cast<const uint8_t*>(__ldg(reinterpret_cast<const unsigned long long*>(t) + e));
+}
+__device__ __forceinline__ const float* ex_gu_scale(const void* const* t, int E, int e) {
+    return reinterpret_cast<const float*>(__ldg(reinterpret_cast<const unsigned long long*>(t) + E + e));
+}
+__device__ __forceinline__ const uint8_t* ex_down(const void* const* t, int E, int e) {
+    return reinterpret_cast<const uint8_t*>(__ldg(reinterpret_cast<const unsigned long long*>(t) + 2 * E + e));
+}
+__device__ __forceinline__ const float* ex_dn_scale(const void* const* t, int E, int e) {
+    return reinterpret_cast<const float*>(__ldg(reinterpret_cast<const unsigned long long*>(t) + 3 * E + e));
+}
+
 struct LayerDims {
     int d, f, E, k, S, f_shared, router, wkind, out_bf16;
     float scaling;
     int pdl = 1;           // chain dependent kernels with programmatic dependent launch
+    uint64_t wait_ns = 2000000000ull;   // limit of the grouped-GEMM kernels' bounded waits
+    int test_skip_b = 0;   // test hook: the grouped GEMM's B producer issues no copies
+    RouterOpts ropts;      // router variants (off by default)
 };
 
 // Optional per-kernel event timing (defined in layer.cu).  `prof` may be null.
@@ -146,6 +180,9 @@ cudaError_t prepare_bucket(const LayerDims& L);
 cudaError_t prepare_decode(const LayerDims& L);
 
 cudaError_t launch_pack_int4(const float* w, int64_t rows, int64_t cols, uint8_t* packed, float* scales,
+                             int* status, cudaStream_t s);
+// bits = 8 (int8 container) or 2 (packed int2)
+cudaError_t launch_pack_tier(int bits, const float* w, int64_t rows, int64_t cols, uint8_t* packed, float* scales,
                              int* status, cudaStream_t s);
 cudaError_t launch_router(const LayerDims& L, const float* router_w, const float* router_bias,
                           const uint16_t* x, int T, double* logits, double* xsum, int32_t* idx, float* wts,

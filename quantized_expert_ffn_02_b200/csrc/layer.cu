@@ -85,6 +85,7 @@ struct moe_layer {
     int64_t prefill_min_tokens = 128;    // batches at least this large take the grouped-GEMM path
     int t1_mode = 0;                     // T = 1: 2 single launch, 1 single-token kernels, 0 general
     bool fused_ok = false;               // the single-launch path is usable for this layer
+    bool ragged = false;                 // some routed expert lives outside the contiguous [E] arrays
 };
 
 namespace {
@@ -98,6 +99,24 @@ moe_status from_cuda(cudaError_t e) {
 }
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Bytes of one weight row of `cols` columns in the container (scales are separate arrays).
+size_t row_bytes(int wkind, size_t cols) {
+    switch (wkind) {
+        case MOE_W_INT4_ROWSCALE: return cols / 2;
+        case MOE_W_INT8_ROWSCALE: return cols;
+        case MOE_W_INT2_ROWSCALE: return cols / 4;
+        default: return cols * 2;
+    }
+}
+
+__global__ void set_expert_kernel(const void** etab, int E, int e, const void* gu, const void* gus, const void* dn,
+                                  const void* dns) {
+    etab[e] = gu;
+    etab[E + e] = gus;
+    etab[2 * E + e] = dn;
+    etab[3 * E + e] = dns;
+}
 
 // Carves the workspace out of one allocation.  With base == nullptr it only measures.
 // max_groups > 0 adds the grouped-GEMM path's buffers.
@@ -129,6 +148,7 @@ size_t carve(const moe_config& c, size_t max_groups, char* base, qe::Workspace* 
     w.Y = (float*)take(sizeof(float) * slots * (size_t)c.d);
     w.status = (int32_t*)take(sizeof(int32_t));
     w.counter = (uint32_t*)take(sizeof(uint32_t));
+    w.etab = (const void**)take(sizeof(void*) * 4 * E);
     w.rpart = (double*)take(sizeof(double) * E * (c.d / 1024 > 0 ? (size_t)c.d / 1024 : 1));
     w.gbar = (unsigned long long*)take(sizeof(unsigned long long));
     w.trace = (unsigned long long*)take(sizeof(unsigned long long) * qe::kTraceCtas * qe::kTraceStamps);
@@ -155,11 +175,11 @@ moe_status check_config(const moe_config* c, const moe_weights* w) {
     if (c->n_shared && (c->f_shared <= 0 || c->f_shared % 64)) return MOE_ERR_INVALID_ARG;
     if (c->max_tokens < 1) return MOE_ERR_INVALID_ARG;
     if (c->router != MOE_ROUTER_SOFTMAX_TOPK && c->router != MOE_ROUTER_SIGMOID_BIAS) return MOE_ERR_INVALID_ARG;
-    if (c->wkind != MOE_W_INT4_ROWSCALE && c->wkind != MOE_W_BF16) return MOE_ERR_INVALID_ARG;
+    if (c->wkind < MOE_W_INT4_ROWSCALE || c->wkind > MOE_W_INT2_ROWSCALE) return MOE_ERR_INVALID_ARG;
     if (!(c->routed_scaling_factor == c->routed_scaling_factor)) return MOE_ERR_INVALID_ARG;
     if (c->d > 14336) return MOE_ERR_UNSUPPORTED;     // router x tile must fit in shared memory
     if ((size_t)c->max_tokens * (size_t)(c->top_k + 1) > (size_t)INT32_MAX / 2) return MOE_ERR_UNSUPPORTED;
-    const bool q = c->wkind == MOE_W_INT4_ROWSCALE;
+    const bool q = c->wkind != MOE_W_BF16;     // a container with per-row scales
     if (!w->router_w || !w->gate_up || !w->down) return MOE_ERR_INVALID_ARG;
     if (q && (!w->gate_up_scale || !w->down_scale)) return MOE_ERR_INVALID_ARG;
     if (c->n_shared && (!w->shared_gate_up || !w->shared_down)) return MOE_ERR_INVALID_ARG;
@@ -209,6 +229,38 @@ moe_status moe_pack_int4(const float* w, int64_t rows, int64_t cols, uint8_t* pa
     return host_status ? (moe_status)host_status : MOE_OK;
 }
 
+// The int8 and packed int2 tiers: the same synchronous shape as moe_pack_int4.
+static moe_status pack_tier(int bits, const float* w, int64_t rows, int64_t cols, uint8_t* packed, float* scales,
+                            moe_stream stream) {
+    const int per_byte = 8 / bits;
+    if (rows < 0 || cols <= 0 || (cols % per_byte)) return MOE_ERR_INVALID_ARG;
+    if (rows == 0) return MOE_OK;
+    if (!w || !packed || !scales) return MOE_ERR_INVALID_ARG;
+    if (((uintptr_t)w & 3) || ((uintptr_t)scales & 3)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    int* status = nullptr;
+    cudaError_t e = cudaMallocAsync((void**)&status, sizeof(int), s);
+    if (e != cudaSuccess) return from_cuda(e);
+    e = cudaMemsetAsync(status, 0, sizeof(int), s);
+    if (e == cudaSuccess) e = qe::launch_pack_tier(bits, w, rows, cols, packed, scales, status, s);
+    int host_status = 0;
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&host_status, status, sizeof(int), cudaMemcpyDeviceToHost, s);
+    cudaError_t e2 = cudaFreeAsync(status, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = e2;
+    if (e != cudaSuccess) return from_cuda(e);
+    return host_status ? (moe_status)host_status : MOE_OK;
+}
+
+moe_status moe_pack_int8(const float* w, int64_t rows, int64_t cols, int8_t* q, float* scales, moe_stream stream) {
+    return pack_tier(8, w, rows, cols, reinterpret_cast<uint8_t*>(q), scales, stream);
+}
+
+moe_status moe_pack_int2(const float* w, int64_t rows, int64_t cols, uint8_t* packed, float* scales,
+                         moe_stream stream) {
+    return pack_tier(2, w, rows, cols, packed, scales, stream);
+}
+
 moe_status moe_layer_create(const moe_config* cfg, const moe_weights* w, moe_layer** out) {
     if (!out) return MOE_ERR_INVALID_ARG;
     moe_status st = check_config(cfg, w);
@@ -243,6 +295,20 @@ moe_status moe_layer_create(const moe_config* cfg, const moe_weights* w, moe_lay
     }
     carve(*cfg, max_groups, (char*)L->ws_base, &L->ws, &L->x_stage, &L->out_stage);
     e = cudaMemset(L->ws_base, 0, L->ws_bytes);
+    if (e == cudaSuccess) {
+        // the pointer table: expert e at its place in the contiguous [E] arrays
+        const size_t E = (size_t)cfg->n_experts, f = (size_t)cfg->f, d = (size_t)cfg->d;
+        const size_t gu_bytes = 2 * f * row_bytes(cfg->wkind, d), dn_bytes = d * row_bytes(cfg->wkind, f);
+        std::vector<const void*> tab(4 * E);
+        const bool scaled = cfg->wkind != MOE_W_BF16;
+        for (size_t i = 0; i < E; ++i) {
+            tab[i] = static_cast<const char*>(w->gate_up) + i * gu_bytes;
+            tab[E + i] = scaled ? w->gate_up_scale + i * 2 * f : nullptr;
+            tab[2 * E + i] = static_cast<const char*>(w->down) + i * dn_bytes;
+            tab[3 * E + i] = scaled ? w->down_scale + i * d : nullptr;
+        }
+        e = cudaMemcpy(L->ws.etab, tab.data(), sizeof(void*) * 4 * E, cudaMemcpyHostToDevice);
+    }
     if (e != cudaSuccess) {
         cudaFree(L->ws_base);
         delete L;
@@ -266,6 +332,7 @@ moe_status moe_route(moe_layer* L, const uint16_t* x, int32_t T, int32_t* idx, f
     if (!L || T < 0 || T > L->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!x || !idx || !w || !aligned16(x) || ((uintptr_t)idx & 3) || ((uintptr_t)w & 3)) return MOE_ERR_INVALID_ARG;
+    cudaGetLastError();   // an error left pending by an earlier, unrelated call is not this call's
     cudaStream_t s = (cudaStream_t)stream;
     int launches = 0;
     const qe::Launch ctx{s, &launches, &L->prof};
@@ -280,13 +347,16 @@ moe_status moe_forward(moe_layer* L, const uint16_t* x, int32_t T, void* out, mo
     if (!L || T < 0 || T > L->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!x || !out || !aligned16(x) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    cudaGetLastError();   // an error left pending by an earlier, unrelated call is not this call's
     cudaStream_t s = (cudaStream_t)stream;
     int launches = 0;
     const qe::Launch ctx{s, &launches, &L->prof};
     const qe::Workspace& ws = L->ws;
-    const bool gemm = L->plan && T >= L->prefill_min_tokens;
+    const bool gemm = L->plan && !L->ragged && T >= L->prefill_min_tokens;
     cudaError_t e;
-    if (T == 1 && L->t1_mode == 2) {
+    // the single-token paths take the plain router only (a router variant may drop experts)
+    const bool variant = L->dims.ropts.active();
+    if (T == 1 && L->t1_mode == 2 && !variant) {
         e = qe::launch_decode_fused(L->dims, L->w, x, ws, out, L->num_sms, ctx);
         L->last_stream = s;
         L->last_launches = launches;
@@ -303,7 +373,7 @@ moe_status moe_forward(moe_layer* L, const uint16_t* x, int32_t T, void* out, mo
         if (gemm) {
             e = qe::launch_prefill_experts(L->dims, L->plan, L->w, x, T, ws, L->num_sms, ctx);
             if (e == cudaSuccess) e = qe::launch_combine(L->dims, T, ws, out, ctx);
-        } else if (T == 1 && L->t1_mode >= 1) {
+        } else if (T == 1 && L->t1_mode >= 1 && !variant) {
             e = qe::launch_decode_t1(L->dims, L->w, x, ws, out, L->num_sms, ctx);
         } else {
             e = qe::launch_decode_experts(L->dims, L->w, x, T, ws, L->num_sms, ctx);
@@ -313,6 +383,24 @@ moe_status moe_forward(moe_layer* L, const uint16_t* x, int32_t T, void* out, mo
     L->last_stream = s;
     L->last_launches = launches;
     return from_cuda(e);
+}
+
+moe_status moe_layer_set_expert(moe_layer* L, int32_t e, const void* gate_up, const float* gate_up_scale,
+                                const void* down, const float* down_scale, moe_stream stream) {
+    if (!L || e < 0 || e >= L->cfg.n_experts || !gate_up || !down) return MOE_ERR_INVALID_ARG;
+    const bool scaled = L->cfg.wkind != MOE_W_BF16;
+    if (scaled && (!gate_up_scale || !down_scale)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(gate_up) || !aligned16(down) || (scaled && (!aligned16(gate_up_scale) || !aligned16(down_scale))))
+        return MOE_ERR_INVALID_ARG;
+    cudaGetLastError();
+    cudaStream_t s = (cudaStream_t)stream;
+    set_expert_kernel<<<1, 1, 0, s>>>(L->ws.etab, L->cfg.n_experts, e, gate_up, scaled ? gate_up_scale : nullptr, down,
+                                      scaled ? down_scale : nullptr);
+    const cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return from_cuda(err);
+    L->ragged = true;
+    L->last_stream = s;
+    return MOE_OK;
 }
 
 moe_status moe_forward_host_async(moe_layer* L, const uint16_t* x_host, int32_t T, void* out_host,
@@ -378,6 +466,32 @@ moe_status moe_layer_set_option(moe_layer* L, int32_t option, int64_t value) {
             if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
             L->dims.pdl = (int)value;
             return MOE_OK;
+        case MOE_OPT_WAIT_LIMIT_US:
+            if (value < 100 || value > 10000000) return MOE_ERR_INVALID_ARG;
+            L->dims.wait_ns = (uint64_t)value * 1000ull;
+            return MOE_OK;
+        case MOE_OPT_TEST_SKIP_GEMM_B_COPIES:
+            if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+            L->dims.test_skip_b = (int)value;
+            return MOE_OK;
+        case MOE_OPT_ROUTER_GROUPS: {
+            const int G = (int)(value & 0xFFFF), TG = (int)(value >> 16);
+            if (value < 0 || G < 1) return MOE_ERR_INVALID_ARG;
+            if (G == 1) {
+                L->dims.ropts.n_group = 1;
+                L->dims.ropts.topk_group = 1;
+                return MOE_OK;
+            }
+            const int E = L->cfg.n_experts;
+            if (G > 32 || E % G || TG < 1 || TG > G || (int64_t)TG * (E / G) < L->cfg.top_k) return MOE_ERR_INVALID_ARG;
+            L->dims.ropts.n_group = G;
+            L->dims.ropts.topk_group = TG;
+            return MOE_OK;
+        }
+        case MOE_OPT_ROUTER_TOP_P:
+            if (value < 0 || value > 1000000) return MOE_ERR_INVALID_ARG;
+            L->dims.ropts.top_p = (double)value * 1e-6;
+            return MOE_OK;
         default:
             return MOE_ERR_INVALID_ARG;
     }
@@ -412,9 +526,15 @@ moe_status moe_layer_get_option(const moe_layer* L, int32_t option, int64_t* val
     if (!L || !value) return MOE_ERR_INVALID_ARG;
     switch (option) {
         case MOE_OPT_PREFILL_MIN_TOKENS: *value = L->prefill_min_tokens; return MOE_OK;
-        case MOE_OPT_PREFILL_AVAILABLE: *value = L->plan ? 1 : 0; return MOE_OK;
+        case MOE_OPT_PREFILL_AVAILABLE: *value = L->plan && !L->ragged ? 1 : 0; return MOE_OK;
         case MOE_OPT_SINGLE_TOKEN_KERNELS: *value = L->t1_mode; return MOE_OK;
         case MOE_OPT_PROGRAMMATIC_LAUNCH: *value = L->dims.pdl; return MOE_OK;
+        case MOE_OPT_WAIT_LIMIT_US: *value = (int64_t)(L->dims.wait_ns / 1000ull); return MOE_OK;
+        case MOE_OPT_TEST_SKIP_GEMM_B_COPIES: *value = L->dims.test_skip_b; return MOE_OK;
+        case MOE_OPT_ROUTER_GROUPS:
+            *value = L->dims.ropts.n_group + ((int64_t)L->dims.ropts.topk_group << 16);
+            return MOE_OK;
+        case MOE_OPT_ROUTER_TOP_P: *value = (int64_t)(L->dims.ropts.top_p * 1e6 + 0.5); return MOE_OK;
         default: return MOE_ERR_INVALID_ARG;
     }
 }

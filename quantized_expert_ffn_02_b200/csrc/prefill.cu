@@ -24,15 +24,17 @@
 // in that order and the GEMM-1 epilogue writes h in that order.  A dot product does not depend
 // on the order of its terms.
 //
-// Roles (192 threads, one CTA per SM, persistent over tiles):
-//   warp 0    TMA producer of the packed A rows                 smem ring of 128 KB (16 or 32 stages)
-//   warp 10   TMA producer of the B tiles                       smem ring of kBStages
-//   warp 1    TMEM allocator and MMA issuer                      TMEM A ring of kAStages
-//   warps 2-9 converters (A rows -> TMEM), then the epilogue     thread <-> TMEM lane; two sets
-//             of four (one warp per TMEM lane quarter each) take alternate K steps and alternate
-//             16-column blocks of the epilogue
-// Every wait is bounded (about 2 s); on expiry the CTA latches MOE_ERR_TIMEOUT, drains what it
-// issued, frees its TMEM and returns.
+// Roles (608 threads, one CTA per SM, persistent over tiles):
+//   warp 0     TMA producer of the packed A rows                 smem ring of 128 KB (16 or 32 stages)
+//   warp 18    TMA producer of the B tiles (a box of 16, 32, 64 smem ring of kBStages
+//              or 128 rows: the group's tokens rounded up)
+//   warp 1     TMEM allocator and MMA issuer                      TMEM A ring of kAStages
+//   warps 2-17 converters (A rows -> TMEM), then the epilogue    thread <-> TMEM lane; four sets
+//              of four (one warp per TMEM lane quarter each) take every fourth K step, so a
+//              set has four MMA steps to hide its TMEM store, and every fourth 16-column block
+//              of the epilogue
+// Every wait is bounded (2 s by default; the layer option MOE_OPT_WAIT_LIMIT_US sets it); on
+// expiry the CTA latches MOE_ERR_TIMEOUT, drains what it issued, frees its TMEM and returns.
 #include "internal.cuh"
 
 #include <cuda.h>
@@ -57,11 +59,13 @@ constexpr int kBStages = 4;                           // B tiles (x or h, from L
 constexpr uint32_t kASmBytes = 128 * 1024;            // packed A tiles (from HBM) in shared memory
 constexpr int kASmStagesMax = 32;
 constexpr int kAStages = 4;                           // converted A tiles in TMEM
-constexpr int kGemmThreads = 352;
+constexpr int kConvSets = 4;                          // converter warp sets, one K step in kConvSets each
+constexpr int kConvWarps = 4 * kConvSets;             // one warp per TMEM lane quarter per set
+constexpr int kBWarp = 2 + kConvWarps;                // the B producer
+constexpr int kGemmThreads = (kBWarp + 1) * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kPackedTile = BM * BK / 2;         // 4 KB of packed int4 per 128 x 64 tile
 constexpr uint32_t kBTile = BN * BK * 2;              // 16 KB of bf16 / fp16
-constexpr uint64_t kWaitLimitNs = 2000000000ull;      // 2 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -97,16 +101,16 @@ __device__ __forceinline__ uint64_t globaltimer() {
     return t;
 }
 
-// Bounded wait on an mbarrier phase.  Gives up when another role has aborted, or after the
-// time limit (then it latches the timeout and raises the CTA's abort flag).
-__device__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status) {
+// Bounded wait on an mbarrier phase.  Gives up when another role has aborted, or after
+// limit_ns (then it latches the timeout and raises the CTA's abort flag).
+__device__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status, uint64_t limit_ns) {
     if (mbar_try(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try(bar, parity)) return true;
         if ((it & 63) == 0) {
             if (*abort_flag) return false;
-            if (globaltimer() - t0 > kWaitLimitNs) {
+            if (globaltimer() - t0 > limit_ns) {
                 *abort_flag = 1;
                 latch_status(status, MOE_ERR_TIMEOUT);
                 return false;
@@ -115,10 +119,10 @@ __device__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag
     }
 }
 // Bounded wait used while draining (ignores the abort flag).
-__device__ bool wait_bar_drain(uint32_t bar, uint32_t parity) {
+__device__ bool wait_bar_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
     const uint64_t t0 = globaltimer();
     while (!mbar_try(bar, parity))
-        if (globaltimer() - t0 > kWaitLimitNs) return false;
+        if (globaltimer() - t0 > limit_ns) return false;
     return true;
 }
 
@@ -239,6 +243,8 @@ struct GemmArgs {
     void* out;                // h (fp16 bits) or Y (fp32)
     int* status;
     const float* xsum_slot;   // gate/up: sum of x of each slot's token
+    uint64_t wait_ns;         // limit of every bounded wait
+    int skip_b;               // test hook: the B producer issues no copies (the MMA's wait runs out)
 };
 
 template <bool GATED>
@@ -284,7 +290,9 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, int t, int nr) {
 template <bool GATED>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA_sh,
-            const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+            const __grid_constant__ CUtensorMap tmB16, const __grid_constant__ CUtensorMap tmB32,
+            const __grid_constant__ CUtensorMap tmB64, const __grid_constant__ CUtensorMap tmB128,
+            const GemmArgs args) {
     constexpr int NA = GATED ? 2 : 1;                     // A tiles per stage
     // The packed weights stream from HBM and need many bytes in flight; B comes from L2.  So A and
     // B have rings of their own, A's much deeper.
@@ -298,7 +306,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     __shared__ __align__(8) uint64_t bars[2 * kASmStagesMax + 2 * kBStages + 2 * kAStages + 3];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
-    __shared__ int consumed_sh[8];                        // A stages consumed by each converter warp
+    __shared__ int consumed_sh[kConvWarps];               // A stages consumed by each converter warp
     __shared__ int issued_sh;                             // A stages issued
     __shared__ int b_issued_sh, b_consumed_sh;
     const uint32_t bar0 = smem_u32(bars);
@@ -327,7 +335,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             mbar_init(aempty_bar(s), 1);
         }
         mbar_init(accfull_bar, 1);
-        mbar_init(accempty_bar, 8);
+        mbar_init(accempty_bar, kConvWarps);
         mbar_init(final_bar, 1);
         abort_flag = 0;
         issued_sh = 0;
@@ -354,6 +362,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     const int n_tiles = nr * args.mt_r + ns * args.mt_s;
     volatile int* abortp = &abort_flag;
     int* status = args.status;
+    const uint64_t lim = args.wait_ns;
 
     if (warp == 0) {
         // ------------------------------------------------------------------ TMA producer
@@ -365,7 +374,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 const CUtensorMap* mapA = tl.shared ? &tmA_sh : &tmA;
                 for (int kk = 0; kk < tl.ksteps; ++kk, ++ks) {
                     const int s = ks % kSA;
-                    if (!(ok = wait_bar(empty_bar(s), ((ks / kSA) & 1) ^ 1, abortp, status))) break;
+                    if (!(ok = wait_bar(empty_bar(s), ((ks / kSA) & 1) ^ 1, abortp, status, lim))) break;
                     mbar_expect_tx(full_bar(s), NA * kPackedTile);
                     tma_load_2d(sA + s * NA * kPackedTile, mapA, full_bar(s), kk * (BK / 2), tl.a_row0);
                     if (GATED) tma_load_2d(sA + s * NA * kPackedTile + kPackedTile, mapA, full_bar(s), kk * (BK / 2),
@@ -383,12 +392,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 const Tile tl = decode_tile<GATED>(args, t, nr);
                 const int nmma = (tl.n + 15) & ~15;
                 const uint32_t idesc = idesc_f16(nmma, GATED);
-                if (!(ok = wait_bar(accempty_bar, (tc & 1) ^ 1, abortp, status))) break;
+                if (!(ok = wait_bar(accempty_bar, (tc & 1) ^ 1, abortp, status, lim))) break;
                 tc_fence_after();
                 for (int kk = 0; kk < tl.ksteps; ++kk, ++ks) {
                     const int s = ks % kBStages, sa = ks % kAStages;
-                    if (!(ok = wait_bar(bfull_bar(s), (ks / kBStages) & 1, abortp, status))) break;
-                    if (!(ok = wait_bar(afull_bar(sa), (ks / kAStages) & 1, abortp, status))) break;
+                    if (!(ok = wait_bar(bfull_bar(s), (ks / kBStages) & 1, abortp, status, lim))) break;
+                    if (!(ok = wait_bar(afull_bar(sa), (ks / kAStages) & 1, abortp, status, lim))) break;
                     tc_fence_after();
                     const uint64_t bdesc = sw128_desc(sB + s * kBTile);
                     const uint32_t a0 = a_ring + sa * kAStageCols;
@@ -406,21 +415,24 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             b_consumed_sh = ks;
             // drain: every MMA issued so far completes before TMEM is released
             mma_commit(final_bar);
-            wait_bar_drain(final_bar, 0);
+            wait_bar_drain(final_bar, 0, lim);
         }
         __syncwarp();
-    } else if (warp == 10) {
+    } else if (warp == kBWarp) {
         // ------------------------------------------------------------------ TMA producer of B
         if (lane == 0) {
             int ks = 0;
-            bool ok = true;
+            bool ok = !args.skip_b;
             for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
                 const Tile tl = decode_tile<GATED>(args, t, nr);
+                // the smallest box that holds the group's tokens (rows past them are not read)
+                const int nbox = tl.n <= 16 ? 16 : tl.n <= 32 ? 32 : tl.n <= 64 ? 64 : 128;
+                const CUtensorMap* mapB = nbox == 16 ? &tmB16 : nbox == 32 ? &tmB32 : nbox == 64 ? &tmB64 : &tmB128;
                 for (int kk = 0; kk < tl.ksteps; ++kk, ++ks) {
                     const int s = ks % kBStages;
-                    if (!(ok = wait_bar(bempty_bar(s), ((ks / kBStages) & 1) ^ 1, abortp, status))) break;
-                    mbar_expect_tx(bfull_bar(s), kBTile);
-                    tma_load_2d(sB + s * kBTile, &tmB, bfull_bar(s), kk * BK, tl.slot0);
+                    if (!(ok = wait_bar(bempty_bar(s), ((ks / kBStages) & 1) ^ 1, abortp, status, lim))) break;
+                    mbar_expect_tx(bfull_bar(s), (uint32_t)nbox * BK * 2u);
+                    tma_load_2d(sB + s * kBTile, mapB, bfull_bar(s), kk * BK, tl.slot0);
                 }
             }
             b_issued_sh = ks;
@@ -429,7 +441,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     } else {
         // ------------------------------------------------------------------ converters + epilogue
         const int q = warp & 3;                            // TMEM lane quarter of this warp
-        const int set = (warp - 2) / 4;                    // K steps with ks % 2 == set
+        const int set = (warp - 2) / 4;                    // K steps with ks % kConvSets == set
         const int r = 32 * q + lane;                       // tile row owned by this thread
         const uint32_t lane_off = (uint32_t)(32 * q) << 16;
         int ks = 0, tc = 0;
@@ -437,9 +449,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tc) {
             const Tile tl = decode_tile<GATED>(args, t, nr);
             for (int kk = 0; kk < tl.ksteps; ++kk, ++ks) {
-                if ((ks & 1) != set) continue;
+                if (ks % kConvSets != set) continue;
                 const int s = ks % kSA, sa = ks % kAStages;
-                ok = wait_bar(full_bar(s), (ks / kSA) & 1, abortp, status);
+                ok = wait_bar(full_bar(s), (ks / kSA) & 1, abortp, status, lim);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 // packed rows, 32-byte swizzle: the 16-byte halves of rows with bit 2 set are swapped
@@ -453,7 +465,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     const uint4 hi = lds_v4(rowp + 16u * (sw ^ 1));
                     const uint32_t words[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
                     if (a == 0) {
-                        ok = wait_bar(aempty_bar(sa), ((ks / kAStages) & 1) ^ 1, abortp, status);
+                        ok = wait_bar(aempty_bar(sa), ((ks / kAStages) & 1) ^ 1, abortp, status, lim);
                         ok = __all_sync(0xffffffffu, ok);
                         if (!ok) break;
                     }
@@ -472,14 +484,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             }
             if (!ok) break;
             // epilogue of this tile
-            ok = wait_bar(accfull_bar, tc & 1, abortp, status);
+            ok = wait_bar(accfull_bar, tc & 1, abortp, status, lim);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
             const int nmma = (tl.n + 15) & ~15;
             const float s0 = __ldg(tl.sc0 + r);
             const float s1 = GATED ? __ldg(tl.sc1 + r) : 0.0f;
-            for (int c0 = 16 * set; c0 < nmma; c0 += 32) {
+            for (int c0 = 16 * set; c0 < nmma; c0 += 16 * kConvSets) {
                 uint32_t v0[16], v1[16];
                 tmem_ld16(acc0 + c0 + lane_off, v0);
                 if (GATED) tmem_ld16(acc1 + c0 + lane_off, v1);
@@ -515,10 +527,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     // drain TMA copies that were issued but not consumed (only after an abort)
     if (warp == 0 && lane == 0) {
         int consumed = consumed_sh[0];
-        for (int i = 1; i < 8; ++i) consumed = min(consumed, consumed_sh[i]);
-        for (int k2 = consumed; k2 < issued_sh; ++k2) wait_bar_drain(full_bar(k2 % kSA), (k2 / kSA) & 1);
+        for (int i = 1; i < kConvWarps; ++i) consumed = min(consumed, consumed_sh[i]);
+        for (int k2 = consumed; k2 < issued_sh; ++k2) wait_bar_drain(full_bar(k2 % kSA), (k2 / kSA) & 1, lim);
         for (int k2 = b_consumed_sh; k2 < b_issued_sh; ++k2)
-            wait_bar_drain(bfull_bar(k2 % kBStages), (k2 / kBStages) & 1);
+            wait_bar_drain(bfull_bar(k2 % kBStages), (k2 / kBStages) & 1, lim);
     }
     tc_fence_before();
     __syncthreads();
@@ -530,12 +542,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 // gather: xg[slot] = x[token of slot] with K permuted within groups of 8 as [0,4,1,5,2,6,3,7]
 // ---------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
-gather_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, const double* __restrict__ xsum,
-              int T, int k, int S, int d, uint16_t* __restrict__ xg, float* __restrict__ xsum_slot) {
+gather_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, const int32_t* __restrict__ off,
+              const double* __restrict__ xsum, int T, int k, int S, int E, int d, uint16_t* __restrict__ xg,
+              float* __restrict__ xsum_slot) {
     const int per_row = d / 8;
     const size_t total = (size_t)T * (k + S) * per_row;
+    const int n_routed = off[E];          // routed slots in use (adaptive top-p may leave fewer than T k)
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
         const int slot = (int)(i / per_row), c = (int)(i % per_row);
+        if (slot < T * k && slot >= n_routed) continue;
         const int t = slot < T * k ? perm[slot] / k : slot - T * k;
         const uint4 v = ld_ro16(x + (size_t)t * d + 8 * c);
         uint4 o;
@@ -626,7 +641,8 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem
 
 // Tensor maps of one layer (weights and workspace never move, so they are built once).
 struct PrefillPlan {
-    CUtensorMap a1, a1_sh, b1, a2, a2_sh, b2;
+    CUtensorMap a1, a1_sh, a2, a2_sh;
+    CUtensorMap b1[4], b2[4];             // B boxes of 16, 32, 64 and 128 rows
     bool ok = false;
 };
 
@@ -654,8 +670,13 @@ PrefillPlan* prefill_plan_create(const LayerDims& L, const moe_weights& W, const
         p->a1_sh = p->a1;
         p->a2_sh = p->a2;
     }
-    ok &= make_map(&p->b1, ws.xg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L.d, slots, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok &= make_map(&p->b2, ws.h, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, fmax, slots, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t rows = 16u << i;
+        ok &= make_map(&p->b1[i], ws.xg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L.d, slots, BK, rows,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+        ok &= make_map(&p->b2[i], ws.h, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, fmax, slots, BK, rows,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    }
     p->ok = ok;
     if (!ok) {
         delete p;
@@ -691,15 +712,20 @@ cudaError_t launch_prefill_experts(const LayerDims& L, const PrefillPlan* p, con
     const size_t work = (size_t)T * (L.k + L.S) * (L.d / 8);
     const unsigned gg = (unsigned)std::min<size_t>((work + 255) / 256, (size_t)num_sms * 16);
     QE_LAUNCH(ctx, MOE_KERNEL_GATHER,
-              (gather_kernel<<<gg, 256, 0, ctx.s>>>(x, ws.perm, ws.xsum, T, L.k, L.S, L.d, ws.xg, ws.xsum_slot)));
+              (gather_kernel<<<gg, 256, 0, ctx.s>>>(x, ws.perm, ws.off, ws.xsum, T, L.k, L.S, L.E, L.d, ws.xg,
+                                                    ws.xsum_slot)));
     GemmArgs a1{groups, ws.n_groups, W.gate_up_scale, W.shared_gate_up_scale, 2 * L.f, L.f, L.S ? L.f_shared : L.f,
-                L.f / BM, L.S ? L.f_shared / BM : 1, L.d, L.d, fmax, ws.h, ws.status, ws.xsum_slot};
+                L.f / BM, L.S ? L.f_shared / BM : 1, L.d, L.d, fmax, ws.h, ws.status, ws.xsum_slot, L.wait_ns,
+                L.test_skip_b};
     QE_LAUNCH(ctx, MOE_KERNEL_GEMM_GATEUP,
-              (gemm_kernel<true><<<num_sms, kGemmThreads, gemm_smem_bytes(true), ctx.s>>>(p->a1, p->a1_sh, p->b1, a1)));
+              (gemm_kernel<true><<<num_sms, kGemmThreads, gemm_smem_bytes(true), ctx.s>>>(
+                  p->a1, p->a1_sh, p->b1[0], p->b1[1], p->b1[2], p->b1[3], a1)));
     GemmArgs a2{groups, ws.n_groups, W.down_scale, W.shared_down_scale, L.d, L.f, L.S ? L.f_shared : L.f,
-                L.d / BM, L.d / BM, L.f, L.S ? L.f_shared : L.f, L.d, ws.Y, ws.status, nullptr};
+                L.d / BM, L.d / BM, L.f, L.S ? L.f_shared : L.f, L.d, ws.Y, ws.status, nullptr, L.wait_ns,
+                L.test_skip_b};
     QE_LAUNCH(ctx, MOE_KERNEL_GEMM_DOWN,
-              (gemm_kernel<false><<<num_sms, kGemmThreads, gemm_smem_bytes(false), ctx.s>>>(p->a2, p->a2_sh, p->b2, a2)));
+              (gemm_kernel<false><<<num_sms, kGemmThreads, gemm_smem_bytes(false), ctx.s>>>(
+                  p->a2, p->a2_sh, p->b2[0], p->b2[1], p->b2[2], p->b2[3], a2)));
     return cudaSuccess;
 }
 

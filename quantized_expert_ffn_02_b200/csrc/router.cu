@@ -163,7 +163,8 @@ router_gemm_kernel(const float* __restrict__ wr, const uint16_t* __restrict__ x,
 template <int MAXPER>
 __global__ void __launch_bounds__(256)
 topk_kernel(const double* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k, int router,
-            float scaling, int32_t* __restrict__ idx_out, float* __restrict__ w_out, int32_t* __restrict__ asc_out) {
+            float scaling, int32_t* __restrict__ idx_out, float* __restrict__ w_out, int32_t* __restrict__ asc_out,
+            const RouterOpts opts) {
     const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
     const int t = blockIdx.x * (blockDim.x / kWarp) + warp;
     if (t >= T) return;
@@ -175,7 +176,7 @@ topk_kernel(const double* __restrict__ logits, const float* __restrict__ bias, i
     }
     float bv[MAXPER];
     load_bias<MAXPER>(bias, E, lane, bv);
-    const TopkPick p = warp_topk<MAXPER>(lg, bv, E, k, router, scaling, lane);
+    const TopkPick p = warp_topk<MAXPER>(lg, bv, E, k, router, scaling, lane, opts);
     if (lane < k) {
         idx_out[(size_t)t * k + lane] = p.e;
         w_out[(size_t)t * k + lane] = p.w;
@@ -195,7 +196,8 @@ constexpr int kSmallMaxE = 1024;
 // Selection for one token whose logits other blocks wrote (read through L2).
 template <int MAXPER>
 __device__ void warp_select(const double* __restrict__ lg, const float* __restrict__ bias, int E, int k, int router,
-                            float scaling, int lane, int32_t* idx_out, float* w_out, int32_t* asc_out) {
+                            float scaling, int lane, int32_t* idx_out, float* w_out, int32_t* asc_out,
+                            const RouterOpts& opts) {
     double l[MAXPER];
 #pragma unroll
     for (int m = 0; m < MAXPER; ++m) {
@@ -204,7 +206,7 @@ __device__ void warp_select(const double* __restrict__ lg, const float* __restri
     }
     float bv[MAXPER];
     load_bias<MAXPER>(bias, E, lane, bv);
-    const TopkPick p = warp_topk<MAXPER>(l, bv, E, k, router, scaling, lane);
+    const TopkPick p = warp_topk<MAXPER>(l, bv, E, k, router, scaling, lane, opts);
     if (lane < k) {
         idx_out[lane] = p.e;
         w_out[lane] = p.w;
@@ -219,7 +221,7 @@ route_small_kernel(const float* __restrict__ wr, const float* __restrict__ bias,
                    double* __restrict__ xsum, int32_t* __restrict__ idx, float* __restrict__ wts,
                    int32_t* __restrict__ asc, int32_t* __restrict__ cnt, int32_t* __restrict__ off,
                    int32_t* __restrict__ perm, int32_t* __restrict__ slot_of, int32_t* __restrict__ ulist,
-                   int32_t* __restrict__ n_unique, unsigned int* __restrict__ counter) {
+                   int32_t* __restrict__ n_unique, unsigned int* __restrict__ counter, const RouterOpts opts) {
     __shared__ double red[kSmallThreads / kWarp][kSmallMaxT];
     __shared__ double redx[kSmallThreads / kWarp];
     __shared__ int s_cnt[kSmallMaxE], s_off[kSmallMaxE], s_scan[kSmallThreads];
@@ -285,11 +287,12 @@ route_small_kernel(const float* __restrict__ wr, const float* __restrict__ bias,
     __threadfence();
     for (int t = warp; t < T; t += kSmallThreads / kWarp)
         warp_select<MAXPER>(logits + (size_t)t * E, bias, E, k, router, scaling, lane, idx + (size_t)t * k,
-                            wts + (size_t)t * k, asc + (size_t)t * k);
+                            wts + (size_t)t * k, asc + (size_t)t * k, opts);
     for (int i = tid; i < E; i += kSmallThreads) s_cnt[i] = 0;
     __syncthreads();
     __threadfence_block();
-    for (int i = tid; i < T * k; i += kSmallThreads) atomicAdd(&s_cnt[idx[i]], 1);
+    for (int i = tid; i < T * k; i += kSmallThreads)
+        if (idx[i] >= 0) atomicAdd(&s_cnt[idx[i]], 1);            // -1: dropped by adaptive top-p
     __syncthreads();
     // exclusive scan of the counts (each thread owns a run of experts) and of the used flags
     const int per = (E + kSmallThreads - 1) / kSmallThreads;
@@ -324,8 +327,11 @@ route_small_kernel(const float* __restrict__ wr, const float* __restrict__ bias,
         for (int t = 0; t < T; ++t) {
             if (lane < k) {
                 const int ex = idx[(size_t)t * k + lane];
-                const int p = s_off[ex]++;
-                perm[p] = t * k + lane;
+                int p = -1;                                // -1: dropped by adaptive top-p
+                if (ex >= 0) {
+                    p = s_off[ex]++;                       // a token's kept experts are distinct
+                    perm[p] = t * k + lane;
+                }
                 slot_of[(size_t)t * k + lane] = p;
             }
             __syncwarp();
@@ -345,17 +351,17 @@ cudaError_t launch_route_small(const LayerDims& L, const float* router_w, const 
         QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,
                   (route_small_kernel<1><<<L.E, kSmallThreads, 0, ctx.s>>>(
                       router_w, bias, x, T, L.d, L.E, L.k, L.router, L.scaling, ws.logits, ws.xsum, ws.idx, ws.wts,
-                      ws.asc, ws.cnt, ws.off, ws.perm, ws.slot_of, ws.ulist, ws.n_unique, counter)));
+                      ws.asc, ws.cnt, ws.off, ws.perm, ws.slot_of, ws.ulist, ws.n_unique, counter, L.ropts)));
     else if (L.E <= 256)
         QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,
                   (route_small_kernel<8><<<L.E, kSmallThreads, 0, ctx.s>>>(
                       router_w, bias, x, T, L.d, L.E, L.k, L.router, L.scaling, ws.logits, ws.xsum, ws.idx, ws.wts,
-                      ws.asc, ws.cnt, ws.off, ws.perm, ws.slot_of, ws.ulist, ws.n_unique, counter)));
+                      ws.asc, ws.cnt, ws.off, ws.perm, ws.slot_of, ws.ulist, ws.n_unique, counter, L.ropts)));
     else
         QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,
                   (route_small_kernel<32><<<L.E, kSmallThreads, 0, ctx.s>>>(
                       router_w, bias, x, T, L.d, L.E, L.k, L.router, L.scaling, ws.logits, ws.xsum, ws.idx, ws.wts,
-                      ws.asc, ws.cnt, ws.off, ws.perm, ws.slot_of, ws.ulist, ws.n_unique, counter)));
+                      ws.asc, ws.cnt, ws.off, ws.perm, ws.slot_of, ws.ulist, ws.n_unique, counter, L.ropts)));
     return cudaSuccess;
 }
 
@@ -388,13 +394,13 @@ cudaError_t launch_router(const LayerDims& L, const float* router_w, const float
     const float* bias = L.router == MOE_ROUTER_SIGMOID_BIAS ? router_bias : nullptr;
     if (L.E <= 32)
         QE_LAUNCH(ctx, MOE_KERNEL_TOPK, (topk_kernel<1><<<g, tpb * kWarp, 0, s>>>(logits, bias, T, L.E, L.k, L.router,
-                                                                                    L.scaling, idx, wts, asc)));
+                                                                                    L.scaling, idx, wts, asc, L.ropts)));
     else if (L.E <= 256)
         QE_LAUNCH(ctx, MOE_KERNEL_TOPK, (topk_kernel<8><<<g, tpb * kWarp, 0, s>>>(logits, bias, T, L.E, L.k, L.router,
-                                                                                    L.scaling, idx, wts, asc)));
+                                                                                    L.scaling, idx, wts, asc, L.ropts)));
     else
         QE_LAUNCH(ctx, MOE_KERNEL_TOPK, (topk_kernel<32><<<g, tpb * kWarp, 0, s>>>(logits, bias, T, L.E, L.k, L.router,
-                                                                                     L.scaling, idx, wts, asc)));
+                                                                                     L.scaling, idx, wts, asc, L.ropts)));
     return cudaSuccess;
 }
 
@@ -463,6 +469,7 @@ extern "C" moe_status moe_route_noalloc(const moe_config* cfg, const float* rout
     const size_t logits_bytes = ((size_t)T * cfg->n_experts * sizeof(double) + 255) & ~(size_t)255;
     const size_t need = logits_bytes + (size_t)T * sizeof(double);
     if (need > qe::kRouteScratchBytes) return MOE_ERR_UNSUPPORTED;
+    cudaGetLastError();   // an error left pending by an earlier, unrelated call is not this call's
     void* scratch = nullptr;
     moe_status st = qe::route_scratch_for_current_device(&scratch);
     if (st != MOE_OK) return st;

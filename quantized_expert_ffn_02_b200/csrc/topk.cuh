@@ -18,14 +18,15 @@ __device__ __forceinline__ bool topk_beats(double ka, int ia, double kb, int ib)
 }
 
 struct TopkPick {
-    int e;       // lane r < k: the rank-r expert
-    float w;     // its gate weight (fp64 arithmetic, rounded once)
-    int pos;     // its position among the k experts in ascending index order
+    int e;       // lane r < k: the rank-r expert (-1 if adaptive top-p dropped it)
+    float w;     // its gate weight (fp64 arithmetic, rounded once; 0 if dropped)
+    int pos;     // its position among the k entries in ascending (expert, rank) order
 };
 
 // Gate weights of the chosen experts and their positions in ascending index order.  Lane r < k
 // holds the rank-r expert e and its logit l (fp64 arithmetic, rounded once to fp32).
-__device__ __forceinline__ TopkPick topk_finish(int my_e, double my_l, int k, int router, float scaling, int lane) {
+__device__ __forceinline__ TopkPick topk_finish(int my_e, double my_l, int k, int router, float scaling, int lane,
+                                                double top_p = 0.0) {
     const bool mine = lane < k;
     double num, den;
     if (router == MOE_ROUTER_SIGMOID_BIAS) {
@@ -38,16 +39,80 @@ __device__ __forceinline__ TopkPick topk_finish(int my_e, double my_l, int k, in
         num = mine ? exp(my_l - m) : 0.0;
         den = warp_sum_d(num);
     }
+    double w = mine ? (double)scaling * num / den : 0.0;
+    if (top_p > 0.0 && top_p < 1.0) {
+        // the k weights' total and running share, in rank order (every lane walks the same sums)
+        double total = 0.0;
+        for (int r2 = 0; r2 < k; ++r2) total += __shfl_sync(0xffffffffu, w, r2);
+        double cum = 0.0;
+        int m = k;
+        for (int r2 = 0; r2 < k; ++r2) {
+            cum += __shfl_sync(0xffffffffu, w, r2);
+            if (m == k && cum / total >= top_p) m = r2 + 1;
+        }
+        double kept = 0.0;
+        for (int r2 = 0; r2 < m; ++r2) kept += __shfl_sync(0xffffffffu, w, r2);
+        if (lane < m) {
+            w = w * (total / kept);
+        } else if (mine) {
+            w = 0.0;
+            my_e = -1;
+        }
+    }
     int pos = 0;
     for (int r2 = 0; r2 < k; ++r2) {
         const int e2 = __shfl_sync(0xffffffffu, my_e, r2);
-        if (mine && e2 < my_e) ++pos;
+        if (mine && (e2 < my_e || (e2 == my_e && r2 < lane))) ++pos;
     }
     TopkPick p;
     p.e = mine ? my_e : -1;
-    p.w = mine ? (float)((double)scaling * num / den) : 0.0f;
+    p.w = mine ? (float)w : 0.0f;
     p.pos = pos;
     return p;
+}
+
+// Group-limited selection: marks (in `taken`) every expert outside the topk_group best groups.
+// key[m] is the key of expert lane + 32 m.  n_group <= 32 and E % n_group == 0.
+template <int MAXPER>
+__device__ __forceinline__ void limit_groups(const double (&key)[MAXPER], int E, const RouterOpts& o, int lane,
+                                             uint32_t& taken) {
+    const int G = o.n_group, per = E / G;
+    double my_score = -INFINITY;             // lane g: the score of group g
+    for (int g = 0; g < G; ++g) {
+        double b1 = -INFINITY, b2 = -INFINITY;   // the two largest keys of the group, b1 >= b2
+#pragma unroll
+        for (int m = 0; m < MAXPER; ++m) {
+            const int e = lane + kWarp * m;
+            if (e < E && e / per == g) {
+                if (key[m] > b1) { b2 = b1; b1 = key[m]; }
+                else if (key[m] > b2) b2 = key[m];
+            }
+        }
+#pragma unroll
+        for (int s = 16; s > 0; s >>= 1) {
+            const double o1 = __shfl_xor_sync(0xffffffffu, b1, s), o2 = __shfl_xor_sync(0xffffffffu, b2, s);
+            if (o1 > b1) { b2 = fmax(o2, b1); b1 = o1; }
+            else b2 = fmax(b2, o1);
+        }
+        if (lane == g) my_score = per >= 2 ? b1 + b2 : b1;
+    }
+    uint32_t keep = 0;
+    for (int r = 0; r < o.topk_group; ++r) {
+        double bs = (lane < G && !(keep >> lane & 1u)) ? my_score : -INFINITY;
+        int bg = (lane < G && !(keep >> lane & 1u)) ? lane : 0x7fffffff;
+#pragma unroll
+        for (int s = 16; s > 0; s >>= 1) {
+            const double os = __shfl_xor_sync(0xffffffffu, bs, s);
+            const int og = __shfl_xor_sync(0xffffffffu, bg, s);
+            if (os > bs || (os == bs && og < bg)) { bs = os; bg = og; }
+        }
+        keep |= 1u << bg;
+    }
+#pragma unroll
+    for (int m = 0; m < MAXPER; ++m) {
+        const int e = lane + kWarp * m;
+        if (e < E && !(keep >> (e / per) & 1u)) taken |= 1u << m;
+    }
 }
 
 // The selection key of one expert: the logit (softmax router) or sigmoid(logit) + bias; NaN
@@ -61,7 +126,8 @@ __device__ __forceinline__ double topk_key(double l, float bias, int router) {
 // with an index >= E are ignored.  Every lane of the warp calls it; lanes >= k get e = -1.
 template <int MAXPER>
 __device__ __forceinline__ TopkPick warp_topk(const double (&lg)[MAXPER], const float (&bv)[MAXPER], int E, int k,
-                                              int router, float scaling, int lane) {
+                                              int router, float scaling, int lane,
+                                              const RouterOpts& opts = RouterOpts()) {
     double key[MAXPER];
     uint32_t taken = 0;
 #pragma unroll
@@ -75,6 +141,7 @@ __device__ __forceinline__ TopkPick warp_topk(const double (&lg)[MAXPER], const 
         }
         key[m] = kv;
     }
+    if (opts.n_group > 1) limit_groups<MAXPER>(key, E, opts, lane, taken);
     int my_e = -1;
     double my_l = 0.0;
     for (int r = 0; r < k; ++r) {
@@ -101,7 +168,7 @@ __device__ __forceinline__ TopkPick warp_topk(const double (&lg)[MAXPER], const 
         wl = __shfl_sync(0xffffffffu, wl, owner);
         if (lane == r) { my_e = bi; my_l = wl; }
     }
-    return topk_finish(my_e, my_l, k, router, scaling, lane);
+    return topk_finish(my_e, my_l, k, router, scaling, lane, opts.top_p);
 }
 
 // The biases of experts lane + 32 m (0 where there is none).

@@ -40,17 +40,41 @@ def _fp32_dev(cfg, e, which, seed, host: bool, dev):
 
 
 def build_gpu_layer(cfg: syn.LayerConfig, seed: int = 0, host_experts: Optional[Iterable[int]] = None,
-                    max_tokens: Optional[int] = None, out_bf16: Optional[bool] = None, device="cuda"):
-    """Returns (MoELayer, weights dict of device tensors).  host_experts=None draws every expert on the host."""
+                    max_tokens: Optional[int] = None, out_bf16: Optional[bool] = None, device="cuda",
+                    oracle_experts: Optional[dict] = None):
+    """Returns (MoELayer, weights dict of device tensors).  host_experts=None draws every expert on the host.
+
+    oracle_experts: if a dict is given, every host-drawn expert is also stored there in the
+    oracle's storage format (packed on the host by the oracle's packer, or bf16 bits), keyed by
+    expert id or "shared", so a full-size expert is drawn once for both sides."""
     dev = torch.device(device)
     E, d, f = cfg.E, cfg.d, cfg.f
-    int4 = cfg.wkind == syn.W_INT4
+    int4 = cfg.wkind != syn.W_BF16          # a packed container with per-row scales (int4, int8, int2)
     hset = None if host_experts is None else set(int(e) for e in host_experts)
     W = {}
+    # bytes per row of n columns, storage dtype, the GPU packer and the oracle's packer per kind
+    per = {syn.W_INT4: (2, torch.uint8), syn.W_INT8: (1, torch.int8), syn.W_INT2: (4, torch.uint8)}
+
+    def cols(n):
+        return n // per[cfg.wkind][0]
+
+    def gpu_pack(w, dst, dst_s):
+        {syn.W_INT4: qe.moe_pack_int4, syn.W_INT8: qe.moe_pack_int8, syn.W_INT2: qe.moe_pack_int2}[cfg.wkind](
+            w, dst, dst_s)
+
+    def oracle_pack(w):
+        import oracle
+        if cfg.wkind == syn.W_INT8:
+            return oracle.quantize_tier(w, 8)
+        if cfg.wkind == syn.W_INT2:
+            return oracle.pack_int2(w)
+        return oracle.pack_int4(w)
+
     if int4:
-        W["gate_up"] = torch.empty((E, 2 * f, d // 2), dtype=torch.uint8, device=dev)
+        dt = per[cfg.wkind][1]
+        W["gate_up"] = torch.empty((E, 2 * f, cols(d)), dtype=dt, device=dev)
         W["gate_up_scale"] = torch.empty((E, 2 * f), dtype=torch.float32, device=dev)
-        W["down"] = torch.empty((E, d, f // 2), dtype=torch.uint8, device=dev)
+        W["down"] = torch.empty((E, d, cols(f)), dtype=dt, device=dev)
         W["down_scale"] = torch.empty((E, d), dtype=torch.float32, device=dev)
     else:
         W["gate_up"] = torch.empty((E, 2 * f, d), dtype=torch.int16, device=dev)
@@ -59,11 +83,21 @@ def build_gpu_layer(cfg: syn.LayerConfig, seed: int = 0, host_experts: Optional[
     def put(e, which, dst, dst_s):
         host = hset is None or e == "shared" or e in hset
         if not int4 and host:
-            dst.copy_(torch.from_numpy(syn.gen_expert_bf16(cfg, e, which, seed).view(np.int16)).to(dev))
+            bits = syn.gen_expert_bf16(cfg, e, which, seed)
+            if oracle_experts is not None:
+                oracle_experts.setdefault(e, {})[which] = bits
+            dst.copy_(torch.from_numpy(bits.view(np.int16)).to(dev))
             return
-        w = _fp32_dev(cfg, e, which, seed, host, dev)
+        if host and oracle_experts is not None:
+            w_host = syn.gen_expert_fp32(cfg, e, which, seed)
+            rec = oracle_experts.setdefault(e, {})
+            rec[which], rec[which + "_scale"] = oracle_pack(w_host)
+            w = torch.from_numpy(w_host).to(dev)
+            del w_host
+        else:
+            w = _fp32_dev(cfg, e, which, seed, host, dev)
         if int4:
-            qe.moe_pack_int4(w, dst, dst_s)
+            gpu_pack(w, dst, dst_s)
         else:
             dst.copy_(w.to(torch.bfloat16).view(torch.int16))
 
@@ -73,9 +107,10 @@ def build_gpu_layer(cfg: syn.LayerConfig, seed: int = 0, host_experts: Optional[
     if cfg.n_shared:
         fs = cfg.f_shared
         if int4:
-            W["shared_gate_up"] = torch.empty((2 * fs, d // 2), dtype=torch.uint8, device=dev)
+            dt = per[cfg.wkind][1]
+            W["shared_gate_up"] = torch.empty((2 * fs, cols(d)), dtype=dt, device=dev)
             W["shared_gate_up_scale"] = torch.empty((2 * fs,), dtype=torch.float32, device=dev)
-            W["shared_down"] = torch.empty((d, fs // 2), dtype=torch.uint8, device=dev)
+            W["shared_down"] = torch.empty((d, cols(fs)), dtype=dt, device=dev)
             W["shared_down_scale"] = torch.empty((d,), dtype=torch.float32, device=dev)
         else:
             W["shared_gate_up"] = torch.empty((2 * fs, d), dtype=torch.int16, device=dev)

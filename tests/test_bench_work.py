@@ -100,3 +100,14 @@ def test_traffic_is_reported_only_for_unchanged_sources():
 def test_traffic_is_null_once_a_source_changes(monkeypatch):
     monkeypatch.setattr(bench, "source_sha", lambda paths: "0" * 16)
     assert bench.traffic_for("fused") is None
+
+
+def test_every_workload_is_measured_once_with_the_headline_first():
+    import argparse
+    a = argparse.Namespace(workload="glm_decode", workloads="all")
+    names = bench.selected_workloads(a)
+    assert names[0] == "glm_decode" and sorted(names) == sorted(bench.WORKLOADS)
+    a = argparse.Namespace(workload="granite", workloads="none")
+    assert bench.selected_workloads(a) == ["granite"]
+    a = argparse.Namespace(workload="tiny", workloads="glm_prefill,tiny")
+    assert bench.selected_workloads(a) == ["tiny", "glm_prefill"]

@@ -14,7 +14,7 @@ import oracle
 import quantized_expert_ffn_02_b200 as qe
 import synthetic as syn
 from gpu_layers import build_gpu_layer, check_close, run_forward, run_route, x_dev
-from layers import oracle_layer, router_only, small_config
+from layers import oracle_layer, oracle_layer_from, router_only, small_config
 
 pytestmark = pytest.mark.gpu
 
@@ -84,30 +84,53 @@ def test_pack_nonfinite_reports_range():
 GLM = syn.CONFIGS["glm_decode"]
 DECODE_TOKENS = [0, 1]                     # T = 1 calls on tokens 0 and 1 of stream x
 UNION2_OFFSET = 100                        # T = 2: tokens 100, 101
-UNION32_OFFSET = 200                       # T = 32: tokens 200 .. 231; oracle on two of them
-UNION32_SAMPLE = [0, 31]
-PREFILL_OFFSET = 1000                      # T = 2048: tokens 1000 .. 3047; oracle on two of them
-PREFILL_SAMPLE = [0, 2047]
+UNION32_OFFSET = 200                       # T = 32: tokens 200 .. 231, every one compared
+PREFILL_OFFSET = 1000                      # T = 2048: tokens 1000 .. 3047, a sample compared
 
 
 def _glm_x(T, offset):
     return syn.gen_x(GLM, 0, T=T, token_offset=offset)
 
 
+def prefill_sample(idx: np.ndarray, group: int = 128) -> list:
+    """Tokens of the 2048-token batch that the oracle checks.
+
+    * Two tokens of every 128-token block of the batch: the shared expert runs over the whole
+      batch in blocks of 128 tokens (one GEMM column block each), so every block is checked.
+    * The largest routed bucket: its first and last token and the first token of each further
+      128-token block of that bucket (the routed GEMMs also split a bucket into blocks of 128).
+    * Every token of the smallest non-empty routed bucket.
+    """
+    T = idx.shape[0]
+    pick = set()
+    for b in range(0, T, group):
+        pick.add(b + 3)
+        pick.add(min(T - 1, b + group - 5))
+    cnt = np.bincount(idx.reshape(-1), minlength=GLM.E)
+    big = int(np.argmax(cnt))
+    toks = np.nonzero((idx == big).any(axis=1))[0]
+    pick.update(int(t) for t in toks[::group])
+    pick.add(int(toks[-1]))
+    small = int(np.argmin(np.where(cnt > 0, cnt, np.iinfo(np.int64).max)))
+    pick.update(int(t) for t in np.nonzero((idx == small).any(axis=1))[0])
+    return sorted(pick)
+
+
 @pytest.fixture(scope="module")
 def glm():
     router = router_only(GLM)
-    sample_rows = [_glm_x(1, t) for t in DECODE_TOKENS] + [_glm_x(2, UNION2_OFFSET)]
     x32 = _glm_x(32, UNION32_OFFSET)
-    sample_rows.append(x32[UNION32_SAMPLE])
     xp = _glm_x(2048, PREFILL_OFFSET)
-    sample_rows.append(xp[PREFILL_SAMPLE])
+    psample = prefill_sample(router.route(xp)["idx"])
+    sample_rows = [_glm_x(1, t) for t in DECODE_TOKENS] + [_glm_x(2, UNION2_OFFSET), x32, xp[psample]]
     touched = set()
     for xr in sample_rows:
         touched |= set(router.route(xr)["idx"].reshape(-1).tolist())
-    layer, W = build_gpu_layer(GLM, host_experts=touched, max_tokens=2048)
-    ora = oracle_layer(GLM, experts=touched)
-    yield {"layer": layer, "W": W, "oracle": ora, "router": router, "x32": x32, "xp": xp}
+    drawn = {}
+    layer, W = build_gpu_layer(GLM, host_experts=touched, max_tokens=2048, oracle_experts=drawn)
+    ora = oracle_layer_from(GLM, drawn)
+    yield {"layer": layer, "W": W, "oracle": ora, "router": router, "x32": x32, "xp": xp,
+           "psample": psample, "touched": touched}
     layer.close()
 
 
@@ -136,19 +159,33 @@ def test_glm_union_t2(glm):
     check_close(run_forward(glm["layer"], x), ref["out"])
 
 
-def test_glm_union_t32_sampled(glm):
+def test_glm_union_t32_every_token(glm):
     out = run_forward(glm["layer"], glm["x32"])
-    ref = glm["oracle"].forward(glm["x32"][UNION32_SAMPLE])
-    check_close(out[UNION32_SAMPLE], ref["out"])
+    ref = glm["oracle"].forward(glm["x32"])
+    check_close(out, ref["out"])
+    for t in range(32):                   # and token by token
+        check_close(out[t:t + 1], ref["out"][t:t + 1])
+
+
+def test_glm_prefill_sample_covers_every_block(glm):
+    ps = glm["psample"]
+    blocks = {t // 128 for t in ps}
+    assert blocks == set(range(16)), "every 128-token block of the batch is sampled"
+    assert len(ps) >= 32
 
 
 def test_glm_prefill_t2048_sampled_and_properties(glm):
-    out = run_forward(glm["layer"], glm["xp"])
-    ref = glm["oracle"].forward(glm["xp"][PREFILL_SAMPLE])
-    check_close(out[PREFILL_SAMPLE], ref["out"])
+    layer = glm["layer"]
+    assert layer.has_gemm_path
+    out = run_forward(layer, glm["xp"])
+    ps = glm["psample"]
+    ref = glm["oracle"].forward(glm["xp"][ps])
+    check_close(out[ps], ref["out"])
+    worst = max(np.linalg.norm(out[t] - ref["out"][i]) / np.linalg.norm(ref["out"][i]) for i, t in enumerate(ps))
+    assert worst <= 2e-3, worst
     # properties at full size: finite, deterministic run to run
     assert np.isfinite(out).all()
-    out2 = run_forward(glm["layer"], glm["xp"])
+    out2 = run_forward(layer, glm["xp"])
     assert np.array_equal(out, out2)
 
 

@@ -30,7 +30,7 @@ def _router_layer(cfg, seed=0):
     W["gate_up_scale"] = torch.zeros((cfg.E, 2 * cfg.f), dtype=torch.float32, device=dev)
     W["down"] = torch.zeros((cfg.E, cfg.d, cfg.f // 2), dtype=torch.uint8, device=dev)
     W["down_scale"] = torch.zeros((cfg.E, cfg.d), dtype=torch.float32, device=dev)
-    layer = qe.MoELayer(cfg.d, cfg.f, cfg.E, cfg.k, 64, cfg.router, syn.W_INT4, W, routed_scaling_factor=cfg.scaling)
+    layer = qe.MoELayer(cfg.d, cfg.f, cfg.E, cfg.k, 512, cfg.router, syn.W_INT4, W, routed_scaling_factor=cfg.scaling)
     return layer, W
 
 
@@ -57,6 +57,19 @@ def test_noalloc_route_matches_moe_route_on_consecutive_calls(name):
     for T, offset in ((32, 0), (5, 777)):
         ia, wa, ib, wb = _both(layer, W, cfg, syn.gen_x(cfg, 0, T=T, token_offset=offset))
         assert np.array_equal(ia, ib)
+        np.testing.assert_allclose(wb, wa, rtol=1e-6)
+    layer.close()
+
+
+def test_noalloc_route_long_batches_match_moe_route():
+    # T >= 64 with E = 256 takes the tiled fp64 router GEMM, whose logits and sums of x land in
+    # the static array at its 256-byte aligned offsets; T = 200 is not a multiple of the 64-token
+    # tile and T = 510 is the largest batch the array holds
+    cfg = syn.LayerConfig(**{**syn.CONFIGS["glm_decode"].__dict__, "f": 64})
+    layer, W = _router_layer(cfg)
+    for T, offset in ((64, 40), (200, 1234), (510, 9), (64, 40)):
+        ia, wa, ib, wb = _both(layer, W, cfg, syn.gen_x(cfg, 0, T=T, token_offset=offset))
+        assert np.array_equal(ia, ib), T
         np.testing.assert_allclose(wb, wa, rtol=1e-6)
     layer.close()
 
