@@ -3,15 +3,20 @@
 // For one token the layer reads each weight byte once, so its time is the time to stream the
 // router matrix and k + 1 experts from HBM.  Separate kernels for the router, gate/up and down
 // each pay the ramp of a fresh grid and leave HBM idle while the previous grid drains; here one
-// persistent CTA per SM (8 warps) runs the steps back to back and keeps its copies in flight
-// across the joins.  Each warp streams its weight rows through a private ring of TMA bulk copies
-// (a gate row, the matching up row and two 16-byte slivers holding their scales per stage).
+// persistent CTA per SM runs the steps back to back and keeps its copies in flight
+// across the joins.  Each warp streams its weight rows through a private two-stage ring of TMA
+// bulk copies (a gate row, the matching up row and two 16-byte slivers holding their scales per
+// stage).  Up to 16 warps per CTA: as many as the rings fit in shared memory beside x.
 //
-//   A  router + shared expert.  The warps queue their shared-expert row pairs (they need no
-//      routing) at once; one bulk copy brings x in while each warp's first router piece (one
-//      expert x 1024 columns, coalesced loads) is in flight.  The warps compute their router
-//      pieces in fp64 and store them, turn x into their fp16 operand registers (below), and the
-//      CTA arrives on grid barrier 0; the warps reduce their shared rows while the others arrive.
+// Shared memory: x as the MMA operand (x~ below), one block per lane holding the lane's groups in
+// the order it visits them, then the rings.  Phase A parks the plain bf16 x in the rings' last
+// stage; phase B keeps the router pieces, keys and logits at the start of the idle rings.
+//
+//   A  router + shared expert.  One bulk copy brings x in while each warp's first router piece
+//      (one expert x 1024 columns, coalesced loads) is in flight.  The CTA builds x~ from x, the
+//      warps compute their router pieces in fp64 and store them, the CTA arrives on grid
+//      barrier 0, and the warps reduce the shared expert's row pairs (they need no routing) while
+//      the other CTAs arrive.
 //   B  selection, by the whole CTA: one bulk copy gathers every piece; thread e sums expert e's
 //      pieces (the same order in every CTA, so every CTA selects the same experts) and forms an
 //      order-preserving integer key; the k best of each warp's 32 experts become candidates, and
@@ -66,9 +71,9 @@ namespace {
 
 using namespace dec;
 
-constexpr int kFzWarps = 8;
-constexpr int kFzThreads = kFzWarps * kWarp;
-constexpr int kFzMaxStages = 4;
+constexpr int kFzMaxWarps = 16;
+constexpr int kFzMaxThreads = kFzMaxWarps * kWarp;
+constexpr int kFzStages = 2;
 constexpr int kFzMaxSlots = 10;       // k routed experts + the shared one
 constexpr int kFzMaxPer = 8;          // experts per lane in the selection: E <= 256
 constexpr int kFzRowsMax = 64;        // output rows per CTA
@@ -200,7 +205,7 @@ __device__ __forceinline__ int gu_rot(int lane) {
 }
 template <int NF>
 __device__ __forceinline__ int dn_rot(int lane) {
-    return NF == 2 ? ((lane >> 2) & 1) : 0;
+    return gu_rot<NF>(lane);      // a down row's lane quarter has the same geometry
 }
 
 // 8 bf16 (or fp16) values of one 8-column group, as the four operand pairs of that group:
@@ -245,76 +250,156 @@ __device__ __forceinline__ int scale_exp(float vmax) {
     return max(-100, min(100, 14 - e));
 }
 
-// Diagonal of the two 8 x 8 blocks held by the warp's D fragments (four accumulator chains):
-// this lane's part of (rows 0..7 . columns) and (rows 8..15 . columns); 0 for lanes that hold no
+// Independent accumulator chains per dot product: an MMA's result feeds the next MMA of its chain
+// only, so a chain's latency is paid every kChains MMAs.
+constexpr int kChains = 4;
+
+// The weight kinds of this kernel.  A "group" is the 16 bytes of a weight row that a lane loads at
+// once: 32 int4 codes (8 K steps of the MMA for a row pair) or 8 bf16 values (2 K steps).  XR is the
+// number of 32-bit operand registers of x (or h) that one group meets.
+template <int WK> struct FzKind;
+template <> struct FzKind<MOE_W_INT4_ROWSCALE> {
+    static constexpr int COLS = 32, XR = 16, HR = 16;
+    static constexpr int row_bytes(int cols) { return cols / 2; }
+};
+template <> struct FzKind<MOE_W_BF16> {
+    static constexpr int COLS = 8, XR = 4, HR = 8;     // h: 4 registers of bf16 high parts, 4 of low parts
+    static constexpr int row_bytes(int cols) { return cols * 2; }
+};
+
+// Diagonal of the two 8 x 8 blocks held by the warp's D fragments (the chains added up): this
+// lane's part of (rows 0..7 . columns) and (rows 8..15 . columns); 0 for lanes that hold no
 // diagonal entry.
-__device__ __forceinline__ float2 diag_part(const float (&acc)[4][4], int lane) {
+__device__ __forceinline__ float2 diag_part(const float (&acc)[kChains][4], int lane) {
     const int g = lane >> 2, c = lane & 3;
     if (c != (g >> 1)) return make_float2(0.0f, 0.0f);
-    const float e0 = (acc[0][0] + acc[1][0]) + (acc[2][0] + acc[3][0]);
-    const float e1 = (acc[0][1] + acc[1][1]) + (acc[2][1] + acc[3][1]);
-    const float e2 = (acc[0][2] + acc[1][2]) + (acc[2][2] + acc[3][2]);
-    const float e3 = (acc[0][3] + acc[1][3]) + (acc[2][3] + acc[3][3]);
-    return (g & 1) ? make_float2(e1, e3) : make_float2(e0, e2);
-}
-
-// Gate row . x and up row . x for the row pair of stage st (2^24 times the sums of (s + 8) x~;
-// this lane's part, see diag_part).  xr holds this lane's x~ pairs, group by group in its visiting
-// order; lane_off is the byte offset of its segment quarter within a row.
-template <int NDK>
-__device__ __forceinline__ float2 gu_mma(uint32_t st, uint32_t gu_row, uint32_t lane_off, int rot,
-                                         const uint32_t (&xr)[NDK][16], int lane) {
-    float acc[4][4] = {};          // four independent accumulator chains (one per word of a group)
+    float e[4];
 #pragma unroll
-    for (int j = 0; j < NDK; ++j) {
-        int q = j + rot;
-        if (q >= NDK) q -= NDK;
-        const uint32_t off = lane_off + 16u * (uint32_t)q;
-        const uint4 G = lds16(st + off), U = lds16(st + gu_row + off);
-        const uint32_t gw[4] = {G.x, G.y, G.z, G.w}, uw[4] = {U.x, U.y, U.z, U.w};
+    for (int i = 0; i < 4; ++i) {
+        float t = 0.0f;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            mma16816(acc[w], nib_lo(gw[w]), nib_lo(uw[w]), nib_hi(gw[w]), nib_hi(uw[w]), xr[j][4 * w],
-                     xr[j][4 * w + 1]);
-            const uint32_t g8 = gw[w] >> 8, u8 = uw[w] >> 8;
-            mma16816(acc[w], nib_lo(g8), nib_lo(u8), nib_hi(g8), nib_hi(u8), xr[j][4 * w + 2], xr[j][4 * w + 3]);
-        }
+        for (int ch = 0; ch < kChains; ++ch) t += acc[ch][i];
+        e[i] = t;
     }
-    return diag_part(acc, lane);
+    return (g & 1) ? make_float2(e[1], e[3]) : make_float2(e[0], e[2]);
 }
 
-// Down rows A and B (shared addresses) . h~ of their slot: this lane's parts of 2^24 times the
-// sums of (s + 8) h~ (see diag_part); B may equal A.
-template <int NF>
-__device__ __forceinline__ float2 dn_mma(uint32_t rowA, uint32_t rowB, uint32_t lane_off, int rot,
-                                         const uint32_t (&hr)[NF][16], int lane) {
-    float acc[4][4] = {};
+// The same tile with bf16 operands (the bf16 weight kind).
+__device__ __forceinline__ void mma16816_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two rows (A rows 0..7: the first row's 8 K-segments, rows 8..15: the second row's) times the
+// lane's operand registers xr: this lane's part of both dot products (see diag_part).  G groups
+// per lane, visited from the lane's rotation; lane_off is the byte offset of its segment quarter.
+//   int4: 2^24 times the sums of (s + 8) x~ (codes decoded in place, see nib_lo / nib_hi);
+//   bf16: the sums of w x (the weights are the MMA operand as they are).
+// For the down rows the operand holds h~ (int4) or h split into bf16 high and low parts (bf16,
+// two MMAs per K step).
+template <int WK, int G, int XR, bool SPLIT>
+__device__ __forceinline__ float2 rows_mma(uint32_t rowA, uint32_t rowB, uint32_t lane_off, int rot,
+                                           const uint32_t (&xr)[G][XR], int lane) {
+    float acc[kChains][4] = {};
+    int chain = 0;
 #pragma unroll
-    for (int j = 0; j < NF; ++j) {
+    for (int j = 0; j < G; ++j) {
         int q = j + rot;
-        if (q >= NF) q -= NF;
+        if (q >= G) q -= G;
         const uint32_t off = lane_off + 16u * (uint32_t)q;
         const uint4 A = lds16(rowA + off), B = lds16(rowB + off);
         const uint32_t aw[4] = {A.x, A.y, A.z, A.w}, bw[4] = {B.x, B.y, B.z, B.w};
+        if (WK == MOE_W_INT4_ROWSCALE) {
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            mma16816(acc[w], nib_lo(aw[w]), nib_lo(bw[w]), nib_hi(aw[w]), nib_hi(bw[w]), hr[j][4 * w],
-                     hr[j][4 * w + 1]);
-            const uint32_t a8 = aw[w] >> 8, b8 = bw[w] >> 8;
-            mma16816(acc[w], nib_lo(a8), nib_lo(b8), nib_hi(a8), nib_hi(b8), hr[j][4 * w + 2], hr[j][4 * w + 3]);
+            for (int w = 0; w < 4; ++w) {
+                mma16816(acc[chain++ % kChains], nib_lo(aw[w]), nib_lo(bw[w]), nib_hi(aw[w]), nib_hi(bw[w]),
+                         xr[j][4 * w], xr[j][4 * w + 1]);
+                const uint32_t a8 = aw[w] >> 8, b8 = bw[w] >> 8;
+                mma16816(acc[chain++ % kChains], nib_lo(a8), nib_lo(b8), nib_hi(a8), nib_hi(b8), xr[j][4 * w + 2],
+                         xr[j][4 * w + 3]);
+            }
+        } else {
+            // K step s: columns 4s .. 4s+3 of the group; k-slots (2c, 2c+1) take the first pair
+#pragma unroll
+            for (int st = 0; st < 2; ++st) {
+                mma16816_bf16(acc[chain++ % kChains], aw[2 * st], bw[2 * st], aw[2 * st + 1], bw[2 * st + 1],
+                              xr[j][2 * st], xr[j][2 * st + 1]);
+                if (SPLIT)
+                    mma16816_bf16(acc[chain++ % kChains], aw[2 * st], bw[2 * st], aw[2 * st + 1], bw[2 * st + 1],
+                                  xr[j][4 + 2 * st], xr[j][4 + 2 * st + 1]);
+            }
         }
     }
     return diag_part(acc, lane);
 }
 
-// NDK = d / 1024, NF = f / 1024.
-template <int NDK, int NF>
-__global__ void __launch_bounds__(kFzThreads, 1) decode_fused_kernel(const FusedArgs a) {
-    // [kFzMaxStages][warps][stage]: stage s of every warp is one region; x (plain bf16, 2d bytes)
-    // lands in the last stage's region during phase A
+// The same two-row product with the operand of x read from this lane's block in shared memory
+// (xblk), one 16-byte group at a time: the loop over the groups stays rolled, so the code stays
+// small and the operand takes no long-lived registers.
+template <int WK, int G>
+__device__ __forceinline__ float2 rows_mma_x(uint32_t rowA, uint32_t rowB, uint32_t lane_off, int rot, uint32_t xblk,
+                                             int lane) {
+    float acc[kChains][4] = {};
+    int q = rot;
+#pragma unroll 1
+    for (int j = 0; j < G; ++j) {
+        const uint32_t off = lane_off + 16u * (uint32_t)q;
+        if (++q == G) q = 0;
+        const uint4 A = lds16(rowA + off), B = lds16(rowB + off);
+        const uint32_t aw[4] = {A.x, A.y, A.z, A.w}, bw[4] = {B.x, B.y, B.z, B.w};
+        if (WK == MOE_W_INT4_ROWSCALE) {
+            uint32_t xv[16];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const uint4 v = lds16(xblk + (uint32_t)(64 * j + 16 * m));
+                xv[4 * m] = v.x;
+                xv[4 * m + 1] = v.y;
+                xv[4 * m + 2] = v.z;
+                xv[4 * m + 3] = v.w;
+            }
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                mma16816(acc[w], nib_lo(aw[w]), nib_lo(bw[w]), nib_hi(aw[w]), nib_hi(bw[w]), xv[4 * w], xv[4 * w + 1]);
+                const uint32_t a8 = aw[w] >> 8, b8 = bw[w] >> 8;
+                mma16816(acc[w], nib_lo(a8), nib_lo(b8), nib_hi(a8), nib_hi(b8), xv[4 * w + 2], xv[4 * w + 3]);
+            }
+        } else {
+            const uint4 v = lds16(xblk + (uint32_t)(16 * j));
+            mma16816_bf16(acc[0], aw[0], bw[0], aw[1], bw[1], v.x, v.y);
+            mma16816_bf16(acc[1], aw[2], bw[2], aw[3], bw[3], v.z, v.w);
+        }
+    }
+    return diag_part(acc, lane);
+}
+
+// 8 fp16 values of h as bf16 high and low parts, h = high + low exactly (an fp16 value has 11
+// significant bits, a bf16 8, and the remainder fits in another bf16): registers 0..3 the high
+// parts of the pairs (0, 1) .. (6, 7), 4..7 the low parts.  sum: the values, in fp32.
+__device__ __forceinline__ void hilo_from_f16(uint4 v, uint32_t* p, float& sum) {
+    const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[i]));
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(f.x, f.y);
+        const float2 fh = __bfloat1622float2(hi);
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(f.x - fh.x, f.y - fh.y);
+        p[i] = *reinterpret_cast<const uint32_t*>(&hi);
+        p[4 + i] = *reinterpret_cast<const uint32_t*>(&lo);
+        sum += f.x + f.y;
+    }
+}
+
+// WK: MOE_W_INT4_ROWSCALE or MOE_W_BF16.  NDK: 16-byte groups of a gate/up row per lane (d / 1024
+// for int4, d / 256 for bf16); NF: the same for a down row (f / 1024, f / 256).
+template <int WK, int NDK, int NF>
+__global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const FusedArgs a) {
+    // [x~ lane blocks][kFzStages][warps][stage]: stage s of every warp is one region; x (plain
+    // bf16, 2d bytes) lands in the last stage's region during phase A
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ __align__(8) uint64_t bars[kFzWarps][kFzMaxStages];
-    __shared__ int4 s_desc[kFzWarps][kFzMaxStages];       // gate/up stage: slot, row, scale slots
+    __shared__ __align__(8) uint64_t bars[kFzMaxWarps][kFzStages];
+    __shared__ int4 s_desc[kFzMaxWarps][kFzStages];       // gate/up stage: slot, row, scale slots
     __shared__ __align__(8) uint64_t s_xbar;              // x -> shared memory
     __shared__ __align__(8) uint64_t s_rbar;              // the router pieces -> shared memory
     __shared__ float ys[kFzMaxSlots][kFzRowsMax];
@@ -331,19 +416,27 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode_fused_kernel(const Fused
     __shared__ unsigned long long s_base;                 // arrivals before this launch
     __shared__ int s_ok;
 
-    constexpr int d = 1024 * NDK, f = 1024 * NF;
+    constexpr bool BF = WK == MOE_W_BF16;
+    constexpr int d = 32 * NDK * FzKind<WK>::COLS, f = 32 * NF * FzKind<WK>::COLS;
+    constexpr int XR = FzKind<WK>::XR, HR = FzKind<WK>::HR;
     const int tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
+    const int nwc = blockDim.x / kWarp;                    // warps of this CTA
     const int G = gridDim.x;
-    const int gw = warp * G + blockIdx.x, nw = G * kFzWarps;   // warp-major: low numbers on every SM
+    const int gw = warp * G + blockIdx.x, nw = G * nwc;    // warp-major: low numbers on every SM
     const int k = a.k, E = a.E;
-    constexpr int nst = NDK <= 6 ? kFzMaxStages : kFzMaxStages - 1;   // ring stages per warp
-    constexpr int nch = NDK;                               // 1024-column router pieces per expert
-    constexpr uint32_t gu_row = d / 2, dn_row_b = f / 2;
+    constexpr uint32_t gu_row = FzKind<WK>::row_bytes(d), dn_row_b = FzKind<WK>::row_bytes(f);
+    constexpr int nst = kFzStages;                         // ring stages per warp
+    constexpr int nch = d / 1024;                          // 1024-column router pieces per expert
     constexpr uint32_t stage_bytes = 2 * gu_row + 32;
-    const uint32_t rings_s = saddr(smem);
-    auto st_s = [&](int s) { return rings_s + ((uint32_t)s * kFzWarps + warp) * stage_bytes; };
-    auto st_g = [&](int s) { return smem + ((size_t)s * kFzWarps + warp) * stage_bytes; };
-    const uint32_t xraw_s = rings_s + (uint32_t)(nst - 1) * kFzWarps * stage_bytes;
+    // x~ lane blocks: lane L's groups in its visiting order, padded by 16 bytes so that the lanes'
+    // 16-byte loads meet no bank conflict
+    constexpr uint32_t kLaneBlk = (BF ? 16 : 64) * NDK + 16;
+    constexpr uint32_t kXtBytes = (32 * kLaneBlk + 127) / 128 * 128;
+    const uint32_t xt_s = saddr(smem);
+    const uint32_t rings_s = xt_s + kXtBytes;
+    auto st_s = [&](int s) { return rings_s + ((uint32_t)s * nwc + warp) * stage_bytes; };
+    auto st_g = [&](int s) { return smem + kXtBytes + ((size_t)s * nwc + warp) * stage_bytes; };
+    const uint32_t xraw_s = rings_s + (uint32_t)(nst - 1) * nwc * stage_bytes;
     const int n_sh = a.S ? f : 0;                          // shared row pairs
     const int n_tasks = n_sh + k * f;
     auto count_of = [&](int lo, int hi) {                  // my tasks among [lo, hi)
@@ -357,11 +450,11 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode_fused_kernel(const Fused
     const int j0 = (int)((int64_t)blockIdx.x * d / G), rj = (int)((int64_t)(blockIdx.x + 1) * d / G) - j0;
     const int nslots = k + a.S;
     const int n_items = nslots * rj;
-    const int it0 = (int)((int64_t)warp * n_items / kFzWarps), it1 = (int)((int64_t)(warp + 1) * n_items / kFzWarps);
+    const int it0 = (int)((int64_t)warp * n_items / nwc), it1 = (int)((int64_t)(warp + 1) * n_items / nwc);
     // the lane's segment (g) and quarter (c): byte offsets within a gate/up row and a down row
     const int lg = lane >> 2, lc = lane & 3;
-    const uint32_t gu_lane_off = (uint32_t)lg * (d / 16) + (uint32_t)lc * (16 * NDK);
-    const uint32_t dn_lane_off = (uint32_t)lg * (f / 16) + (uint32_t)lc * (16 * NF);
+    const uint32_t gu_lane_off = (uint32_t)lg * (gu_row / 8) + (uint32_t)lc * (16 * NDK);
+    const uint32_t dn_lane_off = (uint32_t)lg * (dn_row_b / 8) + (uint32_t)lc * (16 * NF);
     const int grot = gu_rot<NDK>(lane), drot = dn_rot<NF>(lane);
     const uint64_t pol_first = policy_evict_first();
 
@@ -419,12 +512,16 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode_fused_kernel(const Fused
                 for (gu_r += nw; gu_r >= f; gu_r -= f) ++gu_u;
             }
             // the consumer finds its row and, in the two 16-byte slivers, its two scales
-            s_desc[warp][sidx] = make_int4(slot, r, (int)(((uintptr_t)sc >> 2) & 3), 4 + (int)(((uintptr_t)(sc + f) >> 2) & 3));
-            bar_expect_tx(bar, stage_bytes);
+            // bf16 rows have no scales (the slivers are not copied)
+            s_desc[warp][sidx] = BF ? make_int4(slot, r, 0, 0)
+                                    : make_int4(slot, r, (int)(((uintptr_t)sc >> 2) & 3), 4 + (int)(((uintptr_t)(sc + f) >> 2) & 3));
+            bar_expect_tx(bar, BF ? 2 * gu_row : stage_bytes);
             bulk_g2s_hint(dst, rows, gu_row, bar, pol_first);
             bulk_g2s_hint(dst + gu_row, rows + (size_t)f * gu_row, gu_row, bar, pol_first);
-            bulk_g2s(dst + 2 * gu_row, sliver(sc), 16, bar);
-            bulk_g2s(dst + 2 * gu_row + 16, sliver(sc + f), 16, bar);
+            if (!BF) {
+                bulk_g2s(dst + 2 * gu_row, sliver(sc), 16, bar);
+                bulk_g2s(dst + 2 * gu_row + 16, sliver(sc + f), 16, bar);
+            }
         } else {
             const int n = dn_count(dn_it, dn_row);
             const uint8_t* W = dn_u < k ? s_dn[dn_u] : a.sh_down;
@@ -449,41 +546,51 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode_fused_kernel(const Fused
                 bar_wait(saddr(&bars[warp][q2 % nst]), (uint32_t)(q2 / nst) & 1u);
     };
 
-    // ---- A: the shared expert's row pairs need no routing: queue them into every stage but the
-    //      last (which takes x), then this warp's first router piece, then wait for x
+    // ---- A: this warp's first router pieces (coalesced loads, all in flight) while x lands; once
+    //      x is in, the shared expert's row pairs (they need no routing) go into every stage but
+    //      the last, which holds x until the router pieces are done
     int limit = my_sh;            // lane 0: uses that may be issued so far
-    if (lane == 0)
-        while (issued < my_sh && issued < nst - 1) issue(issued++);
     const int n_units = E * nch;
-    // this warp's first two router pieces: every load of both in flight at once while x lands
-    float4 rw[8], rw2[8];
-    const int u2 = gw + nw;
+    float4 rw[8];
     if (gw < n_units) {
         const int e = gw / nch, p = gw - e * nch;
         load_router_piece(a.router_w + (size_t)e * d + 1024 * p, lane, rw);
     }
-    if (u2 < n_units) {
-        const int e = u2 / nch, p = u2 - e * nch;
-        load_router_piece(a.router_w + (size_t)e * d + 1024 * p, lane, rw2);
-    }
-    // the shared expert's down rows of this CTA are read last: start pulling them into L2
-    if (a.S && tid == kWarp && rj > 0) prefetch_l2(a.sh_down + (size_t)j0 * dn_row_b, (uint32_t)rj * dn_row_b);
     bool ok = __all_sync(0xffffffffu, bar_wait(saddr(&s_xbar), 0u));
     stamp(11);
-    // x as the lanes' fp16 MMA operand, once per CTA while the router loads are in flight: sigma
-    // from max|x|, then thread t converts the 8-column groups t, t + threads, ... into the lane
-    // blocks (lane L's block holds its groups in its visiting order; blocks are padded by 16 bytes
-    // so that the lanes' 16-byte loads meet no bank conflict).  The sum of x~ (fp64) is reduced
-    // in a fixed order, so every CTA gets the same value.
-    constexpr uint32_t kLaneBlk = 64 * NDK + 16;
-    const uint32_t xt_s = xraw_s + 2u * d;
-    __shared__ float s_redf[kFzWarps];
-    __shared__ double s_redd[kFzWarps];
-    int sig;
-    double xs;                    // sum of x~ = x 2^sigma over the whole row
-    {
+    if (lane == 0)
+        while (issued < my_sh && issued < nst - 1) issue(issued++);
+    // the shared expert's down rows of this CTA are read last: start pulling them into L2
+    if (a.S && tid == kWarp && rj > 0) prefetch_l2(a.sh_down + (size_t)j0 * dn_row_b, (uint32_t)rj * dn_row_b);
+    // x as the lanes' MMA operand, once per CTA: thread t places the 8-column groups t, t + threads,
+    // ... into the lane blocks.  int4: fp16 x~ = x 2^sigma, sigma from max|x|, the pairs of
+    // pairs_from_bf16; bf16: the bf16 values as they are.  The sum of x~ (fp64) is reduced in a
+    // fixed order, so every CTA gets the same value.
+    __shared__ float s_redf[kFzMaxWarps];
+    __shared__ double s_redd[kFzMaxWarps];
+    int sig = 0;
+    double xs = 0.0;              // sum of x~ = x 2^sigma over the whole row (bf16: of x)
+    if constexpr (BF) {
+        float part = 0.0f;
+        for (int g = tid; g < d / 8; g += blockDim.x) {
+            const uint4 v = lds16(xraw_s + 16u * (uint32_t)g);
+            const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) part += __uint_as_float(ws[i] << 16) + __uint_as_float(ws[i] & 0xffff0000u);
+            // group g (8 columns) belongs to lane L = 4 seg + quarter, as its group q
+            const int seg = g / (d / 64), rem = g - seg * (d / 64);
+            const int cq = rem / NDK, q = rem - cq * NDK, L = 4 * seg + cq;
+            int j = q - gu_rot<NDK>(L);
+            if (j < 0) j += NDK;
+            sts16(xt_s + (uint32_t)L * kLaneBlk + (uint32_t)j * 16u, v);
+        }
+        const double pd = warp_sum_d((double)part);
+        if (lane == 0) s_redd[warp] = pd;
+        __syncthreads();
+        for (int w = 0; w < nwc; ++w) xs += s_redd[w];
+    } else {
         float m = 0.0f;
-        for (int g = tid; g < d / 8; g += kFzThreads) {
+        for (int g = tid; g < d / 8; g += blockDim.x) {
             const uint4 v = lds16(xraw_s + 16u * (uint32_t)g);
             const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -495,11 +602,11 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode_fused_kernel(const Fused
         if (lane == 0) s_redf[warp] = m;
         __syncthreads();
         m = 0.0f;
-        for (int w = 0; w < kFzWarps; ++w) m = fmaxf(m, s_redf[w]);
+        for (int w = 0; w < nwc; ++w) m = fmaxf(m, s_redf[w]);
         sig = scale_exp(m);
         const float s1 = exp2i(sig), s16 = exp2i(sig - 4);
         float part = 0.0f;
-        for (int g = tid; g < d / 8; g += kFzThreads) {
+        for (int g = tid; g < d / 8; g += blockDim.x) {
             uint32_t pr[4];
             pairs_from_bf16(lds16(xraw_s + 16u * (uint32_t)g), s1, s16, pr, part);
             // group g belongs to lane L = 4 seg + quarter, as word w of its group q
@@ -513,8 +620,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode_fused_kernel(const Fused
         const double pd = warp_sum_d((double)part);
         if (lane == 0) s_redd[warp] = pd;
         __syncthreads();
-        xs = 0.0;
-        for (int w = 0; w < kFzWarps; ++w) xs += s_redd[w];
+        for (int w = 0; w < nwc; ++w) xs += s_redd[w];
     }
     // router pieces: unit u = (expert u / nch, columns [1024 p, 1024 p + 1024), p = u % nch)
     auto piece = [&](int u, const float4 (&wv)[8]) {
@@ -523,25 +629,13 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode_fused_kernel(const Fused
         if (lane == 0) __stcg(a.rpart + u, v);
     };
     if (gw < n_units) piece(gw, rw);
-    if (u2 < n_units) piece(u2, rw2);
-    for (int u = gw + 2 * nw; u < n_units; u += nw) {
+    for (int u = gw + nw; u < n_units; u += nw) {
         const int e = u / nch, p = u - e * nch;
         load_router_piece(a.router_w + (size_t)e * d + 1024 * p, lane, rw);
         piece(u, rw);
     }
     stamp(1);
-    // this lane's x~ registers, from its block
-    uint32_t xr[NDK][16];
-#pragma unroll
-    for (int j = 0; j < NDK; ++j)
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            const uint4 v = lds16(xt_s + (uint32_t)lane * kLaneBlk + (uint32_t)(4 * j + w) * 16u);
-            xr[j][4 * w] = v.x;
-            xr[j][4 * w + 1] = v.y;
-            xr[j][4 * w + 2] = v.z;
-            xr[j][4 * w + 3] = v.w;
-        }
+    const uint32_t xblk = xt_s + (uint32_t)lane * kLaneBlk;   // this lane's operand block
     const float xoff = 8.0f * (float)xs;                   // 8 sum x~
     const float xunscale = exp2i(-sig) * 16777216.0f;      // 2^(24 - sigma)
     // this thread's selection bias
@@ -571,14 +665,14 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode_fused_kernel(const Fused
         const int s = q % nst;
         const int4 dsc = s_desc[warp][s];
         const float* scs = reinterpret_cast<const float*>(st_g(s) + 2 * gu_row);
-        const float sg = scs[dsc.z], su = scs[dsc.w];
+        const float sg = BF ? 1.0f : scs[dsc.z], su = BF ? 1.0f : scs[dsc.w];
         __syncwarp();                                      // the stage is free again
         if (lane == 0)
             while (issued < limit && issued < q + 1 + nst) issue(issued++);
         const float ag = warp_sum(part.x), au = warp_sum(part.y);
         if (lane == n_pend) {
-            p_g = sg * fmaf(ag, xunscale, -xoff * exp2i(-sig));
-            p_u = su * fmaf(au, xunscale, -xoff * exp2i(-sig));
+            p_g = BF ? ag : sg * fmaf(ag, xunscale, -xoff * exp2i(-sig));
+            p_u = BF ? au : su * fmaf(au, xunscale, -xoff * exp2i(-sig));
             p_h = dsc.x * f + dsc.y;
         }
         if (++n_pend == kWarp) flush();
@@ -589,7 +683,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode_fused_kernel(const Fused
         if (lane == 0)
             while (issued < limit && issued < q + nst) issue(issued++);
         if (!wait_use(q)) { ok = false; break; }
-        gate_up_use(q, gu_mma<NDK>(st_s(q % nst), gu_row, gu_lane_off, grot, xr, lane));
+        gate_up_use(q, rows_mma_x<WK, NDK>(st_s(q % nst), st_s(q % nst) + gu_row, gu_lane_off, grot, xblk, lane));
     }
 
     // ---- B: selection by the whole CTA once every piece of the logits is stored.  The rings are
@@ -597,7 +691,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode_fused_kernel(const Fused
     __syncthreads();
     stamp(3);
     const uint32_t rbytes = ((uint32_t)n_units * 8u + 15u) & ~15u;
-    uint8_t* const rings = smem;
+    uint8_t* const rings = smem + kXtBytes;                // generic address of rings_s
     uint2* keys = reinterpret_cast<uint2*>(rings + rbytes);    // keys, order-preserving integers
     double* lgs = reinterpret_cast<double*>(keys + E);
     if (tid == 0) {
@@ -717,7 +811,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode_fused_kernel(const Fused
         float v = 0.0f;
         if (routed && it < it1) {
             const int u = it / rj, row = it - u * rj;
-            v = __ldg((u < k ? s_dns[u] : a.sh_dn_scale) + j0 + row);
+            v = BF ? 1.0f : __ldg((u < k ? s_dns[u] : a.sh_dn_scale) + j0 + row);
         }
         dsc_r[r] = v;
     }
@@ -734,7 +828,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode_fused_kernel(const Fused
             if (lane == 0)
                 while (issued < limit && issued < q + nst) issue(issued++);
             if (!wait_use(q)) { ok = false; break; }
-            gate_up_use(q, gu_mma<NDK>(st_s(q % nst), gu_row, gu_lane_off, grot, xr, lane));
+            gate_up_use(q, rows_mma_x<WK, NDK>(st_s(q % nst), st_s(q % nst) + gu_row, gu_lane_off, grot, xblk, lane));
         }
         if (ok && lane == 0)
             while (issued < limit && issued < q + nst) issue(issued++);
@@ -755,12 +849,24 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode_fused_kernel(const Fused
 
     // ---- D: down rows of this CTA's output block, slot by slot, two rows per MMA
     if (ok && s_ok) {
-        uint32_t hr[NF][16];
+        uint32_t hr[NF][HR];
         float hoff = 0.0f, hun = 0.0f;                     // 8 sum h~, 2^(24 - tau) of the current slot
         int cu = it0 / max(rj, 1), crow = it0 - cu * rj, hu = -1;
         for (int it = it0; it < it1; ++q) {
             const int n = dn_count(it, crow);
-            if (cu != hu) {                                // this slot's h (written by other CTAs)
+            if (cu != hu && BF) {                          // bf16: h as exact high + low bf16 parts
+                float part = 0.0f;
+#pragma unroll
+                for (int j = 0; j < NF; ++j) {
+                    int qq = j + drot;
+                    if (qq >= NF) qq -= NF;
+                    const uint4 v = ld_cg16(a.h + (size_t)cu * f + 8 * (lg * (f / 64) + lc * NF + qq));
+                    hilo_from_f16(v, &hr[j][0], part);
+                }
+                hoff = 0.0f;
+                hun = 1.0f;                                // the formula below then gives v itself
+                hu = cu;
+            } else if (cu != hu) {                         // int4: this slot's h~ (written by other CTAs)
                 uint4 hv[NF][4];
                 float m = 0.0f;
 #pragma unroll
@@ -783,10 +889,12 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode_fused_kernel(const Fused
                 const int tau = scale_exp(m);
                 const float s1 = exp2i(tau), s16 = exp2i(tau - 4);
                 float part = 0.0f;
+                if constexpr (!BF) {
 #pragma unroll
-                for (int j = 0; j < NF; ++j)
+                    for (int j = 0; j < NF; ++j)
 #pragma unroll
-                    for (int w = 0; w < 4; ++w) pairs_from_f16(hv[j][w], s1, s16, &hr[j][4 * w], part);
+                        for (int w = 0; w < 4; ++w) pairs_from_f16(hv[j][w], s1, s16, &hr[j][4 * w], part);
+                }
                 hoff = 8.0f * warp_sum(part);
                 hun = exp2i(-tau) * 16777216.0f;
                 hu = cu;
@@ -799,7 +907,7 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode_fused_kernel(const Fused
             for (int rr = 0; rr < n; rr += 2) {
                 const uint32_t rowA = st + (uint32_t)rr * dn_row_b;
                 const uint32_t rowB = rr + 1 < n ? rowA + dn_row_b : rowA;
-                const float2 pr = dn_mma<NF>(rowA, rowB, dn_lane_off, drot, hr, lane);
+                const float2 pr = rows_mma<WK, NF, HR, BF>(rowA, rowB, dn_lane_off, drot, hr, lane);
                 const float vA = warp_sum(pr.x), vB = warp_sum(pr.y);
                 const int iA = it + rr - it0, iB = iA + 1;
                 const float sA = __shfl_sync(0xffffffffu, dsc_r[0], iA & 31);
@@ -846,20 +954,42 @@ __global__ void __launch_bounds__(kFzThreads, 1) decode_fused_kernel(const Fused
     stamp(10);
 }
 
-size_t fz_stage_bytes(const LayerDims& L) { return (size_t)L.d + 32; }
-// Ring stages per warp (the kernel's constant for its d): 4 up to d = 6144, 3 above.
-int fz_stages(const LayerDims& L) { return L.d / 1024 <= 6 ? kFzMaxStages : kFzMaxStages - 1; }
-size_t fz_dyn_smem(const LayerDims& L) { return (size_t)fz_stages(L) * kFzWarps * fz_stage_bytes(L); }
+bool fz_bf16(const LayerDims& L) { return L.wkind == MOE_W_BF16; }
+size_t fz_row_bytes(const LayerDims& L, int cols) { return fz_bf16(L) ? (size_t)cols * 2 : (size_t)cols / 2; }
+size_t fz_stage_bytes(const LayerDims& L) { return 2 * fz_row_bytes(L, L.d) + 32; }
+// Bytes of the x~ lane blocks (the kernel's kXtBytes).
+size_t fz_xt_bytes(const LayerDims& L) {
+    const size_t blk = fz_bf16(L) ? 16 * (size_t)(L.d / 256) + 16 : 64 * (size_t)(L.d / 1024) + 16;
+    return (32 * blk + 127) / 128 * 128;
+}
+// Warps per CTA: as many (up to 16) as kFzStages ring stages each fit in shared memory beside the
+// lane blocks.
+int fz_warps(const LayerDims& L) {
+    const size_t room = kSmemLimit - kStaticReserve - fz_xt_bytes(L);
+    const int w = (int)(room / ((size_t)kFzStages * fz_stage_bytes(L)));
+    return w > kFzMaxWarps ? kFzMaxWarps : w;
+}
+size_t fz_dyn_smem(const LayerDims& L) {
+    return fz_xt_bytes(L) + (size_t)kFzStages * fz_warps(L) * fz_stage_bytes(L);
+}
 int fz_dn_rows(const LayerDims& L) {
-    const int r = (int)(fz_stage_bytes(L) / (size_t)(L.f / 2));
+    const int r = (int)(fz_stage_bytes(L) / fz_row_bytes(L, L.f));
     return r > kFzDnRowsMax ? kFzDnRowsMax : r;
 }
 
 template <int NDK>
 const void* fz_pick_f(int nf) {
-    return nf == 1 ? (const void*)decode_fused_kernel<NDK, 1> : (const void*)decode_fused_kernel<NDK, 2>;
+    return nf == 1 ? (const void*)decode_fused_kernel<MOE_W_INT4_ROWSCALE, NDK, 1>
+                   : (const void*)decode_fused_kernel<MOE_W_INT4_ROWSCALE, NDK, 2>;
 }
 const void* fz_pick(const LayerDims& L) {
+    if (fz_bf16(L)) {     // d = 1024 or 2048 (4 or 8 groups), f = 512 or 1024 (2 or 4 groups)
+        if (L.d == 1024)
+            return L.f == 512 ? (const void*)decode_fused_kernel<MOE_W_BF16, 4, 2>
+                              : (const void*)decode_fused_kernel<MOE_W_BF16, 4, 4>;
+        return L.f == 512 ? (const void*)decode_fused_kernel<MOE_W_BF16, 8, 2>
+                          : (const void*)decode_fused_kernel<MOE_W_BF16, 8, 4>;
+    }
     const int nf = L.f / 1024;
     switch (L.d / 1024) {
         case 1: return fz_pick_f<1>(nf);
@@ -876,14 +1006,16 @@ const void* fz_pick(const LayerDims& L) {
 }  // namespace
 
 bool decode_fused_shape_ok(const LayerDims& L) {
-    if (!(L.wkind == MOE_W_INT4_ROWSCALE && L.d % 1024 == 0 && L.d / 1024 >= 1 && L.d / 1024 <= 8 &&
-          (L.f == 1024 || L.f == 2048) && (!L.S || L.f_shared == L.f) && L.k + L.S <= kFzMaxSlots &&
-          L.E <= kWarp * kFzMaxPer && L.k <= L.E && fz_dn_rows(L) >= 1 &&
-          fz_dyn_smem(L) + kStaticReserve <= kSmemLimit))
+    const bool int4_shape = L.wkind == MOE_W_INT4_ROWSCALE && L.d % 1024 == 0 && L.d / 1024 >= 1 && L.d / 1024 <= 8 &&
+                            (L.f == 1024 || L.f == 2048);
+    const bool bf16_shape = L.wkind == MOE_W_BF16 && (L.d == 1024 || L.d == 2048) && (L.f == 512 || L.f == 1024);
+    if (!((int4_shape || bf16_shape) && (!L.S || L.f_shared == L.f) && L.k + L.S <= kFzMaxSlots &&
+          L.E <= kWarp * kFzMaxPer && L.k <= L.E && fz_dn_rows(L) >= 1 && fz_warps(L) >= 4))
         return false;
     // the selection keeps the router pieces, keys and logits in the (idle) rings; E <= threads
+    const size_t rings = (size_t)kFzStages * fz_warps(L) * fz_stage_bytes(L);
     const size_t sel_bytes = ((size_t)L.E * (L.d / 1024) * 8 + 15) / 16 * 16 + 16 * (size_t)L.E;
-    return sel_bytes <= fz_dyn_smem(L) && L.E <= kFzThreads;
+    return sel_bytes <= rings && L.E <= fz_warps(L) * kWarp;
 }
 
 cudaError_t prepare_decode_fused(const LayerDims& L, int num_sms, bool* usable) {
@@ -892,7 +1024,7 @@ cudaError_t prepare_decode_fused(const LayerDims& L, int num_sms, bool* usable) 
         return cudaSuccess;
     // the down items of one warp must fit the scale registers
     const int rows = (L.d + num_sms - 1) / num_sms;
-    if ((L.k + L.S) * rows > kFzWarps * kWarp * kFzScRegs - kFzWarps) return cudaSuccess;
+    if ((L.k + L.S) * rows > fz_warps(L) * (kWarp * kFzScRegs - 1)) return cudaSuccess;
     int dev = 0, coop = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
@@ -906,7 +1038,7 @@ cudaError_t prepare_decode_fused(const LayerDims& L, int num_sms, bool* usable) 
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(kSmemLimit - fa.sharedSizeBytes));
     if (e != cudaSuccess) return e;
     int blocks = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, fn, kFzThreads, dyn);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, fn, fz_warps(L) * kWarp, dyn);
     if (e != cudaSuccess) return e;
     *usable = blocks >= 1;
     return cudaSuccess;
@@ -948,7 +1080,7 @@ cudaError_t launch_decode_fused(const LayerDims& L, const moe_weights& W, const 
     a.scaling = L.scaling;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)num_sms);
-    cfg.blockDim = dim3((unsigned)kFzThreads);
+    cfg.blockDim = dim3((unsigned)(fz_warps(L) * kWarp));
     cfg.dynamicSmemBytes = fz_dyn_smem(L);
     cfg.stream = ctx.s;
     cudaLaunchAttribute attr[1];
