@@ -359,6 +359,40 @@ enum {
 moe_status moe_route_noalloc(const moe_config *cfg, const float *router_w, const float *router_bias,
                              const uint16_t *x, int32_t T, int32_t *idx, float *w, moe_stream stream);
 
+/*
+ * A device-memory tier of routed experts in front of host memory (colibri README, "The idea":
+ * routed experts streamed on demand behind a per-layer LRU cache and an optional pinned hot set;
+ * iliria page, "What's implemented": pinned/LRU slabs behind a ragged descriptor).  n_slots
+ * expert-sized device buffers hold the experts in use; host memory holds all E.
+ *
+ * moe_expert_cache_create -- cfg as for moe_layer_create.  device: router_w, router_bias and the
+ *   shared expert (device pointers, borrowed); its routed-expert fields are ignored.  host: the
+ *   routed experts in host memory (the same fields and layouts as moe_weights; pinned memory
+ *   makes the copies asynchronous), borrowed.  1 <= n_slots <= E.  Allocates the slots
+ *   (n_slots x one expert's bytes) and creates the layer (moe_expert_cache_layer), whose experts
+ *   are read through its pointer table.  Synchronous.
+ * moe_expert_cache_prepare -- route x ([T][d] bf16, device; 0 <= T <= max_tokens) and make every
+ *   expert it routes to resident: a free slot, else the least recently used slot whose expert is
+ *   neither pinned nor needed by this batch, is filled by host-to-device copies on `stream`, and
+ *   the layer's table is pointed at it.  Waits for the routing (the host needs the expert ids);
+ *   the copies stay asynchronous.  Call moe_forward on the same stream afterwards.
+ *   MOE_ERR_UNSUPPORTED: the batch needs more experts than the free and evictable slots.
+ * moe_expert_cache_pin -- pinned = 1 keeps expert e resident once loaded (the hot tier); 0 unpins.
+ * moe_expert_cache_stats -- experts found resident (hits), copied in (misses), bytes copied in,
+ *   and slots in use.  moe_expert_cache_slot_of -- the slot holding expert e, or -1.
+ * moe_expert_cache_destroy -- waits for the layer's last stream, frees the slots and the layer.
+ */
+typedef struct moe_expert_cache moe_expert_cache;
+moe_status moe_expert_cache_create(const moe_config *cfg, const moe_weights *device, const moe_weights *host,
+                                   int32_t n_slots, moe_expert_cache **out);
+moe_layer *moe_expert_cache_layer(moe_expert_cache *cache);
+moe_status moe_expert_cache_prepare(moe_expert_cache *cache, const uint16_t *x, int32_t T, moe_stream stream);
+moe_status moe_expert_cache_pin(moe_expert_cache *cache, int32_t e, int32_t pinned);
+moe_status moe_expert_cache_stats(const moe_expert_cache *cache, int64_t *hits, int64_t *misses, int64_t *bytes_in,
+                                  int32_t *resident);
+int32_t moe_expert_cache_slot_of(const moe_expert_cache *cache, int32_t e);
+void moe_expert_cache_destroy(moe_expert_cache *cache);
+
 moe_status moe_profile_enable(moe_layer *layer, int32_t on);
 moe_status moe_profile_read(moe_layer *layer, int32_t kernel, double *total_ms, int64_t *launches);
 const char *moe_kernel_name(int32_t kernel);

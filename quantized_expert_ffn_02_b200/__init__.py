@@ -25,6 +25,8 @@ EXPORTS = (
     "moe_layer_destroy", "moe_layer_workspace_bytes", "moe_layer_last_launches", "moe_status_str",
     "moe_profile_enable", "moe_profile_read", "moe_kernel_name", "moe_route_noalloc",
     "moe_layer_set_option", "moe_layer_get_option", "moe_layer_debug_read", "moe_layer_set_expert",
+    "moe_expert_cache_create", "moe_expert_cache_layer", "moe_expert_cache_prepare", "moe_expert_cache_pin",
+    "moe_expert_cache_stats", "moe_expert_cache_slot_of", "moe_expert_cache_destroy",
 )
 (MOE_OPT_PREFILL_MIN_TOKENS, MOE_OPT_PREFILL_AVAILABLE, MOE_OPT_SINGLE_TOKEN_KERNELS, MOE_OPT_PROGRAMMATIC_LAUNCH,
  MOE_OPT_WAIT_LIMIT_US, MOE_OPT_TEST_SKIP_GEMM_B_COPIES, MOE_OPT_ROUTER_GROUPS, MOE_OPT_ROUTER_TOP_P) = range(8)
@@ -89,9 +91,23 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         L.moe_layer_get_option.argtypes = [P, I32, ctypes.POINTER(I64)]
         L.moe_layer_debug_read.argtypes = [P, I32, P, I64]
         L.moe_layer_set_expert.argtypes = [P, I32, P, P, P, P, P]
+        L.moe_expert_cache_create.argtypes = [ctypes.POINTER(moe_config), ctypes.POINTER(moe_weights),
+                                              ctypes.POINTER(moe_weights), I32, ctypes.POINTER(P)]
+        L.moe_expert_cache_layer.argtypes = [P]
+        L.moe_expert_cache_layer.restype = P
+        L.moe_expert_cache_prepare.argtypes = [P, P, I32, P]
+        L.moe_expert_cache_pin.argtypes = [P, I32, I32]
+        L.moe_expert_cache_stats.argtypes = [P, ctypes.POINTER(I64), ctypes.POINTER(I64), ctypes.POINTER(I64),
+                                             ctypes.POINTER(I32)]
+        L.moe_expert_cache_slot_of.argtypes = [P, I32]
+        L.moe_expert_cache_slot_of.restype = I32
+        L.moe_expert_cache_destroy.argtypes = [P]
+        L.moe_expert_cache_destroy.restype = None
         for n in ("moe_pack_int4", "moe_pack_int8", "moe_pack_int2", "moe_layer_create", "moe_route", "moe_forward", "moe_forward_host",
                   "moe_forward_host_async", "moe_last_error", "moe_profile_enable", "moe_profile_read", "moe_route_noalloc",
-                  "moe_layer_set_option", "moe_layer_get_option", "moe_layer_debug_read", "moe_layer_set_expert"):
+                  "moe_layer_set_option", "moe_layer_get_option", "moe_layer_debug_read", "moe_layer_set_expert",
+                  "moe_expert_cache_create", "moe_expert_cache_prepare", "moe_expert_cache_pin",
+                  "moe_expert_cache_stats"):
             getattr(L, n).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -308,6 +324,61 @@ class MoELayer:
     def close(self):
         if self.handle:
             moe_layer_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class ExpertCache:
+    """A device-memory tier of routed experts in front of host memory (moe_expert_cache_*, see moe.h).
+
+    ``device`` holds the always-resident tensors (router_w, router_bias, shared_*; CUDA); ``host``
+    the routed experts (gate_up, gate_up_scale, down, down_scale; CPU tensors, pinned for
+    asynchronous copies).  ``layer`` is the layer to call forward on after ``prepare``."""
+
+    def __init__(self, d, f, n_experts, top_k, max_tokens, router, wkind, device: dict, host: dict, n_slots,
+                 n_shared=0, f_shared=0, routed_scaling_factor=1.0, out_bf16=False):
+        self.cfg = moe_config(d=d, f=f, n_experts=n_experts, top_k=top_k, n_shared=n_shared, f_shared=f_shared,
+                              max_tokens=max_tokens, router=router, routed_scaling_factor=routed_scaling_factor,
+                              wkind=wkind, out_bf16=1 if out_bf16 else 0)
+        self._tensors = (dict(device), dict(host))
+        self.dw = moe_weights(**{k: _ptr(v) for k, v in device.items()})
+        self.hw = moe_weights(**{k: _ptr(v) for k, v in host.items()})
+        h = ctypes.c_void_p()
+        _check(load().moe_expert_cache_create(ctypes.byref(self.cfg), ctypes.byref(self.dw), ctypes.byref(self.hw),
+                                              int(n_slots), ctypes.byref(h)), "moe_expert_cache_create")
+        self.handle = h.value
+        self.layer = load().moe_expert_cache_layer(self.handle)
+
+    def prepare(self, x, stream=None):
+        _check(load().moe_expert_cache_prepare(self.handle, _ptr(x), x.shape[0], _stream(stream)),
+               "moe_expert_cache_prepare")
+
+    def forward(self, x, out, stream=None):
+        moe_forward(self.layer, x, x.shape[0], out, stream)
+
+    def pin(self, e: int, on: bool = True):
+        _check(load().moe_expert_cache_pin(self.handle, int(e), 1 if on else 0), "moe_expert_cache_pin")
+
+    def stats(self) -> dict:
+        h, m, b, r = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int32()
+        _check(load().moe_expert_cache_stats(self.handle, ctypes.byref(h), ctypes.byref(m), ctypes.byref(b),
+                                             ctypes.byref(r)), "moe_expert_cache_stats")
+        return {"hits": h.value, "misses": m.value, "bytes_in": b.value, "resident": r.value}
+
+    def slot_of(self, e: int) -> int:
+        return int(load().moe_expert_cache_slot_of(self.handle, int(e)))
+
+    def last_error(self) -> int:
+        return moe_last_error(self.layer)
+
+    def close(self):
+        if self.handle:
+            load().moe_expert_cache_destroy(self.handle)
             self.handle = None
 
     def __del__(self):
