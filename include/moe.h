@@ -289,7 +289,9 @@ moe_status moe_layer_get_option(const moe_layer *layer, int32_t option, int64_t 
  * (waits for the layer's last stream).  For tests and debugging; the contents depend on which
  * kernels ran (see each item).  `bytes` is the size of `dst`; at most the item's size is copied.
  *   MOE_DEBUG_H      h = silu(g) * u, fp16 [slots][fmax] (slot = routed slot, then T*k + t for the
- *                    shared expert; K order of the grouped-GEMM path is permuted in groups of 8)
+ *                    shared expert; K order of the grouped-GEMM path is permuted in groups of 8;
+ *                    the single-launch T = 1 path stores 8-value chunk c of row [k+1][f] at
+ *                    position (c % (f/256)) * 32 + c / (f/256))
  *   MOE_DEBUG_Y      y per slot, fp32 [slots][d] (not written by the single-token kernels)
  *   MOE_DEBUG_IDX / MOE_DEBUG_W / MOE_DEBUG_ASC   int32 / fp32 / int32 [T][k]
  *   MOE_DEBUG_ULIST  int32 [E] unique chosen experts, ascending;  MOE_DEBUG_CNT int32 [E]

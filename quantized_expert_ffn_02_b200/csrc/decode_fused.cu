@@ -21,8 +21,8 @@
 //      pieces (the same order in every CTA, so every CTA selects the same experts) and forms an
 //      order-preserving integer key; the k best of each warp's 32 experts become candidates, and
 //      each candidate's rank among the candidates is its overall rank.  The k experts (ascending)
-//      and their gate weights go to shared memory, and the CTA asks L2 to prefetch the down rows
-//      it will read in D (read once, so the gate/up stream is marked evict-first).
+//      and their gate weights go to shared memory,  (the gate/up stream is
+//      marked evict-first, so the shared expert's down rows pulled into L2 in A stay there).
 //   C  routed gate/up: row pairs of the k experts, strided over every warp of the grid;
 //      h = SiLU(gate) * up in fp16 (global, L2), the SiLU of 32 row pairs at a time.  A warp that
 //      has finished its row pairs queues its first down rows (they do not depend on h), then the
@@ -80,7 +80,7 @@ constexpr int kFzRowsMax = 64;        // output rows per CTA
 constexpr int kFzDnRowsMax = 8;       // down rows per stage
 constexpr int kFzScRegs = 3;          // down-row scales per lane: up to 96 (slot, row) items per warp
 constexpr size_t kSmemLimit = 227 * 1024;
-constexpr int kStaticReserve = 5120;  // static shared memory of the kernel, rounded up
+constexpr int kStaticReserve = 6144;  // static shared memory of the kernel, rounded up
 
 struct FusedArgs {
     const float* router_w;            // [E][d] fp32
@@ -250,6 +250,16 @@ __device__ __forceinline__ int scale_exp(float vmax) {
     return max(-100, min(100, 14 - e));
 }
 
+// Where h[r] of a slot is kept: the lane that reads r in phase D owns the 8-value chunks
+// [L cpl, (L + 1) cpl) of the row (cpl = f / 256 chunks per lane), and chunk m of every lane is
+// stored at m * 32 + L, so that each 16-byte load of the warp reads 512 contiguous bytes.
+template <int F>
+__device__ __forceinline__ int h_pos(int r) {
+    constexpr int cpl = F / 256;
+    const int L = r / (8 * cpl), m = (r >> 3) % cpl;
+    return (m * kWarp + L) * 8 + (r & 7);
+}
+
 // Independent accumulator chains per dot product: an MMA's result feeds the next MMA of its chain
 // only, so a chain's latency is paid every kChains MMAs.
 constexpr int kChains = 4;
@@ -413,6 +423,7 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
     __shared__ int cand_e[kFzMaxPer * kFzMaxSlots];       // selection candidates, k per warp
     __shared__ uint2 cand_k[kFzMaxPer * kFzMaxSlots];     // and their keys
     __shared__ double sel_l[kFzMaxSlots];
+    __shared__ const void* sel_p[kFzMaxSlots][4];          // their weight pointers, rank order
     __shared__ unsigned long long s_base;                 // arrivals before this launch
     __shared__ int s_ok;
 
@@ -673,7 +684,7 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
         if (lane == n_pend) {
             p_g = BF ? ag : sg * fmaf(ag, xunscale, -xoff * exp2i(-sig));
             p_u = BF ? au : su * fmaf(au, xunscale, -xoff * exp2i(-sig));
-            p_h = dsc.x * f + dsc.y;
+            p_h = dsc.x * f + h_pos<f>(dsc.y);
         }
         if (++n_pend == kWarp) flush();
     };
@@ -757,6 +768,9 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
         if (sel && tid < nc) {
             const int e = cand_e[tid];
             if (e >= 0) {
+                // the candidate's weight pointers: loaded while the rank is counted
+                const void* pw[4] = {ex_gate_up(a.etab, E, e), ex_gu_scale(a.etab, E, e), ex_down(a.etab, E, e),
+                                     ex_dn_scale(a.etab, E, e)};
                 const uint2 mk = cand_k[tid];
                 int rank = 0;
 #pragma unroll 8
@@ -765,6 +779,8 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
                 if (rank < k) {
                     sel_e[rank] = e;
                     sel_l[rank] = lgs[e];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) sel_p[rank][i] = pw[i];
                 }
             }
         }
@@ -776,18 +792,16 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
             if (lane < k) {
                 s_e[pk.pos] = pk.e;
                 s_w[pk.pos] = pk.w;
-                s_gu[pk.pos] = ex_gate_up(a.etab, E, pk.e);
-                s_gus[pk.pos] = ex_gu_scale(a.etab, E, pk.e);
-                s_dn[pk.pos] = ex_down(a.etab, E, pk.e);
-                s_dns[pk.pos] = ex_dn_scale(a.etab, E, pk.e);
+                s_gu[pk.pos] = static_cast<const uint8_t*>(sel_p[lane][0]);     // rank lane is expert pk.e
+                s_gus[pk.pos] = static_cast<const float*>(sel_p[lane][1]);
+                s_dn[pk.pos] = static_cast<const uint8_t*>(sel_p[lane][2]);
+                s_dns[pk.pos] = static_cast<const float*>(sel_p[lane][3]);
                 if (blockIdx.x == 0) {
                     a.idx[lane] = pk.e;
                     a.wts[lane] = pk.w;
                     a.asc[pk.pos] = lane;
                     a.ulist[pk.pos] = pk.e;
                 }
-                // this CTA's down rows of the routed expert: into L2 while gate/up streams
-                if (rj > 0) prefetch_l2(ex_down(a.etab, E, pk.e) + (size_t)j0 * dn_row_b, (uint32_t)rj * dn_row_b);
             }
             if (blockIdx.x == 0 && lane == 0) {
                 *a.n_unique = k;
@@ -860,7 +874,7 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
                 for (int j = 0; j < NF; ++j) {
                     int qq = j + drot;
                     if (qq >= NF) qq -= NF;
-                    const uint4 v = ld_cg16(a.h + (size_t)cu * f + 8 * (lg * (f / 64) + lc * NF + qq));
+                    const uint4 v = ld_cg16(a.h + (size_t)cu * f + 8 * (qq * kWarp + lane));
                     hilo_from_f16(v, &hr[j][0], part);
                 }
                 hoff = 0.0f;
@@ -875,7 +889,7 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
                     if (qq >= NF) qq -= NF;
 #pragma unroll
                     for (int w = 0; w < 4; ++w) {
-                        hv[j][w] = ld_cg16(a.h + (size_t)cu * f + 8 * (lg * (f / 64) + lc * 4 * NF + 4 * qq + w));
+                        hv[j][w] = ld_cg16(a.h + (size_t)cu * f + 8 * ((4 * qq + w) * kWarp + lane));
                         const uint32_t ws[4] = {hv[j][w].x, hv[j][w].y, hv[j][w].z, hv[j][w].w};
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
