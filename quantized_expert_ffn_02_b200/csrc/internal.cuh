@@ -121,6 +121,8 @@ struct Workspace {
     // creation; moe_layer_set_expert re-points one expert (a non-contiguous expert slab).
     const void** etab;
     double* rpart;         // [E][d / 1024]: pieces of the router logits
+    double* rsplit;        // partial logits and sums of x of the K-sliced router GEMM
+    size_t rsplit_n;       // its length in doubles (0: none)
     unsigned long long* gbar;  // [1]: grid-barrier arrivals (only grows)
     unsigned long long* trace; // [kTraceCtas][kTraceStamps]: phase timestamps of that path
 };
@@ -184,9 +186,12 @@ cudaError_t launch_pack_int4(const float* w, int64_t rows, int64_t cols, uint8_t
 // bits = 8 (int8 container) or 2 (packed int2)
 cudaError_t launch_pack_tier(int bits, const float* w, int64_t rows, int64_t cols, uint8_t* packed, float* scales,
                              int* status, cudaStream_t s);
+// part (nullable, part_doubles long): room for the K-sliced router GEMM's partial logits and sums
+// of x; router_split_doubles gives the size that lets every batch up to max_tokens use it.
 cudaError_t launch_router(const LayerDims& L, const float* router_w, const float* router_bias,
                           const uint16_t* x, int T, double* logits, double* xsum, int32_t* idx, float* wts,
-                          int32_t* asc, const Launch& ctx);
+                          int32_t* asc, const Launch& ctx, double* part, size_t part_doubles);
+size_t router_split_doubles(int E, int max_tokens);
 cudaError_t launch_bucket(const LayerDims& L, int T, const Workspace& ws, const Launch& ctx);
 // Small batches: logits, top-k, gate weights and bucket tables in one launch.
 constexpr int kRouteSmallMaxT = 32;

@@ -134,6 +134,8 @@ size_t carve(const moe_config& c, size_t max_groups, char* base, qe::Workspace* 
     };
     qe::Workspace w{};
     w.logits = (double*)take(sizeof(double) * T * E);
+    w.rsplit_n = qe::router_split_doubles((int)E, (int)T);
+    w.rsplit = w.rsplit_n ? (double*)take(sizeof(double) * w.rsplit_n) : nullptr;
     w.idx = (int32_t*)take(sizeof(int32_t) * T * k);
     w.wts = (float*)take(sizeof(float) * T * k);
     w.asc = (int32_t*)take(sizeof(int32_t) * T * k);
@@ -337,7 +339,7 @@ moe_status moe_route(moe_layer* L, const uint16_t* x, int32_t T, int32_t* idx, f
     int launches = 0;
     const qe::Launch ctx{s, &launches, &L->prof};
     cudaError_t e = qe::launch_router(L->dims, L->w.router_w, L->w.router_bias, x, T, L->ws.logits, L->ws.xsum, idx, w,
-                                      nullptr, ctx);
+                                      nullptr, ctx, L->ws.rsplit, L->ws.rsplit_n);
     L->last_stream = s;
     L->last_launches = launches;
     return from_cuda(e);
@@ -366,7 +368,7 @@ moe_status moe_forward(moe_layer* L, const uint16_t* x, int32_t T, void* out, mo
         e = qe::launch_route_small(L->dims, L->w.router_w, L->w.router_bias, x, T, ws, ctx);
     } else {
         e = qe::launch_router(L->dims, L->w.router_w, L->w.router_bias, x, T, ws.logits, ws.xsum, ws.idx, ws.wts,
-                              ws.asc, ctx);
+                              ws.asc, ctx, ws.rsplit, ws.rsplit_n);
         if (e == cudaSuccess) e = qe::launch_bucket(L->dims, T, ws, ctx);
     }
     if (e == cudaSuccess) {

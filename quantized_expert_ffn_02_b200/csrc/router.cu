@@ -74,8 +74,14 @@ router_logits_kernel(const float* __restrict__ wr, const uint16_t* __restrict__ 
 // (wm, wn) of the 2 x 4 warp grid owns 32 tokens x 16 experts, i.e. 4 x 2 tiles of 8 x 8.  The
 // next K chunk's global loads are in flight while the current chunk is multiplied.  CTAs of the
 // first expert tile also write sum_i x[t][i].
+//
+// The K range may be split over gridDim.z CTAs (slice z covers [z d / Z, (z + 1) d / Z)): slice z
+// writes its partial logits to logits + z T E and its partial sums of x to xsum + z T, and the
+// top-k kernel adds the slices in slice order.  More CTAs keep every SM's FP64 pipe busy: with
+// one slice a 2048-token batch has 128 CTAs for 148 SMs, each a long chain of dependent chunks.
 // ---------------------------------------------------------------------------------------
 constexpr int kRgT = 64, kRgE = 64, kRgK = 32, kRgThreads = 256;
+constexpr int kRgSplitMax = 3;
 
 __global__ void __launch_bounds__(kRgThreads)
 router_gemm_kernel(const float* __restrict__ wr, const uint16_t* __restrict__ x, int T, int d, int E,
@@ -86,12 +92,15 @@ router_gemm_kernel(const float* __restrict__ wr, const uint16_t* __restrict__ x,
     const int wm = warp / 4, wn = warp % 4;                // 32 tokens x 16 experts per warp
     const int g = lane / 4, tq = lane % 4;                 // fragment row / column group
     const int t0 = blockIdx.x * kRgT, e0 = blockIdx.y * kRgE;
+    const int kz = d / (int)gridDim.z, kb = (int)blockIdx.z * kz;      // this CTA's K slice
+    logits += (size_t)blockIdx.z * T * E;
+    xsum += (size_t)blockIdx.z * T;
     // loader roles: 4 threads per token row (8 bf16 each) and per expert row (8 fp32 each)
     const int lr = tid / 4, lc = (tid % 4) * 8;
     const bool xrow_ok = t0 + lr < T;
     const bool sum_x = blockIdx.y == 0;
-    const uint16_t* xrow = x + (size_t)(xrow_ok ? t0 + lr : 0) * d + lc;
-    const float* wrow = wr + (size_t)(e0 + lr) * d + lc;
+    const uint16_t* xrow = x + (size_t)(xrow_ok ? t0 + lr : 0) * d + kb + lc;
+    const float* wrow = wr + (size_t)(e0 + lr) * d + kb + lc;
     uint4 xv = xrow_ok ? ld_ro16(xrow) : make_uint4(0, 0, 0, 0);
     float4 wa = __ldg(reinterpret_cast<const float4*>(wrow)), wb = __ldg(reinterpret_cast<const float4*>(wrow) + 1);
     double acc[4][2][2];                                   // [token tile][expert tile][c0, c1]
@@ -100,7 +109,7 @@ router_gemm_kernel(const float* __restrict__ wr, const uint16_t* __restrict__ x,
 #pragma unroll
         for (int j = 0; j < 2; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
     double xpart = 0.0;
-    for (int k0 = 0; k0 < d; k0 += kRgK) {
+    for (int k0 = 0; k0 < kz; k0 += kRgK) {
         // convert the staged chunk into shared memory (K-major)
         const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
@@ -115,7 +124,7 @@ router_gemm_kernel(const float* __restrict__ wr, const uint16_t* __restrict__ x,
         for (int q = 0; q < 8; ++q) ws[lc + q][lr] = (double)wv[q];
         __syncthreads();
         // next chunk's loads go out before this chunk is multiplied
-        if (k0 + kRgK < d) {
+        if (k0 + kRgK < kz) {
             xv = xrow_ok ? ld_ro16(xrow + k0 + kRgK) : make_uint4(0, 0, 0, 0);
             wa = __ldg(reinterpret_cast<const float4*>(wrow + k0 + kRgK));
             wb = __ldg(reinterpret_cast<const float4*>(wrow + k0 + kRgK) + 1);
@@ -159,11 +168,14 @@ router_gemm_kernel(const float* __restrict__ wr, const uint16_t* __restrict__ x,
 
 // One warp per token: top-k and gate weights.
 // Writes idx[t][r] / w[t][r] in rank order and asc[t][p] = the rank whose expert is the
-// p-th smallest of the token's k experts.
+// p-th smallest of the token's k experts.  With nsplit > 1 the logits are the sum of nsplit K
+// slices (slice z at logits + z T E, added in slice order), and xsum[t] is formed the same way
+// from the slices at xpart.
 template <int MAXPER>
 __global__ void __launch_bounds__(256)
-topk_kernel(const double* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k, int router,
-            float scaling, int32_t* __restrict__ idx_out, float* __restrict__ w_out, int32_t* __restrict__ asc_out,
+topk_kernel(const double* __restrict__ logits, int nsplit, const double* __restrict__ xpart, double* __restrict__ xsum,
+            const float* __restrict__ bias, int T, int E, int k, int router, float scaling,
+            int32_t* __restrict__ idx_out, float* __restrict__ w_out, int32_t* __restrict__ asc_out,
             const RouterOpts opts) {
     const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
     const int t = blockIdx.x * (blockDim.x / kWarp) + warp;
@@ -172,7 +184,17 @@ topk_kernel(const double* __restrict__ logits, const float* __restrict__ bias, i
 #pragma unroll
     for (int m = 0; m < MAXPER; ++m) {
         const int e = lane + kWarp * m;
-        lg[m] = e < E ? logits[(size_t)t * E + e] : 0.0;
+        double v = 0.0;
+        if (e < E) {
+            v = logits[(size_t)t * E + e];
+            for (int z = 1; z < nsplit; ++z) v += logits[((size_t)z * T + t) * E + e];
+        }
+        lg[m] = v;
+    }
+    if (xpart && lane == 0) {
+        double v = xpart[t];
+        for (int z = 1; z < nsplit; ++z) v += xpart[(size_t)z * T + t];
+        xsum[t] = v;
     }
     float bv[MAXPER];
     load_bias<MAXPER>(bias, E, lane, bv);
@@ -214,7 +236,7 @@ __device__ void warp_select(const double* __restrict__ lg, const float* __restri
     }
 }
 
-template <int MAXPER>
+template <int MAXPER, int MAXC>
 __global__ void __launch_bounds__(kSmallThreads, 2)
 route_small_kernel(const float* __restrict__ wr, const float* __restrict__ bias, const uint16_t* __restrict__ x, int T,
                    int d, int E, int k, int router, float scaling, double* __restrict__ logits,
@@ -222,41 +244,71 @@ route_small_kernel(const float* __restrict__ wr, const float* __restrict__ bias,
                    int32_t* __restrict__ asc, int32_t* __restrict__ cnt, int32_t* __restrict__ off,
                    int32_t* __restrict__ perm, int32_t* __restrict__ slot_of, int32_t* __restrict__ ulist,
                    int32_t* __restrict__ n_unique, unsigned int* __restrict__ counter, const RouterOpts opts) {
+    constexpr int TT = MAXC > 8 ? 1 : MAXPER > 8 ? 2 : 4;  // tokens per pass (within the register budget)
     __shared__ double red[kSmallThreads / kWarp][kSmallMaxT];
-    __shared__ double redx[kSmallThreads / kWarp];
+    __shared__ double redx[kSmallThreads / kWarp][2];
     __shared__ int s_cnt[kSmallMaxE], s_off[kSmallMaxE], s_scan[kSmallThreads];
     __shared__ int am_last;
     const int e = blockIdx.x, tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
     // A kernel launched after this one with programmatic dependent launch may start now: it
     // waits (griddepcontrol.wait) before it reads anything written here.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    // ---- logits of expert e for every token
-    // all of this thread's router-row loads in flight at once (d <= 14336: at most 14 per thread)
-    constexpr int kMaxC = 14;
+    // ---- logits of expert e for every token, TT tokens per pass: the pass's x loads are all in
+    //      flight at once and its TT fp64 chains are independent.  The router row stays in
+    //      registers (MAXC float4 per thread).  Block b also sums x of the tokens t == b (mod E).
     const float4* wrow = reinterpret_cast<const float4*>(wr + (size_t)e * d);
     const int nc = (d / 4 - tid + kSmallThreads - 1) / kSmallThreads;
-    float4 wv[kMaxC];
+    float4 wv[MAXC];
 #pragma unroll
-    for (int j = 0; j < kMaxC; ++j)
+    for (int j = 0; j < MAXC; ++j)
         if (j < nc) wv[j] = __ldg(wrow + tid + kSmallThreads * j);
-    for (int t = 0; t < T; ++t) {
-        const uint2* xr2 = reinterpret_cast<const uint2*>(x + (size_t)t * d) + tid;
-        uint2 xv[kMaxC];
+    int n_sums = 0;                                        // x sums this block owes (tokens e, e + E, ...)
+    for (int t0 = 0; t0 < T; t0 += TT) {
+        uint2 xv[TT][MAXC];
 #pragma unroll
-        for (int j = 0; j < kMaxC; ++j)
-            if (j < nc) xv[j] = __ldg(xr2 + kSmallThreads * j);
-        double a = 0.0;
+        for (int u = 0; u < TT; ++u) {
+            const int t = min(t0 + u, T - 1);
+            const uint2* xr2 = reinterpret_cast<const uint2*>(x + (size_t)t * d) + tid;
 #pragma unroll
-        for (int j = 0; j < kMaxC; ++j) {
+            for (int j = 0; j < MAXC; ++j)
+                if (j < nc) xv[u][j] = __ldg(xr2 + kSmallThreads * j);
+        }
+        double a[TT];
+#pragma unroll
+        for (int u = 0; u < TT; ++u) a[u] = 0.0;
+#pragma unroll
+        for (int j = 0; j < MAXC; ++j) {
             if (j < nc) {
-                a = fma((double)__uint_as_float(xv[j].x << 16), (double)wv[j].x, a);
-                a = fma((double)__uint_as_float(xv[j].x & 0xffff0000u), (double)wv[j].y, a);
-                a = fma((double)__uint_as_float(xv[j].y << 16), (double)wv[j].z, a);
-                a = fma((double)__uint_as_float(xv[j].y & 0xffff0000u), (double)wv[j].w, a);
+#pragma unroll
+                for (int u = 0; u < TT; ++u) {
+                    a[u] = fma((double)__uint_as_float(xv[u][j].x << 16), (double)wv[j].x, a[u]);
+                    a[u] = fma((double)__uint_as_float(xv[u][j].x & 0xffff0000u), (double)wv[j].y, a[u]);
+                    a[u] = fma((double)__uint_as_float(xv[u][j].y << 16), (double)wv[j].z, a[u]);
+                    a[u] = fma((double)__uint_as_float(xv[u][j].y & 0xffff0000u), (double)wv[j].w, a[u]);
+                }
             }
         }
-        a = warp_sum_d(a);
-        if (lane == 0) red[warp][t] = a;
+#pragma unroll
+        for (int u = 0; u < TT; ++u) {
+            const int t = t0 + u;
+            if (t < T) {
+                const double v = warp_sum_d(a[u]);
+                if (lane == 0) red[warp][t] = v;
+                if (t % E == e) {                          // this block's x sum, from the same loads
+                    double sx = 0.0;
+#pragma unroll
+                    for (int j = 0; j < MAXC; ++j)
+                        if (j < nc)
+                            sx += ((double)__uint_as_float(xv[u][j].x << 16) +
+                                   (double)__uint_as_float(xv[u][j].x & 0xffff0000u)) +
+                                  ((double)__uint_as_float(xv[u][j].y << 16) +
+                                   (double)__uint_as_float(xv[u][j].y & 0xffff0000u));
+                    sx = warp_sum_d(sx);
+                    if (lane == 0) redx[warp][n_sums & 1] = sx;
+                    ++n_sums;
+                }
+            }
+        }
     }
     __syncthreads();
     if (tid < T) {
@@ -264,18 +316,24 @@ route_small_kernel(const float* __restrict__ wr, const float* __restrict__ bias,
         for (int w = 0; w < kSmallThreads / kWarp; ++w) s += red[w][tid];
         logits[(size_t)tid * E + e] = s;
     }
-    // ---- sum of x for the tokens t with t % E == e (one block per token)
-    for (int t = e; t < T; t += E) {
-        double s = 0.0;
-        for (int i = tid; i < d; i += kSmallThreads) s += (double)bf16_bits_to_f32(x[(size_t)t * d + i]);
-        s = warp_sum_d(s);
-        __syncthreads();
-        if (lane == 0) redx[warp] = s;
-        __syncthreads();
-        if (tid == 0) {
-            double tot = 0.0;
-            for (int w = 0; w < kSmallThreads / kWarp; ++w) tot += redx[w];
-            xsum[t] = tot;
+    // at most one x sum per block while T <= E; more only for tiny E (then sum them again here)
+    if (n_sums == 1 && tid == 0) {
+        double tot = 0.0;
+        for (int w = 0; w < kSmallThreads / kWarp; ++w) tot += redx[w][0];
+        xsum[e] = tot;
+    } else if (n_sums > 1) {
+        for (int t = e; t < T; t += E) {
+            double sx = 0.0;
+            for (int i = tid; i < d; i += kSmallThreads) sx += (double)bf16_bits_to_f32(x[(size_t)t * d + i]);
+            sx = warp_sum_d(sx);
+            __syncthreads();
+            if (lane == 0) redx[warp][0] = sx;
+            __syncthreads();
+            if (tid == 0) {
+                double tot = 0.0;
+                for (int w = 0; w < kSmallThreads / kWarp; ++w) tot += redx[w][0];
+                xsum[t] = tot;
+            }
         }
     }
     // ---- the last block to finish selects and buckets
@@ -347,21 +405,21 @@ cudaError_t launch_route_small(const LayerDims& L, const float* router_w, const 
     if (T == 0) return cudaSuccess;
     const float* bias = L.router == MOE_ROUTER_SIGMOID_BIAS ? router_bias : nullptr;
     unsigned int* counter = reinterpret_cast<unsigned int*>(ws.counter);
-    if (L.E <= 32)
-        QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,
-                  (route_small_kernel<1><<<L.E, kSmallThreads, 0, ctx.s>>>(
-                      router_w, bias, x, T, L.d, L.E, L.k, L.router, L.scaling, ws.logits, ws.xsum, ws.idx, ws.wts,
-                      ws.asc, ws.cnt, ws.off, ws.perm, ws.slot_of, ws.ulist, ws.n_unique, counter, L.ropts)));
-    else if (L.E <= 256)
-        QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,
-                  (route_small_kernel<8><<<L.E, kSmallThreads, 0, ctx.s>>>(
-                      router_w, bias, x, T, L.d, L.E, L.k, L.router, L.scaling, ws.logits, ws.xsum, ws.idx, ws.wts,
-                      ws.asc, ws.cnt, ws.off, ws.perm, ws.slot_of, ws.ulist, ws.n_unique, counter, L.ropts)));
-    else
-        QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,
-                  (route_small_kernel<32><<<L.E, kSmallThreads, 0, ctx.s>>>(
-                      router_w, bias, x, T, L.d, L.E, L.k, L.router, L.scaling, ws.logits, ws.xsum, ws.idx, ws.wts,
-                      ws.asc, ws.cnt, ws.off, ws.perm, ws.slot_of, ws.ulist, ws.n_unique, counter, L.ropts)));
+    // router-row registers per thread: 6 float4 cover d <= 6144, 14 cover d <= 14336
+    const bool narrow = (L.d / 4 + kSmallThreads - 1) / kSmallThreads <= 6;
+#define QE_ROUTE_SMALL(MAXPER, MAXC)                                                                              \
+    QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,                                                                      \
+              (route_small_kernel<MAXPER, MAXC><<<L.E, kSmallThreads, 0, ctx.s>>>(                              \
+                  router_w, bias, x, T, L.d, L.E, L.k, L.router, L.scaling, ws.logits, ws.xsum, ws.idx, ws.wts,  \
+                  ws.asc, ws.cnt, ws.off, ws.perm, ws.slot_of, ws.ulist, ws.n_unique, counter, L.ropts)))
+    if (L.E <= 32) {
+        if (narrow) QE_ROUTE_SMALL(1, 6); else QE_ROUTE_SMALL(1, 14);
+    } else if (L.E <= 256) {
+        if (narrow) QE_ROUTE_SMALL(8, 6); else QE_ROUTE_SMALL(8, 14);
+    } else {
+        if (narrow) QE_ROUTE_SMALL(32, 6); else QE_ROUTE_SMALL(32, 14);
+    }
+#undef QE_ROUTE_SMALL
     return cudaSuccess;
 }
 
@@ -373,15 +431,32 @@ cudaError_t prepare_router(const LayerDims& L) {
     return cudaFuncSetAttribute(router_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
 }
 
+size_t router_split_doubles(int E, int max_tokens) {
+    if (max_tokens < kRgT || E % kRgE) return 0;
+    return (size_t)kRgSplitMax * ((size_t)max_tokens * E + (size_t)max_tokens);
+}
+
 cudaError_t launch_router(const LayerDims& L, const float* router_w, const float* router_bias,
                           const uint16_t* x, int T, double* logits, double* xsum, int32_t* idx, float* wts,
-                          int32_t* asc, const Launch& ctx) {
+                          int32_t* asc, const Launch& ctx, double* part, size_t part_doubles) {
     if (T == 0) return cudaSuccess;
     const cudaStream_t s = ctx.s;
+    int nsplit = 1;
+    const double* lg = logits;
+    const double* xpart = nullptr;
     if (T >= kRgT && L.E % kRgE == 0 && L.d % kRgK == 0) {
-        dim3 grid((unsigned)((T + kRgT - 1) / kRgT), (unsigned)(L.E / kRgE));
+        for (int z = kRgSplitMax; z > 1 && part; --z)
+            if (L.d % (kRgK * z) == 0 && part_doubles >= (size_t)z * ((size_t)T * L.E + T)) {
+                nsplit = z;
+                break;
+            }
+        double* lg_dst = nsplit > 1 ? part : logits;
+        double* xs_dst = nsplit > 1 ? part + (size_t)nsplit * T * L.E : xsum;
+        lg = lg_dst;
+        if (nsplit > 1) xpart = xs_dst;
+        dim3 grid((unsigned)((T + kRgT - 1) / kRgT), (unsigned)(L.E / kRgE), (unsigned)nsplit);
         QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,
-                  (router_gemm_kernel<<<grid, kRgThreads, 0, s>>>(router_w, x, T, L.d, L.E, logits, xsum)));
+                  (router_gemm_kernel<<<grid, kRgThreads, 0, s>>>(router_w, x, T, L.d, L.E, lg_dst, xs_dst)));
     } else {
         const size_t smem = (size_t)kRouterTokens * L.d * sizeof(uint16_t);
         dim3 grid((L.E + kRouterWarps - 1) / kRouterWarps, (T + kRouterTokens - 1) / kRouterTokens);
@@ -393,13 +468,13 @@ cudaError_t launch_router(const LayerDims& L, const float* router_w, const float
     const unsigned g = (unsigned)((T + tpb - 1) / tpb);
     const float* bias = L.router == MOE_ROUTER_SIGMOID_BIAS ? router_bias : nullptr;
     if (L.E <= 32)
-        QE_LAUNCH(ctx, MOE_KERNEL_TOPK, (topk_kernel<1><<<g, tpb * kWarp, 0, s>>>(logits, bias, T, L.E, L.k, L.router,
+        QE_LAUNCH(ctx, MOE_KERNEL_TOPK, (topk_kernel<1><<<g, tpb * kWarp, 0, s>>>(lg, nsplit, xpart, xsum, bias, T, L.E, L.k, L.router,
                                                                                     L.scaling, idx, wts, asc, L.ropts)));
     else if (L.E <= 256)
-        QE_LAUNCH(ctx, MOE_KERNEL_TOPK, (topk_kernel<8><<<g, tpb * kWarp, 0, s>>>(logits, bias, T, L.E, L.k, L.router,
+        QE_LAUNCH(ctx, MOE_KERNEL_TOPK, (topk_kernel<8><<<g, tpb * kWarp, 0, s>>>(lg, nsplit, xpart, xsum, bias, T, L.E, L.k, L.router,
                                                                                     L.scaling, idx, wts, asc, L.ropts)));
     else
-        QE_LAUNCH(ctx, MOE_KERNEL_TOPK, (topk_kernel<32><<<g, tpb * kWarp, 0, s>>>(logits, bias, T, L.E, L.k, L.router,
+        QE_LAUNCH(ctx, MOE_KERNEL_TOPK, (topk_kernel<32><<<g, tpb * kWarp, 0, s>>>(lg, nsplit, xpart, xsum, bias, T, L.E, L.k, L.router,
                                                                                      L.scaling, idx, wts, asc, L.ropts)));
     return cudaSuccess;
 }
@@ -482,6 +557,6 @@ extern "C" moe_status moe_route_noalloc(const moe_config* cfg, const float* rout
     int launches = 0;
     const qe::Launch ctx{(cudaStream_t)stream, &launches, nullptr};
     const float* bias = cfg->router == MOE_ROUTER_SIGMOID_BIAS ? router_bias : nullptr;
-    cudaError_t e = qe::launch_router(L, router_w, bias, x, T, logits, xsum, idx, w, nullptr, ctx);
+    cudaError_t e = qe::launch_router(L, router_w, bias, x, T, logits, xsum, idx, w, nullptr, ctx, nullptr, 0);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
