@@ -277,10 +277,15 @@ void moe_layer_destroy(moe_layer *layer);
  *                               0 for them, and moe_forward never reads their weights.
  *   While either variant is on, T = 1 batches run on the general decode kernels (the single-token
  *   paths take the plain router only).  moe_route_noalloc always uses the plain router.
+ *   MOE_OPT_UNION_TENSOR_CORES   batches of 2 .. prefill-threshold tokens with int4 experts (d, f and
+ *                               the shared f multiples of 1024): 1 (default) runs gate/up and down as
+ *                               tensor-core products of 16 weight rows by up to 8 tokens; 0 runs the
+ *                               general kernels (FP32-pipe dot products).  Results agree within the
+ *                               layer's tolerance, not bit for bit.
  */
 enum { MOE_OPT_PREFILL_MIN_TOKENS = 0, MOE_OPT_PREFILL_AVAILABLE = 1, MOE_OPT_SINGLE_TOKEN_KERNELS = 2,
        MOE_OPT_PROGRAMMATIC_LAUNCH = 3, MOE_OPT_WAIT_LIMIT_US = 4, MOE_OPT_TEST_SKIP_GEMM_B_COPIES = 5,
-       MOE_OPT_ROUTER_GROUPS = 6, MOE_OPT_ROUTER_TOP_P = 7 };
+       MOE_OPT_ROUTER_GROUPS = 6, MOE_OPT_ROUTER_TOP_P = 7, MOE_OPT_UNION_TENSOR_CORES = 8 };
 moe_status moe_layer_set_option(moe_layer *layer, int32_t option, int64_t value);
 moe_status moe_layer_get_option(const moe_layer *layer, int32_t option, int64_t *value);
 

@@ -193,6 +193,12 @@ cudaError_t launch_router(const LayerDims& L, const float* router_w, const float
                           int32_t* asc, const Launch& ctx, double* part, size_t part_doubles);
 size_t router_split_doubles(int E, int max_tokens);
 cudaError_t launch_bucket(const LayerDims& L, int T, const Workspace& ws, const Launch& ctx);
+// Small batches (T >= 2), int4 experts with d, f (and the shared f) multiples of 1024: gate/up and
+// down as 16-row x 8-token tensor-core products (decode_mma.cu).
+bool decode_mma_ok(const LayerDims& L, int T);
+cudaError_t prepare_decode_mma();
+cudaError_t launch_decode_mma(const LayerDims& L, const moe_weights& W, const uint16_t* x, int T, const Workspace& ws,
+                              int num_sms, const Launch& ctx);
 // Small batches: logits, top-k, gate weights and bucket tables in one launch.
 constexpr int kRouteSmallMaxT = 32;
 cudaError_t launch_route_small(const LayerDims& L, const float* router_w, const float* router_bias, const uint16_t* x,

@@ -85,6 +85,7 @@ struct moe_layer {
     int64_t prefill_min_tokens = 128;    // batches at least this large take the grouped-GEMM path
     int t1_mode = 0;                     // T = 1: 2 single launch, 1 single-token kernels, 0 general
     bool fused_ok = false;               // the single-launch path is usable for this layer
+    bool union_mma = true;               // small batches: the tensor-core union kernels when they fit
     bool ragged = false;                 // some routed expert lives outside the contiguous [E] arrays
 };
 
@@ -280,6 +281,7 @@ moe_status moe_layer_create(const moe_config* cfg, const moe_weights* w, moe_lay
     if (e == cudaSuccess) e = qe::prepare_router(L->dims);
     if (e == cudaSuccess) e = qe::prepare_bucket(L->dims);
     if (e == cudaSuccess) e = qe::prepare_decode(L->dims);
+    if (e == cudaSuccess) e = qe::prepare_decode_mma();
     if (e == cudaSuccess) e = qe::prepare_decode_fused(L->dims, L->num_sms, &L->fused_ok);
     const bool gemm = qe::prefill_supported(L->dims);
     if (e == cudaSuccess && gemm) e = qe::prepare_prefill(L->dims);
@@ -378,7 +380,9 @@ moe_status moe_forward(moe_layer* L, const uint16_t* x, int32_t T, void* out, mo
         } else if (T == 1 && L->t1_mode >= 1 && !variant) {
             e = qe::launch_decode_t1(L->dims, L->w, x, ws, out, L->num_sms, ctx);
         } else {
-            e = qe::launch_decode_experts(L->dims, L->w, x, T, ws, L->num_sms, ctx);
+            e = L->union_mma && qe::decode_mma_ok(L->dims, T)
+                    ? qe::launch_decode_mma(L->dims, L->w, x, T, ws, L->num_sms, ctx)
+                    : qe::launch_decode_experts(L->dims, L->w, x, T, ws, L->num_sms, ctx);
             if (e == cudaSuccess) e = qe::launch_combine(L->dims, T, ws, out, ctx);
         }
     }
@@ -494,6 +498,10 @@ moe_status moe_layer_set_option(moe_layer* L, int32_t option, int64_t value) {
             if (value < 0 || value > 1000000) return MOE_ERR_INVALID_ARG;
             L->dims.ropts.top_p = (double)value * 1e-6;
             return MOE_OK;
+        case MOE_OPT_UNION_TENSOR_CORES:
+            if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+            L->union_mma = value != 0;
+            return MOE_OK;
         default:
             return MOE_ERR_INVALID_ARG;
     }
@@ -537,6 +545,7 @@ moe_status moe_layer_get_option(const moe_layer* L, int32_t option, int64_t* val
             *value = L->dims.ropts.n_group + ((int64_t)L->dims.ropts.topk_group << 16);
             return MOE_OK;
         case MOE_OPT_ROUTER_TOP_P: *value = (int64_t)(L->dims.ropts.top_p * 1e6 + 0.5); return MOE_OK;
+        case MOE_OPT_UNION_TENSOR_CORES: *value = L->union_mma ? 1 : 0; return MOE_OK;
         default: return MOE_ERR_INVALID_ARG;
     }
 }

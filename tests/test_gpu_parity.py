@@ -206,9 +206,9 @@ def test_glm_batch_union_reads_each_expert_once_per_call(glm):
     x = glm["x32"]
     layer = glm["layer"]
     out_b = run_forward(layer, x)
-    for mode, tol in ((0, 1e-5), (1, 1e-4), (2, 1e-4)):
-        # the same kernels give nearly the same sums; the single-token kernels add in another order,
-        # and an fp16 rounding of h can flip, so their bound is looser (still far inside the spec)
+    for mode, tol in ((0, 1e-4), (1, 1e-4), (2, 1e-4)):
+        # every T = 1 path adds the same products in another order than the batch's tensor-core
+        # kernels, and an fp16 rounding of h can flip, so the bound is 1e-4 (far inside the spec)
         assert layer.set_single_token_mode(mode) == mode
         for i in (0, 7, 31):
             out_1 = run_forward(layer, x[i:i + 1])
