@@ -413,17 +413,17 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
     __shared__ __align__(8) uint64_t s_xbar;              // x -> shared memory
     __shared__ __align__(8) uint64_t s_rbar;              // the router pieces -> shared memory
     __shared__ float ys[kFzMaxSlots][kFzRowsMax];
-    __shared__ int s_e[kFzMaxSlots];                       // routed experts, ascending
+    // the routed slots are the chosen experts in rank order
     __shared__ const uint8_t* s_gu[kFzMaxSlots];           // their weights (the layer's pointer table)
     __shared__ const float* s_gus[kFzMaxSlots];
     __shared__ const uint8_t* s_dn[kFzMaxSlots];
     __shared__ const float* s_dns[kFzMaxSlots];
-    __shared__ float s_w[kFzMaxSlots];                     // their gate weights
+    __shared__ float s_w[kFzMaxSlots];                     // their gate weights (set during phase C)
+    __shared__ int s_asc[kFzMaxSlots];                     // slot of the p-th smallest chosen expert
     __shared__ int sel_e[kFzMaxSlots];                     // rank order
     __shared__ int cand_e[kFzMaxPer * kFzMaxSlots];       // selection candidates, k per warp
     __shared__ uint2 cand_k[kFzMaxPer * kFzMaxSlots];     // and their keys
     __shared__ double sel_l[kFzMaxSlots];
-    __shared__ const void* sel_p[kFzMaxSlots][4];          // their weight pointers, rank order
     __shared__ unsigned long long s_base;                 // arrivals before this launch
     __shared__ int s_ok;
 
@@ -707,11 +707,11 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
     double* lgs = reinterpret_cast<double*>(keys + E);
     if (tid == 0) {
         const bool bok = wait_arrivals(a.bar, s_base + (unsigned long long)G);
-        if (bok) {
+        if (!bok) {
+            latch_status(a.status, MOE_ERR_TIMEOUT);
+        } else {
             bar_expect_tx(saddr(&s_rbar), rbytes);
             bulk_g2s(rings_s, a.rpart, rbytes, saddr(&s_rbar));
-        } else {
-            latch_status(a.status, MOE_ERR_TIMEOUT);
         }
         s_ok = bok;
     }
@@ -779,41 +779,21 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
                 if (rank < k) {
                     sel_e[rank] = e;
                     sel_l[rank] = lgs[e];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) sel_p[rank][i] = pw[i];
+                    s_gu[rank] = static_cast<const uint8_t*>(pw[0]);
+                    s_gus[rank] = static_cast<const float*>(pw[1]);
+                    s_dn[rank] = static_cast<const uint8_t*>(pw[2]);
+                    s_dns[rank] = static_cast<const float*>(pw[3]);
                 }
             }
         }
         __syncthreads();
         stamp(13);
-        if (sel && warp == 0) {
-            const TopkPick pk = topk_finish(lane < k ? sel_e[lane] : -1, lane < k ? sel_l[lane] : 0.0, k, a.router,
-                                            a.scaling, lane);
-            if (lane < k) {
-                s_e[pk.pos] = pk.e;
-                s_w[pk.pos] = pk.w;
-                s_gu[pk.pos] = static_cast<const uint8_t*>(sel_p[lane][0]);     // rank lane is expert pk.e
-                s_gus[pk.pos] = static_cast<const float*>(sel_p[lane][1]);
-                s_dn[pk.pos] = static_cast<const uint8_t*>(sel_p[lane][2]);
-                s_dns[pk.pos] = static_cast<const float*>(sel_p[lane][3]);
-                if (blockIdx.x == 0) {
-                    a.idx[lane] = pk.e;
-                    a.wts[lane] = pk.w;
-                    a.asc[pk.pos] = lane;
-                    a.ulist[pk.pos] = pk.e;
-                }
-            }
-            if (blockIdx.x == 0 && lane == 0) {
-                *a.n_unique = k;
-                *a.xsum = xs * (double)exp2i(-sig);
-            }
-        }
     }
     stamp(14);
     // the keys were written through the generic proxy; TMA writes into the same bytes come next
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     stamp(15);
-    __syncthreads();              // s_e, s_w set; the rings may be used again
+    __syncthreads();              // the slots' pointers are set; the rings may be used again
     stamp(6);
     const bool routed = sel;
 
@@ -838,6 +818,28 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
     }
     if (ok && routed) {
         limit = my_tasks + n_dn;
+        if (warp == 0) {
+            // the gate weights are needed only by the combine: warp 0 computes them here, with its
+            // first routed rows already in flight, instead of on the way into this phase
+            if (lane == 0)
+                while (issued < limit && issued < q + nst) issue(issued++);
+            const TopkPick pk = topk_finish(lane < k ? sel_e[lane] : -1, lane < k ? sel_l[lane] : 0.0, k, a.router,
+                                            a.scaling, lane);
+            if (lane < k) {
+                s_w[lane] = pk.w;
+                s_asc[pk.pos] = lane;
+                if (blockIdx.x == 0) {
+                    a.idx[lane] = pk.e;
+                    a.wts[lane] = pk.w;
+                    a.asc[pk.pos] = lane;
+                    a.ulist[pk.pos] = pk.e;
+                }
+            }
+            if (blockIdx.x == 0 && lane == 0) {
+                *a.n_unique = k;
+                *a.xsum = xs * (double)exp2i(-sig);
+            }
+        }
         for (; q < my_tasks; ++q) {
             if (lane == 0)
                 while (issued < limit && issued < q + nst) issue(issued++);
@@ -957,7 +959,10 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
     if (s_ok) {
         for (int i = tid; i < rj; i += blockDim.x) {
             float o = 0.0f;
-            for (int u = 0; u < k; ++u) o = fmaf(s_w[u], ys[u][i], o);
+            for (int p = 0; p < k; ++p) {              // ascending expert order
+                const int u = s_asc[p];
+                o = fmaf(s_w[u], ys[u][i], o);
+            }
             if (a.S) o += ys[k][i];
             if (a.out_bf16)
                 static_cast<__nv_bfloat16*>(a.out)[j0 + i] = __float2bfloat16_rn(o);
