@@ -24,11 +24,15 @@
 // in that order and the GEMM-1 epilogue writes h in that order.  A dot product does not depend
 // on the order of its terms.
 //
-// Roles (608 threads, one CTA per SM, persistent over tiles):
+// Roles (640 threads, one CTA per SM, persistent over tiles):
 //   warp 0     TMA producer of the packed A rows                 smem ring of 128 KB (16 or 32 stages)
 //   warp 18    TMA producer of the B tiles (a box of 16, 32, 64 smem ring of kBStages
 //              or 128 rows: the group's tokens rounded up)
-//   warp 1     TMEM allocator and MMA issuer                      TMEM A ring of kAStages
+//   warp 1     TMEM allocator and MMA issuer 0                    TMEM A ring of kAStages
+//   warp 19    the second MMA issuer: GEMM-1 issues the gate rows' MMAs from warp 1 and the up
+//              rows' from warp 19, each into its own accumulator (one issuing thread alone is a
+//              bottleneck: a tcgen05.mma adding into the result of the one before waits for
+//              it); GEMM-2 issues from warp 1 alone and leaves warp 19 idle
 //   warps 2-17 converters (A rows -> TMEM), then the epilogue    thread <-> TMEM lane; four sets
 //              of four (one warp per TMEM lane quarter each) take every fourth K step, so a
 //              set has four MMA steps to hide its TMEM store, and every fourth 16-column block
@@ -62,7 +66,8 @@ constexpr int kAStages = 4;                           // converted A tiles in TM
 constexpr int kConvSets = 4;                          // converter warp sets, one K step in kConvSets each
 constexpr int kConvWarps = 4 * kConvSets;             // one warp per TMEM lane quarter per set
 constexpr int kBWarp = 2 + kConvWarps;                // the B producer
-constexpr int kGemmThreads = (kBWarp + 1) * 32;
+constexpr int kMaxIssuers = 2;                        // MMA-issuing warps: 1 and kBWarp + 1
+constexpr int kGemmThreads = (kBWarp + kMaxIssuers) * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kPackedTile = BM * BK / 2;         // 4 KB of packed int4 per 128 x 64 tile
 constexpr uint32_t kBTile = BN * BK * 2;              // 16 KB of bf16 / fp16
@@ -294,6 +299,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             const __grid_constant__ CUtensorMap tmB64, const __grid_constant__ CUtensorMap tmB128,
             const GemmArgs args) {
     constexpr int NA = GATED ? 2 : 1;                     // A tiles per stage
+    // MMA issuers.  A tcgen05.mma waits for the one before it from the same thread when both add
+    // into one accumulator, and one thread issues no faster than about one per 36 ns however
+    // independent its MMAs; several issuing warps, each with its own accumulator, share the
+    // tensor pipe instead.  GEMM-1: one warp for the gate rows, one for the up rows (measured
+    // 7 % faster than one warp for both).  GEMM-2 keeps one issuer: three warps dealing its K
+    // steps into three accumulators measured 37 % slower (0.58 against 0.38 us per K step).
+    constexpr int NI = GATED ? 2 : 1;
     // The packed weights stream from HBM and need many bytes in flight; B comes from L2.  So A and
     // B have rings of their own, A's much deeper.
     constexpr int kSA = (int)(kASmBytes / (NA * kPackedTile));   // A stages: 16 (gate/up) or 32
@@ -328,15 +340,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         }
         for (int s = 0; s < kBStages; ++s) {
             mbar_init(bfull_bar(s), 1);
-            mbar_init(bempty_bar(s), 1);
+            mbar_init(bempty_bar(s), NI);
         }
         for (int s = 0; s < kAStages; ++s) {
             mbar_init(afull_bar(s), 4);
-            mbar_init(aempty_bar(s), 1);
+            mbar_init(aempty_bar(s), NI);
         }
-        mbar_init(accfull_bar, 1);
+        mbar_init(accfull_bar, NI);
         mbar_init(accempty_bar, kConvWarps);
-        mbar_init(final_bar, 1);
+        mbar_init(final_bar, NI);
         abort_flag = 0;
         issued_sh = 0;
         b_issued_sh = 0;
@@ -353,9 +365,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
-    // TMEM columns: accumulators [0, 128) (and [128, 256) for the up rows), then the A ring.
-    const uint32_t acc0 = tmem, acc1 = tmem + BN;
-    const uint32_t a_ring = tmem + (GATED ? 2 * BN : BN);
+    // TMEM columns: the accumulators (GEMM-1: gate [0, 128), up [128, 256); GEMM-2: one per
+    // issuer), then the A ring.
+    const uint32_t acc0 = tmem, acc1 = tmem + BN, acc2 = tmem + 2 * BN;
+    const uint32_t a_ring = tmem + (GATED ? 2 * BN : NI * BN);
     constexpr uint32_t kAStageCols = NA * (BK / 2);       // 32 columns per 128 x 64 A tile
 
     const int nr = args.n_groups[0], ns = args.n_groups[1];
@@ -383,8 +396,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             }
             issued_sh = ks;
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || (warp > kBWarp && warp - kBWarp < NI)) {
+        // ------------------------------------------------------------------ MMA issuers
+        const int ii = warp == 1 ? 0 : warp - kBWarp;      // issuer index
+        const uint32_t my_acc = tmem + (uint32_t)ii * BN;
         if (lane == 0) {
             int ks = 0, tc = 0;
             bool ok = true;
@@ -403,16 +418,19 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     const uint32_t a0 = a_ring + sa * kAStageCols;
 #pragma unroll
                     for (int j = 0; j < BK / 16; ++j) {
-                        const uint32_t acc = (kk | j) != 0;
-                        mma_f16(acc0, a0 + 8 * j, bdesc + 2 * j, idesc, acc);
-                        if (GATED) mma_f16(acc1, a0 + BK / 2 + 8 * j, bdesc + 2 * j, idesc, acc);
+                        if (GATED) {               // issuer 0: the gate rows, issuer 1: the up rows
+                            mma_f16(my_acc, a0 + (uint32_t)ii * (BK / 2) + 8 * j, bdesc + 2 * j, idesc, (kk | j) != 0);
+                        } else {
+                            const int u = (BK / 16) * kk + j;          // the tile's u-th MMA
+                            if (u % NI == ii) mma_f16(my_acc, a0 + 8 * j, bdesc + 2 * j, idesc, u >= NI);
+                        }
                     }
                     mma_commit(bempty_bar(s));
                     mma_commit(aempty_bar(sa));
                 }
                 if (ok) mma_commit(accfull_bar);
             }
-            b_consumed_sh = ks;
+            if (ii == 0) b_consumed_sh = ks;
             // drain: every MMA issued so far completes before TMEM is released
             mma_commit(final_bar);
             wait_bar_drain(final_bar, 0, lim);
@@ -438,6 +456,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             b_issued_sh = ks;
         }
         __syncwarp();
+    } else if (warp > kBWarp) {
+        // an issuer warp this GEMM does not use: nothing to do
     } else {
         // ------------------------------------------------------------------ converters + epilogue
         const int q = warp & 3;                            // TMEM lane quarter of this warp
@@ -492,9 +512,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             const float s0 = __ldg(tl.sc0 + r);
             const float s1 = GATED ? __ldg(tl.sc1 + r) : 0.0f;
             for (int c0 = 16 * set; c0 < nmma; c0 += 16 * kConvSets) {
-                uint32_t v0[16], v1[16];
+                uint32_t v0[16], v1[16], v2[16];
                 tmem_ld16(acc0 + c0 + lane_off, v0);
-                if (GATED) tmem_ld16(acc1 + c0 + lane_off, v1);
+                if (GATED || NI > 1) tmem_ld16(acc1 + c0 + lane_off, v1);
+                if (!GATED && NI > 2) tmem_ld16(acc2 + c0 + lane_off, v2);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
@@ -510,8 +531,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                             static_cast<uint16_t*>(args.out)[(size_t)(tl.slot0 + n) * args.ld_out + kperm_pos(tl.m0 + r)] =
                                 __half_as_ushort(hh);
                         } else {
-                            static_cast<float*>(args.out)[(size_t)(tl.slot0 + n) * args.ld_out + tl.m0 + r] =
-                                s0 * __uint_as_float(v0[i]);
+                            float acc = __uint_as_float(v0[i]);
+                            if (NI > 1) acc += __uint_as_float(v1[i]);
+                            if (NI > 2) acc += __uint_as_float(v2[i]);
+                            static_cast<float*>(args.out)[(size_t)(tl.slot0 + n) * args.ld_out + tl.m0 + r] = s0 * acc;
                         }
                     }
                 }
