@@ -122,6 +122,7 @@ struct Workspace {
     const void** etab;
     double* rpart;         // [E][d / 1024]: pieces of the router logits
     double* rsplit;        // partial logits and sums of x of the K-sliced router GEMM
+    double* keys;          // [T][E] selection keys (small-batch router)
     size_t rsplit_n;       // its length in doubles (0: none)
     unsigned long long* gbar;  // [1]: grid-barrier arrivals (only grows)
     unsigned long long* trace; // [kTraceCtas][kTraceStamps]: phase timestamps of that path

@@ -135,6 +135,7 @@ size_t carve(const moe_config& c, size_t max_groups, char* base, qe::Workspace* 
     };
     qe::Workspace w{};
     w.logits = (double*)take(sizeof(double) * T * E);
+    w.keys = (double*)take(sizeof(double) * std::min(T, (size_t)qe::kRouteSmallMaxT) * E);
     w.rsplit_n = qe::router_split_doubles((int)E, (int)T);
     w.rsplit = w.rsplit_n ? (double*)take(sizeof(double) * w.rsplit_n) : nullptr;
     w.idx = (int32_t*)take(sizeof(int32_t) * T * k);

@@ -215,20 +215,19 @@ constexpr int kSmallThreads = 256;
 constexpr int kSmallMaxT = 32;
 constexpr int kSmallMaxE = 1024;
 
-// Selection for one token whose logits other blocks wrote (read through L2).
+// Selection for one token whose logits and keys other blocks wrote (read through L2).
 template <int MAXPER>
-__device__ void warp_select(const double* __restrict__ lg, const float* __restrict__ bias, int E, int k, int router,
+__device__ void warp_select(const double* __restrict__ lg, const double* __restrict__ ky, int E, int k, int router,
                             float scaling, int lane, int32_t* idx_out, float* w_out, int32_t* asc_out,
                             const RouterOpts& opts) {
-    double l[MAXPER];
+    double l[MAXPER], key[MAXPER];
 #pragma unroll
     for (int m = 0; m < MAXPER; ++m) {
         const int e = lane + kWarp * m;
         l[m] = e < E ? __ldcg(lg + e) : 0.0;
+        key[m] = e < E ? __ldcg(ky + e) : -INFINITY;
     }
-    float bv[MAXPER];
-    load_bias<MAXPER>(bias, E, lane, bv);
-    const TopkPick p = warp_topk<MAXPER>(l, bv, E, k, router, scaling, lane, opts);
+    const TopkPick p = warp_topk_keys<MAXPER>(key, l, E, k, router, scaling, lane, opts);
     if (lane < k) {
         idx_out[lane] = p.e;
         w_out[lane] = p.w;
@@ -243,7 +242,8 @@ route_small_kernel(const float* __restrict__ wr, const float* __restrict__ bias,
                    double* __restrict__ xsum, int32_t* __restrict__ idx, float* __restrict__ wts,
                    int32_t* __restrict__ asc, int32_t* __restrict__ cnt, int32_t* __restrict__ off,
                    int32_t* __restrict__ perm, int32_t* __restrict__ slot_of, int32_t* __restrict__ ulist,
-                   int32_t* __restrict__ n_unique, unsigned int* __restrict__ counter, const RouterOpts opts) {
+                   int32_t* __restrict__ n_unique, unsigned int* __restrict__ counter, const RouterOpts opts,
+                   double* __restrict__ keys) {
     constexpr int TT = MAXC > 8 ? 1 : MAXPER > 8 ? 2 : 4;  // tokens per pass (within the register budget)
     __shared__ double red[kSmallThreads / kWarp][kSmallMaxT];
     __shared__ double redx[kSmallThreads / kWarp][2];
@@ -315,6 +315,8 @@ route_small_kernel(const float* __restrict__ wr, const float* __restrict__ bias,
         double s = 0.0;
         for (int w = 0; w < kSmallThreads / kWarp; ++w) s += red[w][tid];
         logits[(size_t)tid * E + e] = s;
+        // the selection key here too, so the selecting block needs no exponentials of its own
+        keys[(size_t)tid * E + e] = topk_key(s, bias ? bias[e] : 0.0f, router);
     }
     // at most one x sum per block while T <= E; more only for tiny E (then sum them again here)
     if (n_sums == 1 && tid == 0) {
@@ -344,7 +346,7 @@ route_small_kernel(const float* __restrict__ wr, const float* __restrict__ bias,
     if (!am_last) return;
     __threadfence();
     for (int t = warp; t < T; t += kSmallThreads / kWarp)
-        warp_select<MAXPER>(logits + (size_t)t * E, bias, E, k, router, scaling, lane, idx + (size_t)t * k,
+        warp_select<MAXPER>(logits + (size_t)t * E, keys + (size_t)t * E, E, k, router, scaling, lane, idx + (size_t)t * k,
                             wts + (size_t)t * k, asc + (size_t)t * k, opts);
     for (int i = tid; i < E; i += kSmallThreads) s_cnt[i] = 0;
     __syncthreads();
@@ -411,7 +413,7 @@ cudaError_t launch_route_small(const LayerDims& L, const float* router_w, const 
     QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,                                                                      \
               (route_small_kernel<MAXPER, MAXC><<<L.E, kSmallThreads, 0, ctx.s>>>(                              \
                   router_w, bias, x, T, L.d, L.E, L.k, L.router, L.scaling, ws.logits, ws.xsum, ws.idx, ws.wts,  \
-                  ws.asc, ws.cnt, ws.off, ws.perm, ws.slot_of, ws.ulist, ws.n_unique, counter, L.ropts)))
+                  ws.asc, ws.cnt, ws.off, ws.perm, ws.slot_of, ws.ulist, ws.n_unique, counter, L.ropts, ws.keys)))
     if (L.E <= 32) {
         if (narrow) QE_ROUTE_SMALL(1, 6); else QE_ROUTE_SMALL(1, 14);
     } else if (L.E <= 256) {

@@ -122,25 +122,18 @@ __device__ __forceinline__ double topk_key(double l, float bias, int router) {
     return isnan(kv) ? -INFINITY : kv;
 }
 
-// lg[m] is the logit of expert lane + 32 m and bv[m] its selection bias (0 without one); entries
+// key[m] and lg[m] are the selection key (topk_key) and the logit of expert lane + 32 m; entries
 // with an index >= E are ignored.  Every lane of the warp calls it; lanes >= k get e = -1.
 template <int MAXPER>
-__device__ __forceinline__ TopkPick warp_topk(const double (&lg)[MAXPER], const float (&bv)[MAXPER], int E, int k,
-                                              int router, float scaling, int lane,
-                                              const RouterOpts& opts = RouterOpts()) {
-    double key[MAXPER];
+__device__ __forceinline__ TopkPick warp_topk_keys(double (&key)[MAXPER], const double (&lg)[MAXPER], int E, int k,
+                                                   int router, float scaling, int lane, const RouterOpts& opts) {
     uint32_t taken = 0;
 #pragma unroll
-    for (int m = 0; m < MAXPER; ++m) {
-        const int e = lane + kWarp * m;
-        double kv = -INFINITY;
-        if (e < E) {
-            kv = topk_key(lg[m], bv[m], router);
-        } else {
+    for (int m = 0; m < MAXPER; ++m)
+        if (lane + kWarp * m >= E) {
             taken |= 1u << m;
+            key[m] = -INFINITY;
         }
-        key[m] = kv;
-    }
     if (opts.n_group > 1) limit_groups<MAXPER>(key, E, opts, lane, taken);
     int my_e = -1;
     double my_l = 0.0;
@@ -169,6 +162,18 @@ __device__ __forceinline__ TopkPick warp_topk(const double (&lg)[MAXPER], const 
         if (lane == r) { my_e = bi; my_l = wl; }
     }
     return topk_finish(my_e, my_l, k, router, scaling, lane, opts.top_p);
+}
+
+// The same from the logits: lg[m] is the logit of expert lane + 32 m and bv[m] its selection bias
+// (0 without one).
+template <int MAXPER>
+__device__ __forceinline__ TopkPick warp_topk(const double (&lg)[MAXPER], const float (&bv)[MAXPER], int E, int k,
+                                              int router, float scaling, int lane,
+                                              const RouterOpts& opts = RouterOpts()) {
+    double key[MAXPER];
+#pragma unroll
+    for (int m = 0; m < MAXPER; ++m) key[m] = lane + kWarp * m < E ? topk_key(lg[m], bv[m], router) : -INFINITY;
+    return warp_topk_keys<MAXPER>(key, lg, E, k, router, scaling, lane, opts);
 }
 
 // The biases of experts lane + 32 m (0 where there is none).
