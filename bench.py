@@ -451,9 +451,9 @@ def kernel_work(cfg, T, n_unique):
     # the single-token kernel adds the slots itself and writes the output; the others write y per slot
     dn = dn_w + (T * cfg.d * 4 if T == 1 else slots * cfg.d * 4)
     mac = T * cfg.k * cfg.d * cfg.f + T * S * cfg.d * cfg.f_shared
-    # the single launch (T = 1): router matrix and bias, then gu (x, gate/up rows, h written) and
-    # dn_w (down rows, h read back), and the output
-    fused = cfg.E * cfg.d * 4 + cfg.E * 4 + gu + dn_w + cfg.d * 4
+    # the single launch (T = 1 or 2): router matrix and bias, then gu (x, gate/up rows, h written)
+    # and dn_w (down rows, h read back), and the output
+    fused = cfg.E * cfg.d * 4 + cfg.E * 4 + gu + dn_w + T * cfg.d * 4
     # router kernels: the fp32 router matrix and x read, fp64 logits written
     router = cfg.E * cfg.d * 4 + T * cfg.d * 2 + T * cfg.E * 8
     return {"gateup": ("hbm", gu), "down": ("hbm", dn), "gemm_gateup": ("tensor", 4 * mac),

@@ -241,7 +241,11 @@ void moe_layer_destroy(moe_layer *layer);
  *                               one; get returns the mode in use.  Same results within tolerance.
  *                               Mode 2 is a cooperative launch of one CTA per SM: it starts when
  *                               every SM can take its CTA, so kernels of other streams running at
- *                               the same time delay it.
+ *                               the same time delay it.  In mode 2 a T = 2 batch with int4
+ *                               weights and ceil(d / SMs) <= 48 (and 16 warps' rings in shared
+ *                               memory where E > 224) also runs as one launch: each shared-expert
+ *                               row is read once for both tokens; mode 1 or 0 sends T = 2 to the
+ *                               batch kernels.  Such a launch does not write MOE_DEBUG_ULIST.
  */
 /*   MOE_OPT_PROGRAMMATIC_LAUNCH  1 (default): chained kernels of the single-token path start
  *                               early with programmatic dependent launch and wait on the device
@@ -295,12 +299,13 @@ moe_status moe_layer_get_option(const moe_layer *layer, int32_t option, int64_t 
  * kernels ran (see each item).  `bytes` is the size of `dst`; at most the item's size is copied.
  *   MOE_DEBUG_H      h = silu(g) * u, fp16 [slots][fmax] (slot = routed slot, then T*k + t for the
  *                    shared expert; K order of the grouped-GEMM path is permuted in groups of 8;
- *                    the single-launch T = 1 path stores 8-value chunk c of row [k+1][f] at
- *                    position (c % (f/256)) * 32 + c / (f/256))
+ *                    the single-launch path (T = 1 or 2) has rows [T*(k+1)][f], routed slot
+ *                    t*k + rank, and stores 8-value chunk c of a row at position
+ *                    (c % (f/256)) * 32 + c / (f/256))
  *   MOE_DEBUG_Y      y per slot, fp32 [slots][d] (not written by the single-token kernels)
  *   MOE_DEBUG_IDX / MOE_DEBUG_W / MOE_DEBUG_ASC   int32 / fp32 / int32 [T][k]
  *   MOE_DEBUG_ULIST  int32 [E] unique chosen experts, ascending;  MOE_DEBUG_CNT int32 [E]
- *                    (CNT is not written by the single-launch T = 1 path)
+ *                    (CNT is not written by the single-launch path, ULIST not by it at T = 2)
  *   MOE_DEBUG_XSUM   fp64 [T]
  *   MOE_DEBUG_TRACE  uint64 [SMs][16]: for the single-launch T = 1 path, the %globaltimer value (ns)
  *                    at which each CTA passed its phase boundaries: 0 start, 1 x rearranged

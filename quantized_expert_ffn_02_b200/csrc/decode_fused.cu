@@ -76,11 +76,22 @@ constexpr int kFzMaxThreads = kFzMaxWarps * kWarp;
 constexpr int kFzStages = 2;
 constexpr int kFzMaxSlots = 10;       // k routed experts + the shared one
 constexpr int kFzMaxPer = 8;          // experts per lane in the selection: E <= 256
-constexpr int kFzRowsMax = 64;        // output rows per CTA
+constexpr int kFzRowsMax = 64;        // output rows per CTA (one token; 48 for two)
 constexpr int kFzDnRowsMax = 8;       // down rows per stage
 constexpr int kFzScRegs = 3;          // down-row scales per lane: up to 96 (slot, row) items per warp
 constexpr size_t kSmemLimit = 227 * 1024;
-constexpr int kStaticReserve = 6144;  // static shared memory of the kernel, rounded up
+// output rows per CTA and the kernel's static shared memory (rounded up), for nt tokens
+constexpr int fz_rows_max(int nt) { return nt == 1 ? kFzRowsMax : 48; }
+constexpr size_t fz_static_reserve(int nt) { return nt == 1 ? 6144 : 8192; }
+// the element i of a per-token register array, without a local-memory copy for a runtime index
+template <int N, typename V>
+__device__ __forceinline__ V pick_tok(const V (&v)[N], int i) {
+    V r = v[0];
+#pragma unroll
+    for (int j = 1; j < N; ++j)
+        if (i == j) r = v[j];
+    return r;
+}
 
 struct FusedArgs {
     const float* router_w;            // [E][d] fp32
@@ -402,8 +413,11 @@ __device__ __forceinline__ void hilo_from_f16(uint4 v, uint32_t* p, float& sum) 
 }
 
 // WK: MOE_W_INT4_ROWSCALE or MOE_W_BF16.  NDK: 16-byte groups of a gate/up row per lane (d / 1024
-// for int4, d / 256 for bf16); NF: the same for a down row (f / 1024, f / 256).
-template <int WK, int NDK, int NF>
+// for int4, d / 256 for bf16); NF: the same for a down row (f / 1024, f / 256).  NT: tokens (1 or
+// 2).  With two tokens the CTA's two halves select for one token each, the routed slots are
+// token-major (t k + rank), the shared expert's slots follow (NT k + t), and each shared row pair
+// is applied to both tokens from one read.
+template <int WK, int NDK, int NF, int NT>
 __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const FusedArgs a) {
     // [x~ lane blocks][kFzStages][warps][stage]: stage s of every warp is one region; x (plain
     // bf16, 2d bytes) lands in the last stage's region during phase A
@@ -412,18 +426,18 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
     __shared__ int4 s_desc[kFzMaxWarps][kFzStages];       // gate/up stage: slot, row, scale slots
     __shared__ __align__(8) uint64_t s_xbar;              // x -> shared memory
     __shared__ __align__(8) uint64_t s_rbar;              // the router pieces -> shared memory
-    __shared__ float ys[kFzMaxSlots][kFzRowsMax];
-    // the routed slots are the chosen experts in rank order
-    __shared__ const uint8_t* s_gu[kFzMaxSlots];           // their weights (the layer's pointer table)
-    __shared__ const float* s_gus[kFzMaxSlots];
-    __shared__ const uint8_t* s_dn[kFzMaxSlots];
-    __shared__ const float* s_dns[kFzMaxSlots];
-    __shared__ float s_w[kFzMaxSlots];                     // their gate weights (set during phase C)
-    __shared__ int s_asc[kFzMaxSlots];                     // slot of the p-th smallest chosen expert
-    __shared__ int sel_e[kFzMaxSlots];                     // rank order
-    __shared__ int cand_e[kFzMaxPer * kFzMaxSlots];       // selection candidates, k per warp
-    __shared__ uint2 cand_k[kFzMaxPer * kFzMaxSlots];     // and their keys
-    __shared__ double sel_l[kFzMaxSlots];
+    __shared__ float ys[NT * kFzMaxSlots][fz_rows_max(NT)];
+    // the routed slots are the chosen experts in rank order (token-major)
+    __shared__ const uint8_t* s_gu[NT * kFzMaxSlots];      // their weights (the layer's pointer table)
+    __shared__ const float* s_gus[NT * kFzMaxSlots];
+    __shared__ const uint8_t* s_dn[NT * kFzMaxSlots];
+    __shared__ const float* s_dns[NT * kFzMaxSlots];
+    __shared__ float s_w[NT * kFzMaxSlots];                // their gate weights (set during phase C)
+    __shared__ int s_asc[NT * kFzMaxSlots];                // slot of the p-th smallest chosen expert
+    __shared__ int sel_e[NT * kFzMaxSlots];                // rank order
+    __shared__ int cand_e[NT][kFzMaxPer * kFzMaxSlots];   // selection candidates, k per warp
+    __shared__ uint2 cand_k[NT][kFzMaxPer * kFzMaxSlots]; // and their keys
+    __shared__ double sel_l[NT * kFzMaxSlots];
     __shared__ unsigned long long s_base;                 // arrivals before this launch
     __shared__ int s_ok;
 
@@ -443,13 +457,14 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
     // 16-byte loads meet no bank conflict
     constexpr uint32_t kLaneBlk = (BF ? 16 : 64) * NDK + 16;
     constexpr uint32_t kXtBytes = (32 * kLaneBlk + 127) / 128 * 128;
-    const uint32_t xt_s = saddr(smem);
-    const uint32_t rings_s = xt_s + kXtBytes;
+    const uint32_t xt_s = saddr(smem);                     // token t's lane blocks at xt_s + t kXtBytes
+    const uint32_t rings_s = xt_s + NT * kXtBytes;
     auto st_s = [&](int s) { return rings_s + ((uint32_t)s * nwc + warp) * stage_bytes; };
-    auto st_g = [&](int s) { return smem + kXtBytes + ((size_t)s * nwc + warp) * stage_bytes; };
-    const uint32_t xraw_s = rings_s + (uint32_t)(nst - 1) * nwc * stage_bytes;
-    const int n_sh = a.S ? f : 0;                          // shared row pairs
-    const int n_tasks = n_sh + k * f;
+    auto st_g = [&](int s) { return smem + NT * kXtBytes + ((size_t)s * nwc + warp) * stage_bytes; };
+    const uint32_t xraw_s = rings_s + (uint32_t)(nst - 1) * nwc * stage_bytes;   // token t at + 2 d t
+    const int n_sh = a.S ? f : 0;                          // shared row pairs (each for every token)
+    const int nrs = NT * k;                                // routed slots
+    const int n_tasks = n_sh + nrs * f;
     auto count_of = [&](int lo, int hi) {                  // my tasks among [lo, hi)
         const int first = lo + ((gw - lo) % nw + nw) % nw; // smallest t >= lo with t == gw (mod nw)
         return first < hi ? (hi - first + nw - 1) / nw : 0;
@@ -459,7 +474,7 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
     // task i of this warp is t = gw + i * nw (shared ones first because gw < nw)
     // this CTA's output rows and the warp's share of the (slot, row) items
     const int j0 = (int)((int64_t)blockIdx.x * d / G), rj = (int)((int64_t)(blockIdx.x + 1) * d / G) - j0;
-    const int nslots = k + a.S;
+    const int nslots = nrs + NT * a.S;
     const int n_items = nslots * rj;
     const int it0 = (int)((int64_t)warp * n_items / nwc), it1 = (int)((int64_t)(warp + 1) * n_items / nwc);
     // the lane's segment (g) and quarter (c): byte offsets within a gate/up row and a down row
@@ -484,8 +499,8 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
     }
     __syncthreads();
     if (tid == 0) {
-        bar_expect_tx(saddr(&s_xbar), 2u * d);
-        bulk_g2s(xraw_s, a.x, 2u * d, saddr(&s_xbar));
+        bar_expect_tx(saddr(&s_xbar), 2u * d * NT);
+        bulk_g2s(xraw_s, a.x, 2u * d * NT, saddr(&s_xbar));
     }
 
     // ---- the ring: use q of this warp goes to stage q % nst
@@ -510,7 +525,7 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
                 rows = a.sh_gate_up + (size_t)t * gu_row;
                 sc = a.sh_gu_scale + t;
                 r = t;
-                slot = k;
+                slot = nrs;                                // the first shared slot
             } else {
                 if (gu_u < 0) {
                     gu_u = (t - n_sh) / f;
@@ -535,7 +550,7 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
             }
         } else {
             const int n = dn_count(dn_it, dn_row);
-            const uint8_t* W = dn_u < k ? s_dn[dn_u] : a.sh_down;
+            const uint8_t* W = dn_u < nrs ? s_dn[dn_u] : a.sh_down;
             bar_expect_tx(bar, (uint32_t)n * dn_row_b);
             bulk_g2s(dst, W + (size_t)(j0 + dn_row) * dn_row_b, (uint32_t)n * dn_row_b, bar);
             dn_it += n;
@@ -579,65 +594,74 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
     // fixed order, so every CTA gets the same value.
     __shared__ float s_redf[kFzMaxWarps];
     __shared__ double s_redd[kFzMaxWarps];
-    int sig = 0;
-    double xs = 0.0;              // sum of x~ = x 2^sigma over the whole row (bf16: of x)
-    if constexpr (BF) {
-        float part = 0.0f;
-        for (int g = tid; g < d / 8; g += blockDim.x) {
-            const uint4 v = lds16(xraw_s + 16u * (uint32_t)g);
-            const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
+    int sig[NT] = {};
+    double xs[NT] = {};           // per token: sum of x~ = x 2^sigma over the whole row (bf16: of x)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) part += __uint_as_float(ws[i] << 16) + __uint_as_float(ws[i] & 0xffff0000u);
-            // group g (8 columns) belongs to lane L = 4 seg + quarter, as its group q
-            const int seg = g / (d / 64), rem = g - seg * (d / 64);
-            const int cq = rem / NDK, q = rem - cq * NDK, L = 4 * seg + cq;
-            int j = q - gu_rot<NDK>(L);
-            if (j < 0) j += NDK;
-            sts16(xt_s + (uint32_t)L * kLaneBlk + (uint32_t)j * 16u, v);
-        }
-        const double pd = warp_sum_d((double)part);
-        if (lane == 0) s_redd[warp] = pd;
-        __syncthreads();
-        for (int w = 0; w < nwc; ++w) xs += s_redd[w];
-    } else {
-        float m = 0.0f;
-        for (int g = tid; g < d / 8; g += blockDim.x) {
-            const uint4 v = lds16(xraw_s + 16u * (uint32_t)g);
-            const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
+    for (int tk = 0; tk < NT; ++tk) {
+        const uint32_t xr = xraw_s + 2u * d * tk;             // token tk's plain x
+        const uint32_t xt = xt_s + kXtBytes * tk;             // and its lane blocks
+        if constexpr (BF) {
+            float part = 0.0f;
+            for (int g = tid; g < d / 8; g += blockDim.x) {
+                const uint4 v = lds16(xr + 16u * (uint32_t)g);
+                const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                m = fmaxf(m, fmaxf(fabsf(__uint_as_float(ws[i] << 16)), fabsf(__uint_as_float(ws[i] & 0xffff0000u))));
-        }
+                for (int i = 0; i < 4; ++i) part += __uint_as_float(ws[i] << 16) + __uint_as_float(ws[i] & 0xffff0000u);
+                // group g (8 columns) belongs to lane L = 4 seg + quarter, as its group q
+                const int seg = g / (d / 64), rem = g - seg * (d / 64);
+                const int cq = rem / NDK, q = rem - cq * NDK, L = 4 * seg + cq;
+                int j = q - gu_rot<NDK>(L);
+                if (j < 0) j += NDK;
+                sts16(xt + (uint32_t)L * kLaneBlk + (uint32_t)j * 16u, v);
+            }
+            const double pd = warp_sum_d((double)part);
+            if (lane == 0) s_redd[warp] = pd;
+            __syncthreads();
+            for (int w = 0; w < nwc; ++w) xs[tk] += s_redd[w];
+        } else {
+            float m = 0.0f;
+            for (int g = tid; g < d / 8; g += blockDim.x) {
+                const uint4 v = lds16(xr + 16u * (uint32_t)g);
+                const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0) s_redf[warp] = m;
-        __syncthreads();
-        m = 0.0f;
-        for (int w = 0; w < nwc; ++w) m = fmaxf(m, s_redf[w]);
-        sig = scale_exp(m);
-        const float s1 = exp2i(sig), s16 = exp2i(sig - 4);
-        float part = 0.0f;
-        for (int g = tid; g < d / 8; g += blockDim.x) {
-            uint32_t pr[4];
-            pairs_from_bf16(lds16(xraw_s + 16u * (uint32_t)g), s1, s16, pr, part);
-            // group g belongs to lane L = 4 seg + quarter, as word w of its group q
-            const int seg = g / (d / 64), rem = g - seg * (d / 64);
-            const int cq = rem / (4 * NDK), rem2 = rem - cq * (4 * NDK);
-            const int q = rem2 >> 2, w = rem2 & 3, L = 4 * seg + cq;
-            int j = q - gu_rot<NDK>(L);
-            if (j < 0) j += NDK;
-            sts16(xt_s + (uint32_t)L * kLaneBlk + (uint32_t)(4 * j + w) * 16u, make_uint4(pr[0], pr[1], pr[2], pr[3]));
+                for (int i = 0; i < 4; ++i)
+                    m = fmaxf(m, fmaxf(fabsf(__uint_as_float(ws[i] << 16)), fabsf(__uint_as_float(ws[i] & 0xffff0000u))));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (lane == 0) s_redf[warp] = m;
+            __syncthreads();
+            m = 0.0f;
+            for (int w = 0; w < nwc; ++w) m = fmaxf(m, s_redf[w]);
+            sig[tk] = scale_exp(m);
+            const float s1 = exp2i(sig[tk]), s16 = exp2i(sig[tk] - 4);
+            float part = 0.0f;
+            for (int g = tid; g < d / 8; g += blockDim.x) {
+                uint32_t pr[4];
+                pairs_from_bf16(lds16(xr + 16u * (uint32_t)g), s1, s16, pr, part);
+                // group g belongs to lane L = 4 seg + quarter, as word w of its group q
+                const int seg = g / (d / 64), rem = g - seg * (d / 64);
+                const int cq = rem / (4 * NDK), rem2 = rem - cq * (4 * NDK);
+                const int q = rem2 >> 2, w = rem2 & 3, L = 4 * seg + cq;
+                int j = q - gu_rot<NDK>(L);
+                if (j < 0) j += NDK;
+                sts16(xt + (uint32_t)L * kLaneBlk + (uint32_t)(4 * j + w) * 16u, make_uint4(pr[0], pr[1], pr[2], pr[3]));
+            }
+            const double pd = warp_sum_d((double)part);
+            if (lane == 0) s_redd[warp] = pd;
+            __syncthreads();
+            for (int w = 0; w < nwc; ++w) xs[tk] += s_redd[w];
         }
-        const double pd = warp_sum_d((double)part);
-        if (lane == 0) s_redd[warp] = pd;
-        __syncthreads();
-        for (int w = 0; w < nwc; ++w) xs += s_redd[w];
+        if (tk + 1 < NT) __syncthreads();                  // s_redf / s_redd are reused
     }
     // router pieces: unit u = (expert u / nch, columns [1024 p, 1024 p + 1024), p = u % nch)
     auto piece = [&](int u, const float4 (&wv)[8]) {
         const int p = u % nch;
-        const double v = warp_sum_d(router_piece(wv, xraw_s + 2048u * p, lane));
-        if (lane == 0) __stcg(a.rpart + u, v);
+#pragma unroll
+        for (int tk = 0; tk < NT; ++tk) {                  // one router row piece, every token
+            const double v = warp_sum_d(router_piece(wv, xraw_s + 2u * d * tk + 2048u * p, lane));
+            if (lane == 0) __stcg(a.rpart + (size_t)tk * n_units + u, v);
+        }
     };
     if (gw < n_units) piece(gw, rw);
     for (int u = gw + nw; u < n_units; u += nw) {
@@ -646,11 +670,17 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
         piece(u, rw);
     }
     stamp(1);
-    const uint32_t xblk = xt_s + (uint32_t)lane * kLaneBlk;   // this lane's operand block
-    const float xoff = 8.0f * (float)xs;                   // 8 sum x~
-    const float xunscale = exp2i(-sig) * 16777216.0f;      // 2^(24 - sigma)
-    // this thread's selection bias
-    const float my_bias = a.bias && tid < E ? a.bias[tid] : 0.0f;
+    const uint32_t xblk = xt_s + (uint32_t)lane * kLaneBlk;   // this lane's operand block (token 0)
+    float xoffs[NT], xunscale[NT];                          // per token: 8 sum x~ 2^-sigma, 2^(24 - sigma)
+#pragma unroll
+    for (int tk = 0; tk < NT; ++tk) {
+        xoffs[tk] = 8.0f * (float)xs[tk] * exp2i(-sig[tk]);
+        xunscale[tk] = exp2i(-sig[tk]) * 16777216.0f;
+    }
+    // selection: the CTA's halves take one token each (NT = 2); thread ltid of half tt holds
+    // expert ltid of token tt
+    const int nwh = nwc / NT, tt = warp / nwh, lw = warp - tt * nwh, ltid = tid - tt * nwh * kWarp;
+    const float my_bias = a.bias && ltid < E ? a.bias[ltid] : 0.0f;
     __syncthreads();                                       // the last stage (x) is free
     if (tid == 0) {                                        // barrier 0: every piece is stored
         const unsigned long long old = arrive(a.bar);
@@ -672,21 +702,37 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
         }
         n_pend = 0;
     };
-    auto gate_up_use = [&](int q, float2 part) {
+    // one gate/up row pair (stage of use q): a routed slot's for its token, a shared one's for
+    // every token (the row pair decoded from the one copy in shared memory)
+    auto gate_up_stage = [&](int q) {
         const int s = q % nst;
         const int4 dsc = s_desc[warp][s];
+        const bool sh = dsc.x >= nrs;
+        const int t0 = sh ? 0 : dsc.x / k;                 // routed slots are token-major
+        const uint32_t ra = st_s(s), rb = ra + gu_row;
+        float2 parts[NT];
+        parts[0] = rows_mma_x<WK, NDK>(ra, rb, gu_lane_off, grot, xblk + kXtBytes * t0, lane);
+#pragma unroll
+        for (int tk = 1; tk < NT; ++tk)
+            if (sh) parts[tk] = rows_mma_x<WK, NDK>(ra, rb, gu_lane_off, grot, xblk + kXtBytes * tk, lane);
         const float* scs = reinterpret_cast<const float*>(st_g(s) + 2 * gu_row);
         const float sg = BF ? 1.0f : scs[dsc.z], su = BF ? 1.0f : scs[dsc.w];
         __syncwarp();                                      // the stage is free again
         if (lane == 0)
             while (issued < limit && issued < q + 1 + nst) issue(issued++);
-        const float ag = warp_sum(part.x), au = warp_sum(part.y);
-        if (lane == n_pend) {
-            p_g = BF ? ag : sg * fmaf(ag, xunscale, -xoff * exp2i(-sig));
-            p_u = BF ? au : su * fmaf(au, xunscale, -xoff * exp2i(-sig));
-            p_h = dsc.x * f + h_pos<f>(dsc.y);
+#pragma unroll
+        for (int tk = 0; tk < NT; ++tk) {
+            if (tk > 0 && !sh) break;
+            const int tok = sh ? tk : t0;
+            const float ag = warp_sum(parts[tk].x), au = warp_sum(parts[tk].y);
+            if (lane == n_pend) {
+                const float xu = pick_tok(xunscale, tok), xo = pick_tok(xoffs, tok);
+                p_g = BF ? ag : sg * fmaf(ag, xu, -xo);
+                p_u = BF ? au : su * fmaf(au, xu, -xo);
+                p_h = (dsc.x + (sh ? tk : 0)) * f + h_pos<f>(dsc.y);
+            }
+            if (++n_pend == kWarp) flush();
         }
-        if (++n_pend == kWarp) flush();
     };
 
     int q = 0;                    // next use to consume
@@ -694,17 +740,17 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
         if (lane == 0)
             while (issued < limit && issued < q + nst) issue(issued++);
         if (!wait_use(q)) { ok = false; break; }
-        gate_up_use(q, rows_mma_x<WK, NDK>(st_s(q % nst), st_s(q % nst) + gu_row, gu_lane_off, grot, xblk, lane));
+        gate_up_stage(q);
     }
 
     // ---- B: selection by the whole CTA once every piece of the logits is stored.  The rings are
     //      idle: the router pieces, then the keys and logits, go to their start.
     __syncthreads();
     stamp(3);
-    const uint32_t rbytes = ((uint32_t)n_units * 8u + 15u) & ~15u;
-    uint8_t* const rings = smem + kXtBytes;                // generic address of rings_s
-    uint2* keys = reinterpret_cast<uint2*>(rings + rbytes);    // keys, order-preserving integers
-    double* lgs = reinterpret_cast<double*>(keys + E);
+    const uint32_t rbytes = ((uint32_t)(NT * n_units) * 8u + 15u) & ~15u;
+    uint8_t* const rings = smem + NT * kXtBytes;           // generic address of rings_s
+    uint2* keys = reinterpret_cast<uint2*>(rings + rbytes);    // [NT][E] keys, order-preserving integers
+    double* lgs = reinterpret_cast<double*>(keys + NT * E);    // [NT][E] logits
     if (tid == 0) {
         const bool bok = wait_arrivals(a.bar, s_base + (unsigned long long)G);
         if (!bok) {
@@ -720,15 +766,15 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
     bool sel = s_ok != 0;
     if (sel) {
         const bool landed = bar_wait(saddr(&s_rbar), 0u);
-        if (landed && tid < E) {
-            const double* rp = reinterpret_cast<const double*>(rings);
+        if (landed && tt < NT && ltid < E) {
+            const double* rp = reinterpret_cast<const double*>(rings) + (size_t)tt * n_units;
             double l = 0.0;
-            for (int p = 0; p < nch; ++p) l += rp[tid * nch + p];
-            lgs[tid] = l;
+            for (int p = 0; p < nch; ++p) l += rp[ltid * nch + p];
+            lgs[tt * E + ltid] = l;
             // key -> unsigned 64-bit integer of the same order (-0 folded into +0; NaN is -inf)
             const long long b = __double_as_longlong(topk_key(l, my_bias, a.router) + 0.0);
             const unsigned long long o = b < 0 ? ~(unsigned long long)b : (unsigned long long)b | (1ull << 63);
-            keys[tid] = make_uint2((uint32_t)(o >> 32), (uint32_t)o);
+            keys[tt * E + ltid] = make_uint2((uint32_t)(o >> 32), (uint32_t)o);
         }
         sel = !__syncthreads_or(!landed);
         if (!sel && tid == 0) latch_status(a.status, MOE_ERR_TIMEOUT);
@@ -741,48 +787,49 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
         auto beats = [](uint2 kj, int j, uint2 ki, int i) {
             return (kj.x > ki.x) | ((kj.x == ki.x) & ((kj.y > ki.y) | ((kj.y == ki.y) & (j < i))));
         };
-        const int nwe = (E + kWarp - 1) / kWarp;           // warps holding experts
-        if (sel && warp < nwe) {
-            const int e = tid;
-            const uint2 mk = e < E ? keys[e] : make_uint2(0u, 0u);   // below every real key
+        const int nwe = (E + kWarp - 1) / kWarp;           // warps holding experts (per half)
+        if (sel && tt < NT && lw < nwe) {
+            const int e = ltid;
+            const uint2 mk = e < E ? keys[tt * E + e] : make_uint2(0u, 0u);   // below every real key
             int rank = 0;
 #pragma unroll 4
             for (int o = 1; o < kWarp; ++o) {
                 const int jl = (lane + o) & (kWarp - 1);
                 const uint2 kj = make_uint2(__shfl_sync(0xffffffffu, mk.x, jl), __shfl_sync(0xffffffffu, mk.y, jl));
-                rank += beats(kj, warp * kWarp + jl, mk, e) ? 1 : 0;
+                rank += beats(kj, lw * kWarp + jl, mk, e) ? 1 : 0;
             }
             if (lane < k) {
-                cand_e[warp * k + lane] = -1;
-                cand_k[warp * k + lane] = make_uint2(0u, 0u);
+                cand_e[tt][lw * k + lane] = -1;
+                cand_k[tt][lw * k + lane] = make_uint2(0u, 0u);
             }
             __syncwarp();
             if (e < E && rank < k) {
-                cand_e[warp * k + rank] = e;
-                cand_k[warp * k + rank] = mk;
+                cand_e[tt][lw * k + rank] = e;
+                cand_k[tt][lw * k + rank] = mk;
             }
         }
         __syncthreads();
         stamp(12);
-        const int nc = nwe * k;                            // candidate slots
-        if (sel && tid < nc) {
-            const int e = cand_e[tid];
+        const int nc = nwe * k;                            // candidate slots per token
+        if (sel && tt < NT && ltid < nc) {
+            const int e = cand_e[tt][ltid];
             if (e >= 0) {
                 // the candidate's weight pointers: loaded while the rank is counted
                 const void* pw[4] = {ex_gate_up(a.etab, E, e), ex_gu_scale(a.etab, E, e), ex_down(a.etab, E, e),
                                      ex_dn_scale(a.etab, E, e)};
-                const uint2 mk = cand_k[tid];
+                const uint2 mk = cand_k[tt][ltid];
                 int rank = 0;
 #pragma unroll 8
                 for (int c = 0; c < nc; ++c)               // empty slots hold key 0, below every real key
-                    rank += beats(cand_k[c], cand_e[c], mk, e) ? 1 : 0;
+                    rank += beats(cand_k[tt][c], cand_e[tt][c], mk, e) ? 1 : 0;
                 if (rank < k) {
-                    sel_e[rank] = e;
-                    sel_l[rank] = lgs[e];
-                    s_gu[rank] = static_cast<const uint8_t*>(pw[0]);
-                    s_gus[rank] = static_cast<const float*>(pw[1]);
-                    s_dn[rank] = static_cast<const uint8_t*>(pw[2]);
-                    s_dns[rank] = static_cast<const float*>(pw[3]);
+                    const int slot = tt * k + rank;
+                    sel_e[slot] = e;
+                    sel_l[slot] = lgs[tt * E + e];
+                    s_gu[slot] = static_cast<const uint8_t*>(pw[0]);
+                    s_gus[slot] = static_cast<const float*>(pw[1]);
+                    s_dn[slot] = static_cast<const uint8_t*>(pw[2]);
+                    s_dns[slot] = static_cast<const float*>(pw[3]);
                 }
             }
         }
@@ -805,7 +852,7 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
         float v = 0.0f;
         if (routed && it < it1) {
             const int u = it / rj, row = it - u * rj;
-            v = BF ? 1.0f : __ldg((u < k ? s_dns[u] : a.sh_dn_scale) + j0 + row);
+            v = BF ? 1.0f : __ldg((u < nrs ? s_dns[u] : a.sh_dn_scale) + j0 + row);
         }
         dsc_r[r] = v;
     }
@@ -818,33 +865,35 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
     }
     if (ok && routed) {
         limit = my_tasks + n_dn;
-        if (warp == 0) {
-            // the gate weights are needed only by the combine: warp 0 computes them here, with its
-            // first routed rows already in flight, instead of on the way into this phase
+        if (lw == 0 && tt < NT) {
+            // the gate weights are needed only by the combine: the first warp of each half
+            // computes its token's here, with its first routed rows already in flight, instead of
+            // on the way into this phase
             if (lane == 0)
                 while (issued < limit && issued < q + nst) issue(issued++);
-            const TopkPick pk = topk_finish(lane < k ? sel_e[lane] : -1, lane < k ? sel_l[lane] : 0.0, k, a.router,
-                                            a.scaling, lane);
+            const int sb = tt * k;                         // the token's first slot
+            const TopkPick pk = topk_finish(lane < k ? sel_e[sb + lane] : -1, lane < k ? sel_l[sb + lane] : 0.0, k,
+                                            a.router, a.scaling, lane);
             if (lane < k) {
-                s_w[lane] = pk.w;
-                s_asc[pk.pos] = lane;
+                s_w[sb + lane] = pk.w;
+                s_asc[sb + pk.pos] = sb + lane;
                 if (blockIdx.x == 0) {
-                    a.idx[lane] = pk.e;
-                    a.wts[lane] = pk.w;
-                    a.asc[pk.pos] = lane;
-                    a.ulist[pk.pos] = pk.e;
+                    a.idx[sb + lane] = pk.e;
+                    a.wts[sb + lane] = pk.w;
+                    a.asc[sb + pk.pos] = lane;
+                    if (NT == 1) a.ulist[pk.pos] = pk.e;
                 }
             }
             if (blockIdx.x == 0 && lane == 0) {
-                *a.n_unique = k;
-                *a.xsum = xs * (double)exp2i(-sig);
+                if (NT == 1) *a.n_unique = k;
+                a.xsum[tt] = pick_tok(xs, tt) * (double)exp2i(-pick_tok(sig, tt));
             }
         }
         for (; q < my_tasks; ++q) {
             if (lane == 0)
                 while (issued < limit && issued < q + nst) issue(issued++);
             if (!wait_use(q)) { ok = false; break; }
-            gate_up_use(q, rows_mma_x<WK, NDK>(st_s(q % nst), st_s(q % nst) + gu_row, gu_lane_off, grot, xblk, lane));
+            gate_up_stage(q);
         }
         if (ok && lane == 0)
             while (issued < limit && issued < q + nst) issue(issued++);
@@ -957,17 +1006,19 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
 
     // ---- combine: routed slots in ascending expert order, then the shared expert
     if (s_ok) {
-        for (int i = tid; i < rj; i += blockDim.x) {
+        for (int it2 = tid; it2 < NT * rj; it2 += blockDim.x) {
+            const int tk = it2 / rj, i = it2 - tk * rj;
             float o = 0.0f;
             for (int p = 0; p < k; ++p) {              // ascending expert order
-                const int u = s_asc[p];
+                const int u = s_asc[tk * k + p];
                 o = fmaf(s_w[u], ys[u][i], o);
             }
-            if (a.S) o += ys[k][i];
+            if (a.S) o += ys[nrs + tk][i];
+            const size_t at = (size_t)tk * d + j0 + i;
             if (a.out_bf16)
-                static_cast<__nv_bfloat16*>(a.out)[j0 + i] = __float2bfloat16_rn(o);
+                static_cast<__nv_bfloat16*>(a.out)[at] = __float2bfloat16_rn(o);
             else
-                static_cast<float*>(a.out)[j0 + i] = o;
+                static_cast<float*>(a.out)[at] = o;
         }
     }
     stamp(10);
@@ -981,92 +1032,98 @@ size_t fz_xt_bytes(const LayerDims& L) {
     const size_t blk = fz_bf16(L) ? 16 * (size_t)(L.d / 256) + 16 : 64 * (size_t)(L.d / 1024) + 16;
     return (32 * blk + 127) / 128 * 128;
 }
-// Warps per CTA: as many (up to 16) as kFzStages ring stages each fit in shared memory beside the
-// lane blocks.
-int fz_warps(const LayerDims& L) {
-    const size_t room = kSmemLimit - kStaticReserve - fz_xt_bytes(L);
-    const int w = (int)(room / ((size_t)kFzStages * fz_stage_bytes(L)));
-    return w > kFzMaxWarps ? kFzMaxWarps : w;
+// Warps per CTA: as many (up to 16; an even number for two tokens, whose selection takes one half
+// each) as kFzStages ring stages each fit in shared memory beside the tokens' lane blocks.
+int fz_warps(const LayerDims& L, int nt) {
+    const size_t room = kSmemLimit - fz_static_reserve(nt) - (size_t)nt * fz_xt_bytes(L);
+    int w = (int)(room / ((size_t)kFzStages * fz_stage_bytes(L)));
+    if (w > kFzMaxWarps) w = kFzMaxWarps;
+    return nt > 1 ? w - w % nt : w;
 }
-size_t fz_dyn_smem(const LayerDims& L) {
-    return fz_xt_bytes(L) + (size_t)kFzStages * fz_warps(L) * fz_stage_bytes(L);
+size_t fz_dyn_smem(const LayerDims& L, int nt) {
+    return (size_t)nt * fz_xt_bytes(L) + (size_t)kFzStages * fz_warps(L, nt) * fz_stage_bytes(L);
 }
 int fz_dn_rows(const LayerDims& L) {
     const int r = (int)(fz_stage_bytes(L) / fz_row_bytes(L, L.f));
     return r > kFzDnRowsMax ? kFzDnRowsMax : r;
 }
 
-template <int NDK>
+template <int NDK, int NT>
 const void* fz_pick_f(int nf) {
-    return nf == 1 ? (const void*)decode_fused_kernel<MOE_W_INT4_ROWSCALE, NDK, 1>
-                   : (const void*)decode_fused_kernel<MOE_W_INT4_ROWSCALE, NDK, 2>;
+    return nf == 1 ? (const void*)decode_fused_kernel<MOE_W_INT4_ROWSCALE, NDK, 1, NT>
+                   : (const void*)decode_fused_kernel<MOE_W_INT4_ROWSCALE, NDK, 2, NT>;
 }
-const void* fz_pick(const LayerDims& L) {
-    if (fz_bf16(L)) {     // d = 1024 or 2048 (4 or 8 groups), f = 512 or 1024 (2 or 4 groups)
-        if (L.d == 1024)
-            return L.f == 512 ? (const void*)decode_fused_kernel<MOE_W_BF16, 4, 2>
-                              : (const void*)decode_fused_kernel<MOE_W_BF16, 4, 4>;
-        return L.f == 512 ? (const void*)decode_fused_kernel<MOE_W_BF16, 8, 2>
-                          : (const void*)decode_fused_kernel<MOE_W_BF16, 8, 4>;
-    }
+template <int NT>
+const void* fz_pick_int4(const LayerDims& L) {
     const int nf = L.f / 1024;
     switch (L.d / 1024) {
-        case 1: return fz_pick_f<1>(nf);
-        case 2: return fz_pick_f<2>(nf);
-        case 3: return fz_pick_f<3>(nf);
-        case 4: return fz_pick_f<4>(nf);
-        case 5: return fz_pick_f<5>(nf);
-        case 6: return fz_pick_f<6>(nf);
-        case 7: return fz_pick_f<7>(nf);
-        default: return fz_pick_f<8>(nf);
+        case 1: return fz_pick_f<1, NT>(nf);
+        case 2: return fz_pick_f<2, NT>(nf);
+        case 3: return fz_pick_f<3, NT>(nf);
+        case 4: return fz_pick_f<4, NT>(nf);
+        case 5: return fz_pick_f<5, NT>(nf);
+        case 6: return fz_pick_f<6, NT>(nf);
+        case 7: return fz_pick_f<7, NT>(nf);
+        default: return fz_pick_f<8, NT>(nf);
     }
+}
+const void* fz_pick(const LayerDims& L, int nt) {
+    if (fz_bf16(L)) {     // one token; d = 1024 or 2048 (4 or 8 groups), f = 512 or 1024 (2 or 4 groups)
+        if (L.d == 1024)
+            return L.f == 512 ? (const void*)decode_fused_kernel<MOE_W_BF16, 4, 2, 1>
+                              : (const void*)decode_fused_kernel<MOE_W_BF16, 4, 4, 1>;
+        return L.f == 512 ? (const void*)decode_fused_kernel<MOE_W_BF16, 8, 2, 1>
+                          : (const void*)decode_fused_kernel<MOE_W_BF16, 8, 4, 1>;
+    }
+    return nt == 2 ? fz_pick_int4<2>(L) : fz_pick_int4<1>(L);
 }
 
 }  // namespace
 
-bool decode_fused_shape_ok(const LayerDims& L) {
+bool decode_fused_shape_ok(const LayerDims& L, int nt) {
     const bool int4_shape = L.wkind == MOE_W_INT4_ROWSCALE && L.d % 1024 == 0 && L.d / 1024 >= 1 && L.d / 1024 <= 8 &&
                             (L.f == 1024 || L.f == 2048);
-    const bool bf16_shape = L.wkind == MOE_W_BF16 && (L.d == 1024 || L.d == 2048) && (L.f == 512 || L.f == 1024);
+    const bool bf16_shape = nt == 1 && L.wkind == MOE_W_BF16 && (L.d == 1024 || L.d == 2048) &&
+                            (L.f == 512 || L.f == 1024);
+    if (nt < 1 || nt > 2) return false;
     if (!((int4_shape || bf16_shape) && (!L.S || L.f_shared == L.f) && L.k + L.S <= kFzMaxSlots &&
-          L.E <= kWarp * kFzMaxPer && L.k <= L.E && fz_dn_rows(L) >= 1 && fz_warps(L) >= 4))
+          L.E <= kWarp * kFzMaxPer && L.k <= L.E && fz_dn_rows(L) >= 1 && fz_warps(L, nt) >= 4))
         return false;
-    // the selection keeps the router pieces, keys and logits in the (idle) rings; E <= threads
-    const size_t rings = (size_t)kFzStages * fz_warps(L) * fz_stage_bytes(L);
-    const size_t sel_bytes = ((size_t)L.E * (L.d / 1024) * 8 + 15) / 16 * 16 + 16 * (size_t)L.E;
-    return sel_bytes <= rings && L.E <= fz_warps(L) * kWarp;
+    // the selection keeps the router pieces, keys and logits in the (idle) rings; each token's
+    // experts fit one thread each in its half of the CTA
+    const size_t rings = (size_t)kFzStages * fz_warps(L, nt) * fz_stage_bytes(L);
+    const size_t sel_bytes = ((size_t)nt * L.E * (L.d / 1024) * 8 + 15) / 16 * 16 + 16 * (size_t)nt * L.E;
+    return sel_bytes <= rings && L.E <= fz_warps(L, nt) / nt * kWarp;
 }
 
-cudaError_t prepare_decode_fused(const LayerDims& L, int num_sms, bool* usable) {
+cudaError_t prepare_decode_fused(const LayerDims& L, int num_sms, bool* usable, int nt) {
     *usable = false;
-    if (!decode_fused_shape_ok(L) || (L.d + num_sms - 1) / num_sms > kFzRowsMax || num_sms > kTraceCtas)
+    if (!decode_fused_shape_ok(L, nt) || (L.d + num_sms - 1) / num_sms > fz_rows_max(nt) || num_sms > kTraceCtas)
         return cudaSuccess;
     // the down items of one warp must fit the scale registers
     const int rows = (L.d + num_sms - 1) / num_sms;
-    if ((L.k + L.S) * rows > fz_warps(L) * (kWarp * kFzScRegs - 1)) return cudaSuccess;
+    if (nt * (L.k + L.S) * rows > fz_warps(L, nt) * (kWarp * kFzScRegs - 1)) return cudaSuccess;
     int dev = 0, coop = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
     if (e != cudaSuccess || !coop) return e;
-    const void* fn = fz_pick(L);
+    const void* fn = fz_pick(L, nt);
     cudaFuncAttributes fa;
     e = cudaFuncGetAttributes(&fa, fn);
     if (e != cudaSuccess) return e;
-    if (fa.sharedSizeBytes > (size_t)kStaticReserve) return cudaSuccess;
-    const size_t dyn = fz_dyn_smem(L);
+    if (fa.sharedSizeBytes > fz_static_reserve(nt)) return cudaSuccess;
+    const size_t dyn = fz_dyn_smem(L, nt);
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(kSmemLimit - fa.sharedSizeBytes));
     if (e != cudaSuccess) return e;
     int blocks = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, fn, fz_warps(L) * kWarp, dyn);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, fn, fz_warps(L, nt) * kWarp, dyn);
     if (e != cudaSuccess) return e;
     *usable = blocks >= 1;
     return cudaSuccess;
 }
 
-size_t decode_fused_rpart_count(const LayerDims& L) { return (size_t)L.E * (L.d / 1024 > 0 ? L.d / 1024 : 1); }
-
 cudaError_t launch_decode_fused(const LayerDims& L, const moe_weights& W, const uint16_t* x, const Workspace& ws,
-                                void* out, int num_sms, const Launch& ctx) {
+                                void* out, int num_sms, const Launch& ctx, int nt) {
     FusedArgs a;
     a.router_w = W.router_w;
     a.bias = L.router == MOE_ROUTER_SIGMOID_BIAS ? W.router_bias : nullptr;
@@ -1099,8 +1156,8 @@ cudaError_t launch_decode_fused(const LayerDims& L, const moe_weights& W, const 
     a.scaling = L.scaling;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)num_sms);
-    cfg.blockDim = dim3((unsigned)(fz_warps(L) * kWarp));
-    cfg.dynamicSmemBytes = fz_dyn_smem(L);
+    cfg.blockDim = dim3((unsigned)(fz_warps(L, nt) * kWarp));
+    cfg.dynamicSmemBytes = fz_dyn_smem(L, nt);
     cfg.stream = ctx.s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;
@@ -1109,7 +1166,7 @@ cudaError_t launch_decode_fused(const LayerDims& L, const moe_weights& W, const 
     cfg.numAttrs = 1;
     void* args[] = {&a};
     prof_mark(ctx.prof, MOE_KERNEL_FUSED, true, ctx.s);
-    cudaError_t e = cudaLaunchKernelExC(&cfg, fz_pick(L), args);
+    cudaError_t e = cudaLaunchKernelExC(&cfg, fz_pick(L, nt), args);
     prof_mark(ctx.prof, MOE_KERNEL_FUSED, false, ctx.s);
     if (e != cudaSuccess) return e;
     ++*ctx.launches;

@@ -120,7 +120,7 @@ struct Workspace {
     // [2E, 3E) down rows, [3E, 4E) down scales.  Filled from the contiguous [E] arrays at layer
     // creation; moe_layer_set_expert re-points one expert (a non-contiguous expert slab).
     const void** etab;
-    double* rpart;         // [E][d / 1024]: pieces of the router logits
+    double* rpart;         // [2][E][d / 1024]: pieces of the router logits of one or two tokens
     double* rsplit;        // partial logits and sums of x of the K-sliced router GEMM
     double* keys;          // [T][E] selection keys (small-batch router)
     size_t rsplit_n;       // its length in doubles (0: none)
@@ -208,12 +208,12 @@ cudaError_t launch_route_small(const LayerDims& L, const float* router_w, const 
 bool decode_t1_supported(const LayerDims& L);
 cudaError_t launch_decode_t1(const LayerDims& L, const moe_weights& W, const uint16_t* x, const Workspace& ws,
                              void* out, int num_sms, const Launch& ctx);
-// One token, int4 experts, the whole layer in one cooperative launch (decode_fused.cu).
-bool decode_fused_shape_ok(const LayerDims& L);
-cudaError_t prepare_decode_fused(const LayerDims& L, int num_sms, bool* usable);
-size_t decode_fused_rpart_count(const LayerDims& L);
+// One or two tokens (nt), int4 experts (bf16 too for one token), the whole layer in one
+// cooperative launch (decode_fused.cu).
+bool decode_fused_shape_ok(const LayerDims& L, int nt);
+cudaError_t prepare_decode_fused(const LayerDims& L, int num_sms, bool* usable, int nt);
 cudaError_t launch_decode_fused(const LayerDims& L, const moe_weights& W, const uint16_t* x, const Workspace& ws,
-                                void* out, int num_sms, const Launch& ctx);
+                                void* out, int num_sms, const Launch& ctx, int nt);
 cudaError_t launch_decode_experts(const LayerDims& L, const moe_weights& W, const uint16_t* x, int T,
                                   const Workspace& ws, int num_sms, const Launch& ctx);
 cudaError_t launch_combine(const LayerDims& L, int T, const Workspace& ws, void* out, const Launch& ctx);

@@ -85,6 +85,7 @@ struct moe_layer {
     int64_t prefill_min_tokens = 128;    // batches at least this large take the grouped-GEMM path
     int t1_mode = 0;                     // T = 1: 2 single launch, 1 single-token kernels, 0 general
     bool fused_ok = false;               // the single-launch path is usable for this layer
+    bool fused2_ok = false;              // ... and for two-token batches
     bool union_mma = true;               // small batches: the tensor-core union kernels when they fit
     bool ragged = false;                 // some routed expert lives outside the contiguous [E] arrays
 };
@@ -153,7 +154,7 @@ size_t carve(const moe_config& c, size_t max_groups, char* base, qe::Workspace* 
     w.status = (int32_t*)take(sizeof(int32_t));
     w.counter = (uint32_t*)take(sizeof(uint32_t));
     w.etab = (const void**)take(sizeof(void*) * 4 * E);
-    w.rpart = (double*)take(sizeof(double) * E * (c.d / 1024 > 0 ? (size_t)c.d / 1024 : 1));
+    w.rpart = (double*)take(sizeof(double) * 2 * E * (c.d / 1024 > 0 ? (size_t)c.d / 1024 : 1));
     w.gbar = (unsigned long long*)take(sizeof(unsigned long long));
     w.trace = (unsigned long long*)take(sizeof(unsigned long long) * qe::kTraceCtas * qe::kTraceStamps);
     if (max_groups) {
@@ -283,7 +284,9 @@ moe_status moe_layer_create(const moe_config* cfg, const moe_weights* w, moe_lay
     if (e == cudaSuccess) e = qe::prepare_bucket(L->dims);
     if (e == cudaSuccess) e = qe::prepare_decode(L->dims);
     if (e == cudaSuccess) e = qe::prepare_decode_mma();
-    if (e == cudaSuccess) e = qe::prepare_decode_fused(L->dims, L->num_sms, &L->fused_ok);
+    if (e == cudaSuccess) e = qe::prepare_decode_fused(L->dims, L->num_sms, &L->fused_ok, 1);
+    if (e == cudaSuccess && cfg->max_tokens >= 2)
+        e = qe::prepare_decode_fused(L->dims, L->num_sms, &L->fused2_ok, 2);
     const bool gemm = qe::prefill_supported(L->dims);
     if (e == cudaSuccess && gemm) e = qe::prepare_prefill(L->dims);
     if (e != cudaSuccess) {
@@ -361,8 +364,8 @@ moe_status moe_forward(moe_layer* L, const uint16_t* x, int32_t T, void* out, mo
     cudaError_t e;
     // the single-token paths take the plain router only (a router variant may drop experts)
     const bool variant = L->dims.ropts.active();
-    if (T == 1 && L->t1_mode == 2 && !variant) {
-        e = qe::launch_decode_fused(L->dims, L->w, x, ws, out, L->num_sms, ctx);
+    if (T <= 2 && L->t1_mode == 2 && !variant && (T == 1 || L->fused2_ok)) {
+        e = qe::launch_decode_fused(L->dims, L->w, x, ws, out, L->num_sms, ctx, T);
         L->last_stream = s;
         L->last_launches = launches;
         return from_cuda(e);

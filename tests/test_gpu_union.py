@@ -49,6 +49,7 @@ def _layer(built, name):
         cfg = _cfg(name, 100)
         drawn = {}
         layer, _ = build_gpu_layer(cfg, max_tokens=100, oracle_experts=drawn)
+        layer.set_single_token_mode(1)     # T = 2 too goes to the batch kernels
         built[name] = (layer, oracle_layer_from(cfg, drawn))
     return built[name]
 
