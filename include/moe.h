@@ -286,10 +286,14 @@ void moe_layer_destroy(moe_layer *layer);
  *                               tensor-core products of 16 weight rows by up to 8 tokens; 0 runs the
  *                               general kernels (FP32-pipe dot products).  Results agree within the
  *                               layer's tolerance, not bit for bit.
+ *   MOE_OPT_PHASE_TRACE          1: the single launch records the phase times that MOE_DEBUG_TRACE
+ *                               returns; 0 (default): it records none (each stamp is a timer read
+ *                               on the path of the CTA's first thread).  Same results.
  */
 enum { MOE_OPT_PREFILL_MIN_TOKENS = 0, MOE_OPT_PREFILL_AVAILABLE = 1, MOE_OPT_SINGLE_TOKEN_KERNELS = 2,
        MOE_OPT_PROGRAMMATIC_LAUNCH = 3, MOE_OPT_WAIT_LIMIT_US = 4, MOE_OPT_TEST_SKIP_GEMM_B_COPIES = 5,
-       MOE_OPT_ROUTER_GROUPS = 6, MOE_OPT_ROUTER_TOP_P = 7, MOE_OPT_UNION_TENSOR_CORES = 8 };
+       MOE_OPT_ROUTER_GROUPS = 6, MOE_OPT_ROUTER_TOP_P = 7, MOE_OPT_UNION_TENSOR_CORES = 8,
+       MOE_OPT_PHASE_TRACE = 9 };
 moe_status moe_layer_set_option(moe_layer *layer, int32_t option, int64_t value);
 moe_status moe_layer_get_option(const moe_layer *layer, int32_t option, int64_t *value);
 
@@ -307,12 +311,13 @@ moe_status moe_layer_get_option(const moe_layer *layer, int32_t option, int64_t 
  *   MOE_DEBUG_ULIST  int32 [E] unique chosen experts, ascending;  MOE_DEBUG_CNT int32 [E]
  *                    (CNT is not written by the single-launch path, ULIST not by it at T = 2)
  *   MOE_DEBUG_XSUM   fp64 [T]
- *   MOE_DEBUG_TRACE  uint64 [SMs][16]: for the single-launch T = 1 path, the %globaltimer value (ns)
- *                    at which each CTA passed its phase boundaries: 0 start, 1 x rearranged
- *                    in shared memory, 2 router pieces stored, 3 shared rows done, 4 first grid barrier passed,
- *                    5 router pieces gathered, 6 experts selected, 7 routed gate/up done, 8 h
- *                    complete, 9 down done, 10 output stored, 11 x in shared memory, 12..15
- *                    steps of the selection (candidates, ranks, gate weights, proxy fence)
+ *   MOE_DEBUG_TRACE  uint64 [SMs][16]: for the single-launch path with MOE_OPT_PHASE_TRACE on, the
+ *                    %globaltimer value (ns) at which each CTA passed its phase boundaries: 0 start,
+ *                    11 x in shared memory, 1 router pieces stored, 2 arrived at the first grid
+ *                    barrier, 3 x rearranged and the shared rows done, 4 first grid barrier passed,
+ *                    5 router pieces gathered, 12 candidates, 13 ranks and pointers, 14 and 15
+ *                    around a proxy fence, 6 experts selected, 7 routed gate/up done, 8 h
+ *                    complete, 9 down done, 10 output stored
  */
 enum { MOE_DEBUG_H = 0, MOE_DEBUG_Y = 1, MOE_DEBUG_IDX = 2, MOE_DEBUG_W = 3, MOE_DEBUG_ASC = 4,
        MOE_DEBUG_ULIST = 5, MOE_DEBUG_CNT = 6, MOE_DEBUG_XSUM = 7, MOE_DEBUG_TRACE = 8 };

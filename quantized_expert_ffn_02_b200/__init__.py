@@ -30,7 +30,7 @@ EXPORTS = (
 )
 (MOE_OPT_PREFILL_MIN_TOKENS, MOE_OPT_PREFILL_AVAILABLE, MOE_OPT_SINGLE_TOKEN_KERNELS, MOE_OPT_PROGRAMMATIC_LAUNCH,
  MOE_OPT_WAIT_LIMIT_US, MOE_OPT_TEST_SKIP_GEMM_B_COPIES, MOE_OPT_ROUTER_GROUPS, MOE_OPT_ROUTER_TOP_P,
- MOE_OPT_UNION_TENSOR_CORES) = range(9)
+ MOE_OPT_UNION_TENSOR_CORES, MOE_OPT_PHASE_TRACE) = range(10)
 DEBUG_ITEMS = {"h": 0, "y": 1, "idx": 2, "w": 3, "asc": 4, "ulist": 5, "cnt": 6, "xsum": 7, "trace": 8}
 KERNELS = ("router_logits", "topk", "bucket", "gateup", "down", "combine", "gather", "gemm_gateup", "gemm_down",
            "fused")
@@ -302,6 +302,10 @@ class MoELayer:
     def set_router_top_p(self, p: float):
         """Adaptive expert top-p (0 or 1: off)."""
         moe_layer_set_option(self.handle, MOE_OPT_ROUTER_TOP_P, int(round(p * 1e6)))
+
+    def set_phase_trace(self, on: bool):
+        """Single launch: record the phase times read back as debug item "trace"."""
+        moe_layer_set_option(self.handle, MOE_OPT_PHASE_TRACE, 1 if on else 0)
 
     def set_union_tensor_cores(self, on: bool):
         """Small batches (T >= 2) on the tensor-core union kernels (default) or the general kernels."""

@@ -163,6 +163,7 @@ struct LayerDims {
     int pdl = 1;           // chain dependent kernels with programmatic dependent launch
     uint64_t wait_ns = 2000000000ull;   // limit of the grouped-GEMM kernels' bounded waits
     int test_skip_b = 0;   // test hook: the grouped GEMM's B producer issues no copies
+    int phase_trace = 0;   // the single launch records its phase times
     RouterOpts ropts;      // router variants (off by default)
 };
 

@@ -506,6 +506,10 @@ moe_status moe_layer_set_option(moe_layer* L, int32_t option, int64_t value) {
             if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
             L->union_mma = value != 0;
             return MOE_OK;
+        case MOE_OPT_PHASE_TRACE:
+            if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+            L->dims.phase_trace = (int)value;
+            return MOE_OK;
         default:
             return MOE_ERR_INVALID_ARG;
     }
@@ -550,6 +554,7 @@ moe_status moe_layer_get_option(const moe_layer* L, int32_t option, int64_t* val
             return MOE_OK;
         case MOE_OPT_ROUTER_TOP_P: *value = (int64_t)(L->dims.ropts.top_p * 1e6 + 0.5); return MOE_OK;
         case MOE_OPT_UNION_TENSOR_CORES: *value = L->union_mma ? 1 : 0; return MOE_OK;
+        case MOE_OPT_PHASE_TRACE: *value = L->dims.phase_trace; return MOE_OK;
         default: return MOE_ERR_INVALID_ARG;
     }
 }
