@@ -468,12 +468,13 @@ def source_sha(paths):
     return h.hexdigest()[:16]
 
 
-def traffic_for(kernel):
-    """dram bytes per launch from a committed ncu capture, if the kernel source is unchanged since."""
+def traffic_for(kernel, workload):
+    """dram bytes per launch of `kernel` in `workload` from a committed ncu capture, if the
+    kernel's sources are unchanged since (entries are keyed "workload:kernel")."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
-    rec = json.load(open(path)).get(kernel)
+    rec = json.load(open(path)).get(f"{workload}:{kernel}")
     if not rec:
         return None
     try:
@@ -687,13 +688,13 @@ def measure_workload(a, name, cfg, layer, dev, dist, world, rank, local_rank, fl
             if kind == "hbm":
                 achieved = amount / (per_launch_ms / 1e3) / 1e9
                 roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                        "frac": achieved / hbm, "traffic": traffic_for(dom),
+                        "frac": achieved / hbm, "traffic": traffic_for(dom, name),
                         "peak_kind": f"{peak_kind} copy bandwidth",
                         "algorithmic_bytes_per_launch": amount, "ms_per_launch": per_launch_ms}
             else:
                 achieved = amount / (per_launch_ms / 1e3) / 1e12
                 roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": tf, "unit": "TFLOP/s",
-                        "frac": achieved / tf, "traffic": traffic_for(dom),
+                        "frac": achieved / tf, "traffic": traffic_for(dom, name),
                         "peak_kind": f"{peak_kind} bf16 dense (burst)",
                         "algorithmic_flops_per_launch": amount, "ms_per_launch": per_launch_ms}
     step_bytes = statistics.mean(uniq[(a.warmup + i) % len(xs)] for i in range(a.steps)) * expert_bytes(cfg) + \

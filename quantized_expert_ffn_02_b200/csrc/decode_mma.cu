@@ -39,11 +39,16 @@ using namespace dec;
 
 constexpr int kUMaxWarps = 12;                // (the register budget allows 8 accumulators)
 constexpr int kUStages = 2;                 // ring stages per warp
-constexpr int kUChunk = 512;                // bytes of a weight row per stage (1024 codes)
-constexpr int kUSteps = kUChunk / 64;       // MMA steps (128 codes) per stage
-constexpr int kURowPitch = kUChunk + 64;    // shared-memory bytes per row in a stage: the lanes of
-                                            // rows g and g + 1 then meet different banks
-constexpr int kUStage = 16 * kURowPitch;
+// Bytes of a weight row per stage: 256 (512 codes) for gate/up, 512 for down.  Gate/up holds
+// its 8 columns of x (2d bytes each) beside the rings, so smaller stages buy more warps (12
+// instead of 6 for d = 6144: gate/up 437 -> 383 us at T = 32); down's h columns are small and it
+// already runs 10 warps, where 256-byte stages measured slower (178 -> 195 us).
+template <bool GU> constexpr int u_chunk() { return GU ? 256 : 512; }
+template <bool GU> constexpr int u_steps() { return u_chunk<GU>() / 64; }   // MMA steps (128 codes) per stage
+// Shared-memory bytes per row in a stage: the lanes of rows g and g + 1 then meet different
+// banks (the pitch is 16 words past a multiple of 32 words for both chunk sizes).
+template <bool GU> constexpr int u_pitch() { return u_chunk<GU>() + 64; }
+template <bool GU> constexpr int u_stage() { return 16 * u_pitch<GU>(); }
 constexpr int kUCols = 8;                   // columns (tokens or slots) per unit
 constexpr int kUChains = 8;                 // independent accumulators per warp
 constexpr size_t kUSmemLimit = 227 * 1024;
@@ -148,6 +153,7 @@ __global__ void __launch_bounds__(kUMaxWarps * kWarp, 1) union_mma_kernel(const 
     const uint32_t vrs = (uint32_t)Kmax * 2u + 16u;       // v row pitch (bytes)
     const uint32_t v_s = saddr(smem);
     const uint32_t rings_s = v_s + (uint32_t)a.vrows * vrs;
+    constexpr int kUChunk = u_chunk<GU>(), kUSteps = u_steps<GU>(), kURowPitch = u_pitch<GU>(), kUStage = u_stage<GU>();
     const uint32_t ring_s = rings_s + (uint32_t)warp * kUStages * kUStage;
     const int nu = *a.n_unique;
     const int nb_r = GU ? a.f / 8 : a.d / 16;              // blocks of a routed unit
@@ -469,9 +475,9 @@ __global__ void __launch_bounds__(kUMaxWarps * kWarp, 1) union_mma_kernel(const 
     __syncwarp();
 }
 
-int union_warps(size_t vbytes) {
+int union_warps(size_t vbytes, int stage) {
     const size_t room = kUSmemLimit - kUStaticReserve - vbytes;
-    const int w = (int)(room / ((size_t)kUStages * kUStage));
+    const int w = (int)(room / ((size_t)kUStages * stage));
     return w > kUMaxWarps ? kUMaxWarps : w;
 }
 
@@ -484,7 +490,7 @@ bool decode_mma_ok(const LayerDims& L, int T) {
     const int vrows = T < kUCols ? T : kUCols;
     const size_t gu_v = (size_t)vrows * (2 * (size_t)L.d + 16);
     const size_t dn_v = (size_t)vrows * (2 * (size_t)(L.S && L.f_shared > L.f ? L.f_shared : L.f) + 16);
-    return union_warps(gu_v) >= 2 && union_warps(dn_v) >= 2;
+    return union_warps(gu_v, u_stage<true>()) >= 2 && union_warps(dn_v, u_stage<false>()) >= 2;
 }
 
 cudaError_t prepare_decode_mma() {
@@ -526,8 +532,8 @@ cudaError_t launch_decode_mma(const LayerDims& L, const moe_weights& W, const ui
         g.dst = ws.h;
         g.dst_ld = fmax;
         const size_t vb = (size_t)vrows * (2 * (size_t)L.d + 16);
-        const int warps = union_warps(vb);
-        const size_t smem = vb + (size_t)warps * kUStages * kUStage;
+        const int warps = union_warps(vb, u_stage<true>());
+        const size_t smem = vb + (size_t)warps * kUStages * u_stage<true>();
         QE_LAUNCH(ctx, MOE_KERNEL_GATEUP,
                   (union_mma_kernel<true><<<num_sms, warps * kWarp, smem, ctx.s>>>(g)));
     }
@@ -541,8 +547,8 @@ cudaError_t launch_decode_mma(const LayerDims& L, const moe_weights& W, const ui
         dn.dst = ws.Y;
         dn.dst_ld = L.d;
         const size_t vb = (size_t)vrows * (2 * (size_t)fmax + 16);
-        const int warps = union_warps(vb);
-        const size_t smem = vb + (size_t)warps * kUStages * kUStage;
+        const int warps = union_warps(vb, u_stage<false>());
+        const size_t smem = vb + (size_t)warps * kUStages * u_stage<false>();
         QE_LAUNCH(ctx, MOE_KERNEL_DOWN,
                   (union_mma_kernel<false><<<num_sms, warps * kWarp, smem, ctx.s>>>(dn)));
     }

@@ -123,6 +123,8 @@ struct Workspace {
     double* rpart;         // [2][E][d / 1024]: pieces of the router logits of one or two tokens
     double* rsplit;        // partial logits and sums of x of the K-sliced router GEMM
     double* keys;          // [T][E] selection keys (small-batch router)
+    double* rsmall;        // small-batch router: [slices][T][E] partial logits, [slices][T] partial x sums
+    unsigned int* rsmall_cnt;   // small-batch router: finished blocks per expert group
     size_t rsplit_n;       // its length in doubles (0: none)
     unsigned long long* gbar;  // [1]: grid-barrier arrivals (only grows)
     unsigned long long* trace; // [kTraceCtas][kTraceStamps]: phase timestamps of that path
@@ -203,8 +205,11 @@ cudaError_t launch_decode_mma(const LayerDims& L, const moe_weights& W, const ui
                               int num_sms, const Launch& ctx);
 // Small batches: logits, top-k, gate weights and bucket tables in one launch.
 constexpr int kRouteSmallMaxT = 32;
+bool route_small_ok(const LayerDims& L, int num_sms);
+size_t route_small_part_doubles(int E, int max_tokens);
+size_t route_small_groups(int E);
 cudaError_t launch_route_small(const LayerDims& L, const float* router_w, const float* router_bias, const uint16_t* x,
-                               int T, const Workspace& ws, const Launch& ctx);
+                               int T, const Workspace& ws, int num_sms, const Launch& ctx);
 // One token, int4 experts: gate/up and down+combine kernels (decode1.cu).
 bool decode_t1_supported(const LayerDims& L);
 cudaError_t launch_decode_t1(const LayerDims& L, const moe_weights& W, const uint16_t* x, const Workspace& ws,

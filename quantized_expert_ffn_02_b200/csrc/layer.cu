@@ -137,6 +137,8 @@ size_t carve(const moe_config& c, size_t max_groups, char* base, qe::Workspace* 
     qe::Workspace w{};
     w.logits = (double*)take(sizeof(double) * T * E);
     w.keys = (double*)take(sizeof(double) * std::min(T, (size_t)qe::kRouteSmallMaxT) * E);
+    w.rsmall = (double*)take(sizeof(double) * qe::route_small_part_doubles((int)E, (int)T));
+    w.rsmall_cnt = (unsigned int*)take(sizeof(unsigned int) * qe::route_small_groups((int)E));
     w.rsplit_n = qe::router_split_doubles((int)E, (int)T);
     w.rsplit = w.rsplit_n ? (double*)take(sizeof(double) * w.rsplit_n) : nullptr;
     w.idx = (int32_t*)take(sizeof(int32_t) * T * k);
@@ -370,8 +372,8 @@ moe_status moe_forward(moe_layer* L, const uint16_t* x, int32_t T, void* out, mo
         L->last_launches = launches;
         return from_cuda(e);
     }
-    if (T <= qe::kRouteSmallMaxT) {
-        e = qe::launch_route_small(L->dims, L->w.router_w, L->w.router_bias, x, T, ws, ctx);
+    if (T <= qe::kRouteSmallMaxT && qe::route_small_ok(L->dims, L->num_sms)) {
+        e = qe::launch_route_small(L->dims, L->w.router_w, L->w.router_bias, x, T, ws, L->num_sms, ctx);
     } else {
         e = qe::launch_router(L->dims, L->w.router_w, L->w.router_bias, x, T, ws.logits, ws.xsum, ws.idx, ws.wts,
                               ws.asc, ctx, ws.rsplit, ws.rsplit_n);

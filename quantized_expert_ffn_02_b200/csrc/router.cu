@@ -5,6 +5,8 @@
 // iliria page, "What's implemented": noaux_tc).  Logits are accumulated in fp64: every
 // product bf16 * fp32 is exact in fp64, so the only rounding is in the sums and the top-k
 // boundary is decided at fp64 resolution.  Equal keys go to the lower expert index.
+#include <algorithm>
+
 #include "internal.cuh"
 #include "topk.cuh"
 
@@ -208,12 +210,40 @@ topk_kernel(const double* __restrict__ logits, int nsplit, const double* __restr
 
 // ---------------------------------------------------------------------------------------
 // Small batches (T <= 32): one launch for logits, top-k, gate weights and bucketing.
-// grid = E blocks of 256 threads, block e computes logits[t][e] for every token; the last block
-// to finish (an atomic counter, reset by that block) selects and buckets all T tokens.
+//
+// Block (g, z) of the (NG, KS) grid owns the 16 experts 16 g .. 16 g + 15 (one per warp) and
+// the K slice z: columns [64 ns z, 64 ns (z + 1)).  It stages the slice of every token's x in
+// shared memory once, keeps its warp's router-row slice in registers (lane l: the column pairs
+// 64 i + 2 l), and writes fp64 partial logits [z][t][e] for 8 tokens per pass; a transposed
+// shuffle reduction leaves each token's sum in four lanes.  The last block of a group to finish
+// (a per-group counter) adds the KS partials of its experts in slice order and writes their
+// logits and selection keys; the last group to finish (a second counter) selects and buckets
+// every token, a warp per token.  Every sum has a fixed order, so the logits do not depend on
+// which block finished first.
 // ---------------------------------------------------------------------------------------
-constexpr int kSmallThreads = 256;
+constexpr int kSmallThreads = 512;
+constexpr int kSmallWarps = kSmallThreads / kWarp;      // experts per block
 constexpr int kSmallMaxT = 32;
 constexpr int kSmallMaxE = 1024;
+constexpr int kSmallMaxSteps = 16;                      // 64-column steps per slice (32 floats per lane)
+constexpr int kSmallMaxSlices = 16;
+
+struct SmallArgs {
+    const float* wr;            // [E][d] fp32 router
+    const float* bias;          // [E] selection bias or null
+    const uint16_t* x;          // [T][d] bf16
+    int T, d, E, k, router, ns; // ns: 64-column steps per slice
+    float scaling;
+    double* part;               // [KS][T][E] partial logits, then [KS][T] partial x sums
+    unsigned int* gcnt;         // [NG] blocks of each group done (reset by the group's last block)
+    unsigned int* counter;      // groups done (reset by the last group)
+    double* logits;             // [T][E]
+    double* keys;               // [T][E]
+    double* xsum;               // [T]
+    int32_t *idx, *asc, *cnt, *off, *perm, *slot_of, *ulist, *n_unique;
+    float* wts;
+    RouterOpts opts;
+};
 
 // Selection for one token whose logits and keys other blocks wrote (read through L2).
 template <int MAXPER>
@@ -235,124 +265,128 @@ __device__ void warp_select(const double* __restrict__ lg, const double* __restr
     }
 }
 
-template <int MAXPER, int MAXC>
-__global__ void __launch_bounds__(kSmallThreads, 2)
-route_small_kernel(const float* __restrict__ wr, const float* __restrict__ bias, const uint16_t* __restrict__ x, int T,
-                   int d, int E, int k, int router, float scaling, double* __restrict__ logits,
-                   double* __restrict__ xsum, int32_t* __restrict__ idx, float* __restrict__ wts,
-                   int32_t* __restrict__ asc, int32_t* __restrict__ cnt, int32_t* __restrict__ off,
-                   int32_t* __restrict__ perm, int32_t* __restrict__ slot_of, int32_t* __restrict__ ulist,
-                   int32_t* __restrict__ n_unique, unsigned int* __restrict__ counter, const RouterOpts opts,
-                   double* __restrict__ keys) {
-    constexpr int TT = MAXC > 8 ? 1 : MAXPER > 8 ? 2 : 4;  // tokens per pass (within the register budget)
-    __shared__ double red[kSmallThreads / kWarp][kSmallMaxT];
-    __shared__ double redx[kSmallThreads / kWarp][2];
+// The sum over the warp of eight per-lane values v[0..7], reduced by halves: afterwards lane l
+// holds the total of v[4 b4 + 2 b3 + b2] (b = the bits of l), the same in the four lanes that
+// share those bits.  Fixed order, so every run gives the same value.
+__device__ __forceinline__ double warp_sum8_scatter(const double (&v)[8], int lane) {
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+    double r4[4], r2[2];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const double keep = b4 ? v[j + 4] : v[j], send = b4 ? v[j] : v[j + 4];
+        r4[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const double keep = b3 ? r4[j + 2] : r4[j], send = b3 ? r4[j] : r4[j + 2];
+        r2[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    double s = (b2 ? r2[1] : r2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? r2[0] : r2[1], 4);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    return s;
+}
+
+template <int MAXPER>
+__global__ void __launch_bounds__(kSmallThreads, 1) route_small_kernel(const SmallArgs a) {
+    extern __shared__ __align__(16) uint32_t xsm[];   // [T][32 ns] bf16 pairs of the slice
     __shared__ int s_cnt[kSmallMaxE], s_off[kSmallMaxE], s_scan[kSmallThreads];
     __shared__ int am_last;
-    const int e = blockIdx.x, tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
+    const int g = blockIdx.x, z = blockIdx.y, NG = gridDim.x, KS = gridDim.y;
+    const int tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
+    const int T = a.T, d = a.d, E = a.E, ns = a.ns;
+    const int c0 = 64 * ns * z;                    // the slice's first column
+    const int e = g * kSmallWarps + warp;          // this warp's expert
     // A kernel launched after this one with programmatic dependent launch may start now: it
     // waits (griddepcontrol.wait) before it reads anything written here.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    // ---- logits of expert e for every token, TT tokens per pass: the pass's x loads are all in
-    //      flight at once and its TT fp64 chains are independent.  The router row stays in
-    //      registers (MAXC float4 per thread).  Block b also sums x of the tokens t == b (mod E).
-    const float4* wrow = reinterpret_cast<const float4*>(wr + (size_t)e * d);
-    const int nc = (d / 4 - tid + kSmallThreads - 1) / kSmallThreads;
-    float4 wv[MAXC];
+    // ---- the router-row slice (lane: column pairs 64 i + 2 lane) and x's slice for every token
+    float w0[kSmallMaxSteps], w1[kSmallMaxSteps];
 #pragma unroll
-    for (int j = 0; j < MAXC; ++j)
-        if (j < nc) wv[j] = __ldg(wrow + tid + kSmallThreads * j);
-    int n_sums = 0;                                        // x sums this block owes (tokens e, e + E, ...)
-    for (int t0 = 0; t0 < T; t0 += TT) {
-        uint2 xv[TT][MAXC];
-#pragma unroll
-        for (int u = 0; u < TT; ++u) {
-            const int t = min(t0 + u, T - 1);
-            const uint2* xr2 = reinterpret_cast<const uint2*>(x + (size_t)t * d) + tid;
-#pragma unroll
-            for (int j = 0; j < MAXC; ++j)
-                if (j < nc) xv[u][j] = __ldg(xr2 + kSmallThreads * j);
-        }
-        double a[TT];
-#pragma unroll
-        for (int u = 0; u < TT; ++u) a[u] = 0.0;
-#pragma unroll
-        for (int j = 0; j < MAXC; ++j) {
-            if (j < nc) {
-#pragma unroll
-                for (int u = 0; u < TT; ++u) {
-                    a[u] = fma((double)__uint_as_float(xv[u][j].x << 16), (double)wv[j].x, a[u]);
-                    a[u] = fma((double)__uint_as_float(xv[u][j].x & 0xffff0000u), (double)wv[j].y, a[u]);
-                    a[u] = fma((double)__uint_as_float(xv[u][j].y << 16), (double)wv[j].z, a[u]);
-                    a[u] = fma((double)__uint_as_float(xv[u][j].y & 0xffff0000u), (double)wv[j].w, a[u]);
-                }
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < TT; ++u) {
-            const int t = t0 + u;
-            if (t < T) {
-                const double v = warp_sum_d(a[u]);
-                if (lane == 0) red[warp][t] = v;
-                if (t % E == e) {                          // this block's x sum, from the same loads
-                    double sx = 0.0;
-#pragma unroll
-                    for (int j = 0; j < MAXC; ++j)
-                        if (j < nc)
-                            sx += ((double)__uint_as_float(xv[u][j].x << 16) +
-                                   (double)__uint_as_float(xv[u][j].x & 0xffff0000u)) +
-                                  ((double)__uint_as_float(xv[u][j].y << 16) +
-                                   (double)__uint_as_float(xv[u][j].y & 0xffff0000u));
-                    sx = warp_sum_d(sx);
-                    if (lane == 0) redx[warp][n_sums & 1] = sx;
-                    ++n_sums;
-                }
-            }
-        }
+    for (int i = 0; i < kSmallMaxSteps; ++i) {
+        float2 v = make_float2(0.0f, 0.0f);
+        if (i < ns && e < E) v = __ldg(reinterpret_cast<const float2*>(a.wr + (size_t)e * d + c0 + 64 * i) + lane);
+        w0[i] = v.x;
+        w1[i] = v.y;
+    }
+    const int row16 = 8 * ns;                      // 16-byte groups of a token's slice
+    for (int i = tid; i < T * row16; i += kSmallThreads) {
+        const int t = i / row16, c = i - t * row16;
+        reinterpret_cast<uint4*>(xsm)[i] = ld_ro16(reinterpret_cast<const uint4*>(a.x + (size_t)t * d + c0) + c);
     }
     __syncthreads();
-    if (tid < T) {
-        double s = 0.0;
-        for (int w = 0; w < kSmallThreads / kWarp; ++w) s += red[w][tid];
-        logits[(size_t)tid * E + e] = s;
-        // the selection key here too, so the selecting block needs no exponentials of its own
-        keys[(size_t)tid * E + e] = topk_key(s, bias ? bias[e] : 0.0f, router);
-    }
-    // at most one x sum per block while T <= E; more only for tiny E (then sum them again here)
-    if (n_sums == 1 && tid == 0) {
-        double tot = 0.0;
-        for (int w = 0; w < kSmallThreads / kWarp; ++w) tot += redx[w][0];
-        xsum[e] = tot;
-    } else if (n_sums > 1) {
-        for (int t = e; t < T; t += E) {
-            double sx = 0.0;
-            for (int i = tid; i < d; i += kSmallThreads) sx += (double)bf16_bits_to_f32(x[(size_t)t * d + i]);
-            sx = warp_sum_d(sx);
-            __syncthreads();
-            if (lane == 0) redx[warp][0] = sx;
-            __syncthreads();
-            if (tid == 0) {
-                double tot = 0.0;
-                for (int w = 0; w < kSmallThreads / kWarp; ++w) tot += redx[w][0];
-                xsum[t] = tot;
+    double* const xpart = a.part + (size_t)KS * T * E;     // [KS][T] partial sums of x
+    if (g == 0) {                                  // the slice's x sums, one warp per token
+        for (int t = warp; t < T; t += kSmallWarps) {
+            double s = 0.0;
+            for (int i = 0; i < ns; ++i) {
+                const uint32_t v = xsm[(size_t)t * 32 * ns + 32 * i + lane];
+                s += (double)__uint_as_float(v << 16) + (double)__uint_as_float(v & 0xffff0000u);
             }
+            s = warp_sum_d(s);
+            if (lane == 0) xpart[(size_t)z * T + t] = s;
         }
     }
-    // ---- the last block to finish selects and buckets
+    // ---- partial logits, 8 tokens per pass
+    for (int t0 = 0; t0 < T; t0 += 8) {
+        double acc[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] = 0.0;
+#pragma unroll
+        for (int i = 0; i < kSmallMaxSteps; ++i) {
+            if (i < ns) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int t = min(t0 + j, T - 1);          // rows past T repeat the last (unused)
+                    const uint32_t v = xsm[(size_t)t * 32 * ns + 32 * i + lane];
+                    acc[j] = fma((double)__uint_as_float(v << 16), (double)w0[i], acc[j]);
+                    acc[j] = fma((double)__uint_as_float(v & 0xffff0000u), (double)w1[i], acc[j]);
+                }
+            }
+        }
+        const double s = warp_sum8_scatter(acc, lane);
+        const int t = t0 + 4 * ((lane >> 4) & 1) + 2 * ((lane >> 3) & 1) + ((lane >> 2) & 1);
+        if (e < E && (lane & 3) == 0 && t < T) a.part[((size_t)z * T + t) * E + e] = s;
+    }
+    // ---- the last block of the group: logits and keys of its experts, slices added in order
     __threadfence();
     __syncthreads();
-    if (tid == 0) am_last = atomicAdd(counter, 1u) == gridDim.x - 1;
+    if (tid == 0) am_last = atomicAdd(a.gcnt + g, 1u) == (unsigned)KS - 1u;
     __syncthreads();
     if (!am_last) return;
     __threadfence();
-    for (int t = warp; t < T; t += kSmallThreads / kWarp)
-        warp_select<MAXPER>(logits + (size_t)t * E, keys + (size_t)t * E, E, k, router, scaling, lane, idx + (size_t)t * k,
-                            wts + (size_t)t * k, asc + (size_t)t * k, opts);
+    for (int i = tid; i < T * kSmallWarps; i += kSmallThreads) {
+        const int t = i / kSmallWarps, ee = g * kSmallWarps + (i - t * kSmallWarps);
+        if (ee < E) {
+            double s = 0.0;
+            for (int zz = 0; zz < KS; ++zz) s += __ldcg(a.part + ((size_t)zz * T + t) * E + ee);
+            a.logits[(size_t)t * E + ee] = s;
+            a.keys[(size_t)t * E + ee] = topk_key(s, a.bias ? a.bias[ee] : 0.0f, a.router);
+        }
+    }
+    if (g == 0)
+        for (int t = tid; t < T; t += kSmallThreads) {
+            double s = 0.0;
+            for (int zz = 0; zz < KS; ++zz) s += __ldcg(xpart + (size_t)zz * T + t);
+            a.xsum[t] = s;
+        }
+    if (tid == 0) a.gcnt[g] = 0u;
+    // ---- the last group: select and bucket every token
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) am_last = atomicAdd(a.counter, 1u) == (unsigned)NG - 1u;
+    __syncthreads();
+    if (!am_last) return;
+    __threadfence();
+    const int k = a.k;
+    for (int t = warp; t < T; t += kSmallWarps)
+        warp_select<MAXPER>(a.logits + (size_t)t * E, a.keys + (size_t)t * E, E, k, a.router, a.scaling, lane,
+                            a.idx + (size_t)t * k, a.wts + (size_t)t * k, a.asc + (size_t)t * k, a.opts);
     for (int i = tid; i < E; i += kSmallThreads) s_cnt[i] = 0;
     __syncthreads();
     __threadfence_block();
     for (int i = tid; i < T * k; i += kSmallThreads)
-        if (idx[i] >= 0) atomicAdd(&s_cnt[idx[i]], 1);            // -1: dropped by adaptive top-p
+        if (a.idx[i] >= 0) atomicAdd(&s_cnt[a.idx[i]], 1);         // -1: dropped by adaptive top-p
     __syncthreads();
     // exclusive scan of the counts (each thread owns a run of experts) and of the used flags
     const int per = (E + kSmallThreads - 1) / kSmallThreads;
@@ -367,60 +401,106 @@ route_small_kernel(const float* __restrict__ wr, const float* __restrict__ bias,
         s_scan[tid] += add;
         __syncthreads();
     }
-    int base = tid ? s_scan[tid - 1] : 0;
+    const int base = tid ? s_scan[tid - 1] : 0;
     int run = base & 0xffff, urun = base >> 16;
     for (int i = e0; i < e1; ++i) {
         const int c = s_cnt[i];
         s_off[i] = run;
-        cnt[i] = c;
-        off[i] = run;
-        if (c > 0) ulist[urun++] = i;
+        a.cnt[i] = c;
+        a.off[i] = run;
+        if (c > 0) a.ulist[urun++] = i;
         run += c;
     }
     if (tid == kSmallThreads - 1) {
-        off[E] = s_scan[tid] & 0xffff;
-        *n_unique = s_scan[tid] >> 16;
+        a.off[E] = s_scan[tid] & 0xffff;
+        *a.n_unique = s_scan[tid] >> 16;
     }
     __syncthreads();
     // stable placement in token order (the k experts of a token are distinct)
     if (warp == 0) {
         for (int t = 0; t < T; ++t) {
             if (lane < k) {
-                const int ex = idx[(size_t)t * k + lane];
+                const int ex = a.idx[(size_t)t * k + lane];
                 int p = -1;                                // -1: dropped by adaptive top-p
                 if (ex >= 0) {
                     p = s_off[ex]++;                       // a token's kept experts are distinct
-                    perm[p] = t * k + lane;
+                    a.perm[p] = t * k + lane;
                 }
-                slot_of[(size_t)t * k + lane] = p;
+                a.slot_of[(size_t)t * k + lane] = p;
             }
             __syncwarp();
         }
     }
-    if (tid == 0) *counter = 0u;
+    if (tid == 0) *a.counter = 0u;
+}
+
+// 64-column steps per K slice for a layer of width d and E experts: as many slices (at most 16)
+// as give about one block per SM, each at most 16 steps; 0 if d does not allow it.
+int small_steps(int d, int E, int num_sms) {
+    const int steps = d / 64, ng = (E + kSmallWarps - 1) / kSmallWarps;
+    if (d % 64 || steps < 1) return 0;
+    const int want = std::max(1, std::min(kSmallMaxSlices, (num_sms + ng - 1) / ng));
+    for (int ks = want; ks >= 1; --ks)
+        if (steps % ks == 0 && steps / ks <= kSmallMaxSteps) return steps / ks;
+    for (int ks = want + 1; ks <= kSmallMaxSlices; ++ks)
+        if (steps % ks == 0 && steps / ks <= kSmallMaxSteps) return steps / ks;
+    return 0;
 }
 
 }  // namespace
 
+bool route_small_ok(const LayerDims& L, int num_sms) {
+    return L.E <= kSmallMaxE && small_steps(L.d, L.E, num_sms) > 0;
+}
+
+size_t route_small_part_doubles(int E, int max_tokens) {
+    const size_t t = (size_t)std::min(max_tokens, kSmallMaxT);
+    return (size_t)kSmallMaxSlices * t * ((size_t)E + 1);
+}
+
+size_t route_small_groups(int E) { return (size_t)(E + kSmallWarps - 1) / kSmallWarps; }
+
 cudaError_t launch_route_small(const LayerDims& L, const float* router_w, const float* router_bias, const uint16_t* x,
-                               int T, const Workspace& ws, const Launch& ctx) {
+                               int T, const Workspace& ws, int num_sms, const Launch& ctx) {
     if (T == 0) return cudaSuccess;
-    const float* bias = L.router == MOE_ROUTER_SIGMOID_BIAS ? router_bias : nullptr;
-    unsigned int* counter = reinterpret_cast<unsigned int*>(ws.counter);
-    // router-row registers per thread: 6 float4 cover d <= 6144, 14 cover d <= 14336
-    const bool narrow = (L.d / 4 + kSmallThreads - 1) / kSmallThreads <= 6;
-#define QE_ROUTE_SMALL(MAXPER, MAXC)                                                                              \
-    QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,                                                                      \
-              (route_small_kernel<MAXPER, MAXC><<<L.E, kSmallThreads, 0, ctx.s>>>(                              \
-                  router_w, bias, x, T, L.d, L.E, L.k, L.router, L.scaling, ws.logits, ws.xsum, ws.idx, ws.wts,  \
-                  ws.asc, ws.cnt, ws.off, ws.perm, ws.slot_of, ws.ulist, ws.n_unique, counter, L.ropts, ws.keys)))
-    if (L.E <= 32) {
-        if (narrow) QE_ROUTE_SMALL(1, 6); else QE_ROUTE_SMALL(1, 14);
-    } else if (L.E <= 256) {
-        if (narrow) QE_ROUTE_SMALL(8, 6); else QE_ROUTE_SMALL(8, 14);
-    } else {
-        if (narrow) QE_ROUTE_SMALL(32, 6); else QE_ROUTE_SMALL(32, 14);
-    }
+    if (T > kSmallMaxT) return cudaErrorInvalidValue;
+    const int ns = small_steps(L.d, L.E, num_sms);
+    if (!ns || L.E > kSmallMaxE) return cudaErrorInvalidValue;
+    SmallArgs a;
+    a.wr = router_w;
+    a.bias = L.router == MOE_ROUTER_SIGMOID_BIAS ? router_bias : nullptr;
+    a.x = x;
+    a.T = T;
+    a.d = L.d;
+    a.E = L.E;
+    a.k = L.k;
+    a.router = L.router;
+    a.ns = ns;
+    a.scaling = L.scaling;
+    a.part = ws.rsmall;
+    a.gcnt = ws.rsmall_cnt;
+    a.counter = reinterpret_cast<unsigned int*>(ws.counter);
+    a.logits = ws.logits;
+    a.keys = ws.keys;
+    a.xsum = ws.xsum;
+    a.idx = ws.idx;
+    a.asc = ws.asc;
+    a.cnt = ws.cnt;
+    a.off = ws.off;
+    a.perm = ws.perm;
+    a.slot_of = ws.slot_of;
+    a.ulist = ws.ulist;
+    a.n_unique = ws.n_unique;
+    a.wts = ws.wts;
+    a.opts = L.ropts;
+    const dim3 grid((unsigned)route_small_groups(L.E), (unsigned)(L.d / 64 / ns));
+    const size_t smem = (size_t)T * 128 * ns;
+#define QE_ROUTE_SMALL(MAXPER)                                                          \
+    QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,                                            \
+              (route_small_kernel<MAXPER><<<grid, kSmallThreads, smem, ctx.s>>>(a)))
+    if (L.E <= 32) QE_ROUTE_SMALL(1);
+    else if (L.E <= 256) QE_ROUTE_SMALL(8);
+    else QE_ROUTE_SMALL(32);
 #undef QE_ROUTE_SMALL
     return cudaSuccess;
 }
@@ -430,7 +510,13 @@ cudaError_t launch_route_small(const LayerDims& L, const float* router_w, const 
 cudaError_t prepare_router(const LayerDims& L) {
     const size_t smem = (size_t)kRouterTokens * L.d * sizeof(uint16_t);
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
-    return cudaFuncSetAttribute(router_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    cudaError_t e = cudaFuncSetAttribute(router_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    // the small-batch router's x slices: at most 32 tokens x 16 steps x 128 bytes
+    const int small = kSmallMaxT * kSmallMaxSteps * 128;
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(route_small_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, small);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(route_small_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, small);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(route_small_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, small);
+    return e;
 }
 
 size_t router_split_doubles(int E, int max_tokens) {

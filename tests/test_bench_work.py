@@ -89,17 +89,22 @@ def test_oracle_result_does_not_depend_on_threads():
 def test_traffic_is_reported_only_for_unchanged_sources():
     import json
     rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
-    for kernel in ("fused", "gemm_gateup", "gemm_down"):
-        r = rec[kernel]
+    keys = [key for key in rec if not key.startswith("_")]
+    assert {"glm_decode:fused", "glm_prefill:gemm_gateup", "glm_prefill:gemm_down"} <= set(keys)
+    for key in keys:
+        workload, kernel = key.split(":")
+        assert workload in bench.WORKLOADS
+        r = rec[key]
         fresh = bench.source_sha(r["sources"]) == r["source_sha"]
-        assert bench.traffic_for(kernel) == (r["bytes_per_launch"] if fresh else None)
+        assert bench.traffic_for(kernel, workload) == (r["bytes_per_launch"] if fresh else None)
         assert r["bytes_per_launch"] > 0
-    assert bench.traffic_for("no_such_kernel") is None
+    assert bench.traffic_for("no_such_kernel", "glm_decode") is None
+    assert bench.traffic_for("fused", "no_such_workload") is None
 
 
 def test_traffic_is_null_once_a_source_changes(monkeypatch):
     monkeypatch.setattr(bench, "source_sha", lambda paths: "0" * 16)
-    assert bench.traffic_for("fused") is None
+    assert bench.traffic_for("fused", "glm_decode") is None
 
 
 def test_every_workload_is_measured_once_with_the_headline_first():
