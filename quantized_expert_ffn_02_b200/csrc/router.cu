@@ -243,13 +243,14 @@ struct SmallArgs {
     int32_t *idx, *asc, *cnt, *off, *perm, *slot_of, *ulist, *n_unique;
     float* wts;
     RouterOpts opts;
+    unsigned long long* trace;  // [block][16] %globaltimer at the phase boundaries, or null
 };
 
 // Selection for one token whose logits and keys other blocks wrote (read through L2).
 template <int MAXPER>
 __device__ void warp_select(const double* __restrict__ lg, const double* __restrict__ ky, int E, int k, int router,
                             float scaling, int lane, int32_t* idx_out, float* w_out, int32_t* asc_out,
-                            const RouterOpts& opts) {
+                            const RouterOpts& opts, int32_t* idx_sh) {
     double l[MAXPER], key[MAXPER];
 #pragma unroll
     for (int m = 0; m < MAXPER; ++m) {
@@ -260,6 +261,7 @@ __device__ void warp_select(const double* __restrict__ lg, const double* __restr
     const TopkPick p = warp_topk_keys<MAXPER>(key, l, E, k, router, scaling, lane, opts);
     if (lane < k) {
         idx_out[lane] = p.e;
+        idx_sh[lane] = p.e;
         w_out[lane] = p.w;
         asc_out[p.pos] = lane;
     }
@@ -289,14 +291,24 @@ __device__ __forceinline__ double warp_sum8_scatter(const double (&v)[8], int la
 
 template <int MAXPER>
 __global__ void __launch_bounds__(kSmallThreads, 1) route_small_kernel(const SmallArgs a) {
-    extern __shared__ __align__(16) uint32_t xsm[];   // [T][32 ns] bf16 pairs of the slice
+    extern __shared__ __align__(16) uint32_t xsm[];   // [T][32 ns] bf16 pairs of the slice, then [8][32 ns] fp64 pairs
     __shared__ int s_cnt[kSmallMaxE], s_off[kSmallMaxE], s_scan[kSmallThreads];
+    __shared__ int s_idx[kSmallMaxT * kWarp];        // the chosen experts (k <= 32), for the bucketing
     __shared__ int am_last;
     const int g = blockIdx.x, z = blockIdx.y, NG = gridDim.x, KS = gridDim.y;
     const int tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
     const int T = a.T, d = a.d, E = a.E, ns = a.ns;
     const int c0 = 64 * ns * z;                    // the slice's first column
     const int e = g * kSmallWarps + warp;          // this warp's expert
+    unsigned long long* const tr = a.trace ? a.trace + (size_t)(z * NG + g) * kTraceStamps : nullptr;
+    auto stamp = [&](int i) {
+        if (tid == 0 && tr) {
+            unsigned long long v;
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(v));
+            tr[i] = v;
+        }
+    };
+    stamp(0);
     // A kernel launched after this one with programmatic dependent launch may start now: it
     // waits (griddepcontrol.wait) before it reads anything written here.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -315,6 +327,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1) route_small_kernel(const Sma
         reinterpret_cast<uint4*>(xsm)[i] = ld_ro16(reinterpret_cast<const uint4*>(a.x + (size_t)t * d + c0) + c);
     }
     __syncthreads();
+    stamp(1);
     double* const xpart = a.part + (size_t)KS * T * E;     // [KS][T] partial sums of x
     if (g == 0) {                                  // the slice's x sums, one warp per token
         for (int t = warp; t < T; t += kSmallWarps) {
@@ -327,20 +340,33 @@ __global__ void __launch_bounds__(kSmallThreads, 1) route_small_kernel(const Sma
             if (lane == 0) xpart[(size_t)z * T + t] = s;
         }
     }
-    // ---- partial logits, 8 tokens per pass
+    // ---- partial logits, 8 tokens per pass.  The pass's x slices are converted to fp64 once per
+    //      block, into shared memory after the bf16 rows ([8][32 ns] pairs): converting per use
+    //      (every warp, every element) measured four times slower than the products themselves.
+    double2* const xd = reinterpret_cast<double2*>(xsm + (size_t)T * 32 * ns);
     for (int t0 = 0; t0 < T; t0 += 8) {
+        const int nt = min(8, T - t0);
+        __syncthreads();                                   // the previous pass is done with xd
+        for (int i = tid; i < nt * 32 * ns; i += kSmallThreads) {
+            const int j = i / (32 * ns), p = i - j * 32 * ns;
+            const uint32_t v = xsm[(size_t)(t0 + j) * 32 * ns + p];
+            xd[i] = make_double2((double)__uint_as_float(v << 16), (double)__uint_as_float(v & 0xffff0000u));
+        }
+        __syncthreads();
         double acc[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[j] = 0.0;
 #pragma unroll
         for (int i = 0; i < kSmallMaxSteps; ++i) {
             if (i < ns) {
+                const double wa = w0[i], wb = w1[i];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    const int t = min(t0 + j, T - 1);          // rows past T repeat the last (unused)
-                    const uint32_t v = xsm[(size_t)t * 32 * ns + 32 * i + lane];
-                    acc[j] = fma((double)__uint_as_float(v << 16), (double)w0[i], acc[j]);
-                    acc[j] = fma((double)__uint_as_float(v & 0xffff0000u), (double)w1[i], acc[j]);
+                    if (j < nt) {
+                        const double2 v = xd[(size_t)j * 32 * ns + 32 * i + lane];
+                        acc[j] = fma(v.x, wa, acc[j]);
+                        acc[j] = fma(v.y, wb, acc[j]);
+                    }
                 }
             }
         }
@@ -349,45 +375,63 @@ __global__ void __launch_bounds__(kSmallThreads, 1) route_small_kernel(const Sma
         if (e < E && (lane & 3) == 0 && t < T) a.part[((size_t)z * T + t) * E + e] = s;
     }
     // ---- the last block of the group: logits and keys of its experts, slices added in order
+    stamp(2);
     __threadfence();
     __syncthreads();
     if (tid == 0) am_last = atomicAdd(a.gcnt + g, 1u) == (unsigned)KS - 1u;
     __syncthreads();
+    stamp(3);
     if (!am_last) return;
     __threadfence();
     for (int i = tid; i < T * kSmallWarps; i += kSmallThreads) {
         const int t = i / kSmallWarps, ee = g * kSmallWarps + (i - t * kSmallWarps);
         if (ee < E) {
+            double pz[kSmallMaxSlices];                // every slice's load in flight, then the ordered sum
+#pragma unroll
+            for (int zz = 0; zz < kSmallMaxSlices; ++zz)
+                pz[zz] = zz < KS ? __ldcg(a.part + ((size_t)zz * T + t) * E + ee) : 0.0;
             double s = 0.0;
-            for (int zz = 0; zz < KS; ++zz) s += __ldcg(a.part + ((size_t)zz * T + t) * E + ee);
+#pragma unroll
+            for (int zz = 0; zz < kSmallMaxSlices; ++zz)
+                if (zz < KS) s += pz[zz];
             a.logits[(size_t)t * E + ee] = s;
             a.keys[(size_t)t * E + ee] = topk_key(s, a.bias ? a.bias[ee] : 0.0f, a.router);
         }
     }
     if (g == 0)
         for (int t = tid; t < T; t += kSmallThreads) {
+            double pz[kSmallMaxSlices];
+#pragma unroll
+            for (int zz = 0; zz < kSmallMaxSlices; ++zz) pz[zz] = zz < KS ? __ldcg(xpart + (size_t)zz * T + t) : 0.0;
             double s = 0.0;
-            for (int zz = 0; zz < KS; ++zz) s += __ldcg(xpart + (size_t)zz * T + t);
+#pragma unroll
+            for (int zz = 0; zz < kSmallMaxSlices; ++zz)
+                if (zz < KS) s += pz[zz];
             a.xsum[t] = s;
         }
     if (tid == 0) a.gcnt[g] = 0u;
+    stamp(4);
     // ---- the last group: select and bucket every token
     __threadfence();
     __syncthreads();
     if (tid == 0) am_last = atomicAdd(a.counter, 1u) == (unsigned)NG - 1u;
     __syncthreads();
+    stamp(5);
     if (!am_last) return;
     __threadfence();
     const int k = a.k;
     for (int t = warp; t < T; t += kSmallWarps)
         warp_select<MAXPER>(a.logits + (size_t)t * E, a.keys + (size_t)t * E, E, k, a.router, a.scaling, lane,
-                            a.idx + (size_t)t * k, a.wts + (size_t)t * k, a.asc + (size_t)t * k, a.opts);
+                            a.idx + (size_t)t * k, a.wts + (size_t)t * k, a.asc + (size_t)t * k, a.opts,
+                            s_idx + t * k);
     for (int i = tid; i < E; i += kSmallThreads) s_cnt[i] = 0;
     __syncthreads();
+    stamp(6);
     __threadfence_block();
     for (int i = tid; i < T * k; i += kSmallThreads)
-        if (a.idx[i] >= 0) atomicAdd(&s_cnt[a.idx[i]], 1);         // -1: dropped by adaptive top-p
+        if (s_idx[i] >= 0) atomicAdd(&s_cnt[s_idx[i]], 1);         // -1: dropped by adaptive top-p
     __syncthreads();
+    stamp(7);
     // exclusive scan of the counts (each thread owns a run of experts) and of the used flags
     const int per = (E + kSmallThreads - 1) / kSmallThreads;
     const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
@@ -416,11 +460,12 @@ __global__ void __launch_bounds__(kSmallThreads, 1) route_small_kernel(const Sma
         *a.n_unique = s_scan[tid] >> 16;
     }
     __syncthreads();
+    stamp(8);
     // stable placement in token order (the k experts of a token are distinct)
     if (warp == 0) {
         for (int t = 0; t < T; ++t) {
             if (lane < k) {
-                const int ex = a.idx[(size_t)t * k + lane];
+                const int ex = s_idx[t * k + lane];
                 int p = -1;                                // -1: dropped by adaptive top-p
                 if (ex >= 0) {
                     p = s_off[ex]++;                       // a token's kept experts are distinct
@@ -432,6 +477,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1) route_small_kernel(const Sma
         }
     }
     if (tid == 0) *a.counter = 0u;
+    stamp(9);
 }
 
 // 64-column steps per K slice for a layer of width d and E experts: as many slices (at most 16)
@@ -493,8 +539,9 @@ cudaError_t launch_route_small(const LayerDims& L, const float* router_w, const 
     a.n_unique = ws.n_unique;
     a.wts = ws.wts;
     a.opts = L.ropts;
+    a.trace = L.phase_trace ? ws.trace : nullptr;
     const dim3 grid((unsigned)route_small_groups(L.E), (unsigned)(L.d / 64 / ns));
-    const size_t smem = (size_t)T * 128 * ns;
+    const size_t smem = (size_t)T * 128 * ns + (size_t)8 * 512 * ns;   // bf16 slices, one pass in fp64
 #define QE_ROUTE_SMALL(MAXPER)                                                          \
     QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,                                            \
               (route_small_kernel<MAXPER><<<grid, kSmallThreads, smem, ctx.s>>>(a)))
@@ -512,7 +559,7 @@ cudaError_t prepare_router(const LayerDims& L) {
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(router_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     // the small-batch router's x slices: at most 32 tokens x 16 steps x 128 bytes
-    const int small = kSmallMaxT * kSmallMaxSteps * 128;
+    const int small = kSmallMaxT * kSmallMaxSteps * 128 + 8 * kSmallMaxSteps * 512;
     if (e == cudaSuccess) e = cudaFuncSetAttribute(route_small_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, small);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(route_small_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, small);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(route_small_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, small);

@@ -135,22 +135,27 @@ __device__ __forceinline__ TopkPick warp_topk_keys(double (&key)[MAXPER], const 
             key[m] = -INFINITY;
         }
     if (opts.n_group > 1) limit_groups<MAXPER>(key, E, opts, lane, taken);
+    // Keys as unsigned integers of the same order (-0 folded into +0; the keys are never NaN), so
+    // that each round's warp-wide arg-max is three single-instruction reductions: the largest high
+    // word, then the largest low word among the lanes holding that high word, then the smallest
+    // index among the lanes holding the whole largest key.  0 stands for "none left".
+    unsigned long long ok[MAXPER];
+#pragma unroll
+    for (int m = 0; m < MAXPER; ++m) {
+        const long long b = __double_as_longlong(key[m] + 0.0);
+        ok[m] = b < 0 ? ~(unsigned long long)b : (unsigned long long)b | (1ull << 63);
+    }
     int my_e = -1;
     double my_l = 0.0;
     for (int r = 0; r < k; ++r) {
-        double bk = -INFINITY;
+        unsigned long long bo = 0ull;
         int bi = 0x7fffffff;
 #pragma unroll
-        for (int m = 0; m < MAXPER; ++m) {
-            const int e = lane + kWarp * m;
-            if (!(taken >> m & 1u) && topk_beats(key[m], e, bk, bi)) { bk = key[m]; bi = e; }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const double ok = __shfl_xor_sync(0xffffffffu, bk, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (topk_beats(ok, oi, bk, bi)) { bk = ok; bi = oi; }
-        }
+        for (int m = 0; m < MAXPER; ++m)              // a lane's experts come in ascending index
+            if (!(taken >> m & 1u) && ok[m] > bo) { bo = ok[m]; bi = lane + kWarp * m; }
+        const unsigned hi = (unsigned)(bo >> 32), mh = __reduce_max_sync(0xffffffffu, hi);
+        const unsigned lo = hi == mh ? (unsigned)bo : 0u, ml = __reduce_max_sync(0xffffffffu, lo);
+        bi = (int)__reduce_min_sync(0xffffffffu, hi == mh && lo == ml ? (unsigned)bi : 0xffffffffu);
         // the owner of the winner marks it and hands its logit to lane r
         const int owner = bi % kWarp, wm = bi / kWarp;
         double wl = 0.0;
