@@ -44,14 +44,17 @@ __device__ __forceinline__ TopkPick topk_finish(int my_e, double my_l, int k, in
         // the k weights' total and running share, in rank order (every lane walks the same sums)
         double total = 0.0;
         for (int r2 = 0; r2 < k; ++r2) total += __shfl_sync(0xffffffffu, w, r2);
-        double cum = 0.0;
+        // the running share in rank order; the kept total is that prefix sum where it stops
+        double cum = 0.0, kept = 0.0;
         int m = k;
         for (int r2 = 0; r2 < k; ++r2) {
             cum += __shfl_sync(0xffffffffu, w, r2);
-            if (m == k && cum / total >= top_p) m = r2 + 1;
+            if (cum / total >= top_p) {
+                m = r2 + 1;
+                break;
+            }
         }
-        double kept = 0.0;
-        for (int r2 = 0; r2 < m; ++r2) kept += __shfl_sync(0xffffffffu, w, r2);
+        kept = cum;
         if (lane < m) {
             w = w * (total / kept);
         } else if (mine) {
@@ -71,42 +74,54 @@ __device__ __forceinline__ TopkPick topk_finish(int my_e, double my_l, int k, in
     return p;
 }
 
+// An fp64 key as an unsigned integer of the same order (-0 folded into +0; NaN is not passed),
+// never 0, so that 0 can stand for "none"; and back.
+__device__ __forceinline__ unsigned long long key_order(double v) {
+    const long long b = __double_as_longlong(v + 0.0);
+    return b < 0 ? ~(unsigned long long)b : (unsigned long long)b | (1ull << 63);
+}
+__device__ __forceinline__ double key_value(unsigned long long o) {
+    return __longlong_as_double((long long)(o >> 63 ? o & ~(1ull << 63) : ~o));
+}
+// The warp-wide largest of the lanes' order-mapped values: two single-instruction reductions.
+__device__ __forceinline__ unsigned long long warp_max_order(unsigned long long v) {
+    const unsigned hi = (unsigned)(v >> 32), mh = __reduce_max_sync(0xffffffffu, hi);
+    const unsigned lo = hi == mh ? (unsigned)v : 0u, ml = __reduce_max_sync(0xffffffffu, lo);
+    return ((unsigned long long)mh << 32) | ml;
+}
+
 // Group-limited selection: marks (in `taken`) every expert outside the topk_group best groups.
-// key[m] is the key of expert lane + 32 m.  n_group <= 32 and E % n_group == 0.
+// ok[m] is the order-mapped key of expert lane + 32 m.  n_group <= 32 and E % n_group == 0.
 template <int MAXPER>
-__device__ __forceinline__ void limit_groups(const double (&key)[MAXPER], int E, const RouterOpts& o, int lane,
-                                             uint32_t& taken) {
+__device__ __forceinline__ void limit_groups(const unsigned long long (&ok)[MAXPER], int E, const RouterOpts& o,
+                                             int lane, uint32_t& taken) {
     const int G = o.n_group, per = E / G;
     double my_score = -INFINITY;             // lane g: the score of group g
     for (int g = 0; g < G; ++g) {
-        double b1 = -INFINITY, b2 = -INFINITY;   // the two largest keys of the group, b1 >= b2
+        // this lane's two largest keys of the group (l1 >= l2), then the group's: the largest,
+        // and the largest once the lowest-indexed holder of the largest is set aside
+        unsigned long long l1 = 0ull, l2 = 0ull;
+        int i1 = 0x7fffffff;
 #pragma unroll
         for (int m = 0; m < MAXPER; ++m) {
             const int e = lane + kWarp * m;
             if (e < E && e / per == g) {
-                if (key[m] > b1) { b2 = b1; b1 = key[m]; }
-                else if (key[m] > b2) b2 = key[m];
+                if (ok[m] > l1) { l2 = l1; l1 = ok[m]; i1 = e; }
+                else if (ok[m] > l2) l2 = ok[m];
             }
         }
-#pragma unroll
-        for (int s = 16; s > 0; s >>= 1) {
-            const double o1 = __shfl_xor_sync(0xffffffffu, b1, s), o2 = __shfl_xor_sync(0xffffffffu, b2, s);
-            if (o1 > b1) { b2 = fmax(o2, b1); b1 = o1; }
-            else b2 = fmax(b2, o1);
-        }
-        if (lane == g) my_score = per >= 2 ? b1 + b2 : b1;
+        const unsigned long long m1 = warp_max_order(l1);
+        const unsigned w1 = __reduce_min_sync(0xffffffffu, l1 == m1 ? (unsigned)i1 : 0xffffffffu);
+        const unsigned long long m2 = warp_max_order((unsigned)i1 == w1 ? l2 : l1);
+        if (lane == g) my_score = per >= 2 ? key_value(m1) + key_value(m2) : key_value(m1);
     }
+    // the topk_group best groups (ties to the lower group)
+    const unsigned long long so = lane < G ? key_order(my_score) : 0ull;
     uint32_t keep = 0;
     for (int r = 0; r < o.topk_group; ++r) {
-        double bs = (lane < G && !(keep >> lane & 1u)) ? my_score : -INFINITY;
-        int bg = (lane < G && !(keep >> lane & 1u)) ? lane : 0x7fffffff;
-#pragma unroll
-        for (int s = 16; s > 0; s >>= 1) {
-            const double os = __shfl_xor_sync(0xffffffffu, bs, s);
-            const int og = __shfl_xor_sync(0xffffffffu, bg, s);
-            if (os > bs || (os == bs && og < bg)) { bs = os; bg = og; }
-        }
-        keep |= 1u << bg;
+        const bool open = lane < G && !(keep >> lane & 1u);
+        const unsigned long long mx = warp_max_order(open ? so : 0ull);
+        keep |= 1u << __reduce_min_sync(0xffffffffu, open && so == mx ? (unsigned)lane : 0xffffffffu);
     }
 #pragma unroll
     for (int m = 0; m < MAXPER; ++m) {
@@ -134,17 +149,14 @@ __device__ __forceinline__ TopkPick warp_topk_keys(double (&key)[MAXPER], const 
             taken |= 1u << m;
             key[m] = -INFINITY;
         }
-    if (opts.n_group > 1) limit_groups<MAXPER>(key, E, opts, lane, taken);
-    // Keys as unsigned integers of the same order (-0 folded into +0; the keys are never NaN), so
-    // that each round's warp-wide arg-max is three single-instruction reductions: the largest high
-    // word, then the largest low word among the lanes holding that high word, then the smallest
-    // index among the lanes holding the whole largest key.  0 stands for "none left".
+    // Keys as unsigned integers of the same order (the keys are never NaN), so that each round's
+    // warp-wide arg-max is three single-instruction reductions: the largest high word, then the
+    // largest low word among the lanes holding that high word, then the smallest index among the
+    // lanes holding the whole largest key.  0 stands for "none left".
     unsigned long long ok[MAXPER];
 #pragma unroll
-    for (int m = 0; m < MAXPER; ++m) {
-        const long long b = __double_as_longlong(key[m] + 0.0);
-        ok[m] = b < 0 ? ~(unsigned long long)b : (unsigned long long)b | (1ull << 63);
-    }
+    for (int m = 0; m < MAXPER; ++m) ok[m] = key_order(key[m]);
+    if (opts.n_group > 1) limit_groups<MAXPER>(ok, E, opts, lane, taken);
     int my_e = -1;
     double my_l = 0.0;
     for (int r = 0; r < k; ++r) {
@@ -153,9 +165,8 @@ __device__ __forceinline__ TopkPick warp_topk_keys(double (&key)[MAXPER], const 
 #pragma unroll
         for (int m = 0; m < MAXPER; ++m)              // a lane's experts come in ascending index
             if (!(taken >> m & 1u) && ok[m] > bo) { bo = ok[m]; bi = lane + kWarp * m; }
-        const unsigned hi = (unsigned)(bo >> 32), mh = __reduce_max_sync(0xffffffffu, hi);
-        const unsigned lo = hi == mh ? (unsigned)bo : 0u, ml = __reduce_max_sync(0xffffffffu, lo);
-        bi = (int)__reduce_min_sync(0xffffffffu, hi == mh && lo == ml ? (unsigned)bi : 0xffffffffu);
+        const unsigned long long mx = warp_max_order(bo);
+        bi = (int)__reduce_min_sync(0xffffffffu, bo == mx ? (unsigned)bi : 0xffffffffu);
         // the owner of the winner marks it and hands its logit to lane r
         const int owner = bi % kWarp, wm = bi / kWarp;
         double wl = 0.0;
