@@ -191,21 +191,24 @@ moe_status moe_layer_set_expert(moe_layer *layer, int32_t e, const void *gate_up
 
 /*
  * moe_forward_host -- moe_forward on host buffers: copies x host->device, runs the layer,
- * copies out device->host, and waits for `stream`.  x_host [T][d] bf16; out_host [T][d] fp32
- * or bf16.  Synchronous.  Uses a staging area inside the workspace; pinned host buffers make
- * the copies asynchronous with respect to other streams.
+ * brings out back to the host, and waits for `stream`.  x_host [T][d] bf16; out_host [T][d]
+ * fp32 or bf16.  Synchronous.  x goes through one of two staging areas inside the workspace.
+ * An output of at most 1 MiB in pinned (mapped) host memory is written there by the layer's
+ * last kernel directly; any other output goes through a staging area and one device->host
+ * copy.
  */
 moe_status moe_forward_host(moe_layer *layer, const uint16_t *x_host, int32_t T, void *out_host,
                             moe_stream stream);
 
 /*
- * moe_forward_host_async -- moe_forward_host without the final wait: the host->device copy of
- * x, the layer and the device->host copy of out are enqueued on `stream` and the call returns.
- * Calls on one stream may follow each other at once: stream order keeps each call's copies and
- * kernels apart from the next call's, although they share the layer's staging area.  x_host
- * must stay unchanged until the stream has passed the call (an event or a synchronize), and
- * out_host holds the result only from then on.  With pinned buffers the copies are asynchronous
- * to the host; with pageable ones the runtime may wait inside the call.  Asynchronous.
+ * moe_forward_host_async -- moe_forward_host without the final wait: the layer and the return
+ * of out are enqueued on `stream` and the call returns.  The host->device copy of x runs on a
+ * copy stream of the layer's own, into the staging area the call before last used, so that it
+ * can overlap the previous call's kernels; `stream` waits for it before the layer runs.  Calls
+ * on one stream may follow each other at once.  x_host must stay unchanged until the stream has
+ * passed the call (an event or a synchronize), and out_host holds the result only from then
+ * on.  With pinned buffers the copies are asynchronous to the host; with pageable ones the
+ * runtime may wait inside the call.  Asynchronous.
  */
 moe_status moe_forward_host_async(moe_layer *layer, const uint16_t *x_host, int32_t T, void *out_host,
                                   moe_stream stream);

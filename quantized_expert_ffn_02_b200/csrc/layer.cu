@@ -76,8 +76,12 @@ struct moe_layer {
     int num_sms;
     void* ws_base;
     size_t ws_bytes;
-    uint16_t* x_stage;     // [maxT][d] staging for moe_forward_host
-    void* out_stage;       // [maxT][d] fp32 staging
+    uint16_t* x_stage[2];  // [maxT][d] x staging for the host-buffer calls, used in turn
+    void* out_stage;       // [maxT][d] output staging (when the output cannot be written in place)
+    int x_next = 0;        // the x stage of the next host-buffer call
+    cudaStream_t copy_s = nullptr;           // host -> device copies of x, ahead of the kernels
+    cudaEvent_t x_landed[2] = {nullptr, nullptr};   // a stage's x is on the device
+    cudaEvent_t x_read[2] = {nullptr, nullptr};     // the kernels that read a stage are done
     cudaStream_t last_stream;
     int last_launches;
     qe::Profiler prof;
@@ -93,6 +97,9 @@ struct moe_layer {
 namespace {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+// Outputs up to this size are written straight into mapped pinned host memory by the kernels.
+constexpr size_t kDirectOutputBytes = 1 << 20;
 
 moe_status from_cuda(cudaError_t e) {
     if (e == cudaSuccess) return MOE_OK;
@@ -123,7 +130,7 @@ __global__ void set_expert_kernel(const void** etab, int E, int e, const void* g
 // Carves the workspace out of one allocation.  With base == nullptr it only measures.
 // max_groups > 0 adds the grouped-GEMM path's buffers.
 size_t carve(const moe_config& c, size_t max_groups, char* base, qe::Workspace* ws, uint16_t** x_stage,
-             void** out_stage) {
+             void** out_stage) {   // x_stage: two buffers
     const size_t T = (size_t)c.max_tokens, E = (size_t)c.n_experts, k = (size_t)c.top_k;
     const size_t S = c.n_shared > 0 ? 1 : 0;
     const size_t fmax = S && c.f_shared > c.f ? (size_t)c.f_shared : (size_t)c.f;
@@ -165,12 +172,26 @@ size_t carve(const moe_config& c, size_t max_groups, char* base, qe::Workspace* 
         w.n_groups = (int32_t*)take(sizeof(int32_t) * 2);
         w.xsum_slot = (float*)take(sizeof(float) * slots);
     }
-    uint16_t* xs = (uint16_t*)take(sizeof(uint16_t) * T * (size_t)c.d);
+    uint16_t* xs0 = (uint16_t*)take(sizeof(uint16_t) * T * (size_t)c.d);
+    uint16_t* xs1 = (uint16_t*)take(sizeof(uint16_t) * T * (size_t)c.d);
     void* os = (void*)take(sizeof(float) * T * (size_t)c.d);
     if (ws) *ws = w;
-    if (x_stage) *x_stage = xs;
+    if (x_stage) {
+        x_stage[0] = xs0;
+        x_stage[1] = xs1;
+    }
     if (out_stage) *out_stage = os;
     return o;
+}
+
+void destroy_streams(moe_layer* L) {
+    for (int i = 0; i < 2; ++i) {
+        if (L->x_landed[i]) cudaEventDestroy(L->x_landed[i]);
+        if (L->x_read[i]) cudaEventDestroy(L->x_read[i]);
+        L->x_landed[i] = L->x_read[i] = nullptr;
+    }
+    if (L->copy_s) cudaStreamDestroy(L->copy_s);
+    L->copy_s = nullptr;
 }
 
 moe_status check_config(const moe_config* c, const moe_weights* w) {
@@ -303,7 +324,7 @@ moe_status moe_layer_create(const moe_config* cfg, const moe_weights* w, moe_lay
         delete L;
         return MOE_ERR_OOM;
     }
-    carve(*cfg, max_groups, (char*)L->ws_base, &L->ws, &L->x_stage, &L->out_stage);
+    carve(*cfg, max_groups, (char*)L->ws_base, &L->ws, L->x_stage, &L->out_stage);
     e = cudaMemset(L->ws_base, 0, L->ws_bytes);
     if (e == cudaSuccess) {
         // the pointer table: expert e at its place in the contiguous [E] arrays
@@ -331,6 +352,19 @@ moe_status moe_layer_create(const moe_config* cfg, const moe_weights* w, moe_lay
             delete L;
             return MOE_ERR_CUDA;
         }
+    }
+    // the host-buffer calls' copy stream and the events that order it with the caller's stream
+    e = cudaStreamCreateWithFlags(&L->copy_s, cudaStreamNonBlocking);
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+        e = cudaEventCreateWithFlags(&L->x_landed[i], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L->x_read[i], cudaEventDisableTiming);
+    }
+    if (e != cudaSuccess) {
+        destroy_streams(L);
+        qe::prefill_plan_destroy(L->plan);
+        cudaFree(L->ws_base);
+        delete L;
+        return from_cuda(e);
     }
     L->t1_mode = L->fused_ok ? 2 : qe::decode_t1_supported(L->dims) ? 1 : 0;
     L->last_stream = nullptr;
@@ -423,11 +457,29 @@ moe_status moe_forward_host_async(moe_layer* L, const uint16_t* x_host, int32_t 
     cudaStream_t s = (cudaStream_t)stream;
     const size_t xbytes = sizeof(uint16_t) * (size_t)T * L->cfg.d;
     const size_t obytes = (L->cfg.out_bf16 ? 2 : 4) * (size_t)T * L->cfg.d;
-    cudaError_t e = cudaMemcpyAsync(L->x_stage, x_host, xbytes, cudaMemcpyHostToDevice, s);
+    // x goes in on the layer's copy stream into one of two stages, so that it can land while the
+    // previous call's kernels still run; the stage is reused only once the kernels of the call
+    // before that have read it
+    const int i = L->x_next;
+    L->x_next ^= 1;
+    cudaError_t e = cudaStreamWaitEvent(L->copy_s, L->x_read[i], 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(L->x_stage[i], x_host, xbytes, cudaMemcpyHostToDevice, L->copy_s);
+    if (e == cudaSuccess) e = cudaEventRecord(L->x_landed[i], L->copy_s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, L->x_landed[i], 0);
     if (e != cudaSuccess) return from_cuda(e);
-    moe_status st = moe_forward(L, L->x_stage, T, L->out_stage, stream);
+    // A small output in mapped pinned host memory is written there by the kernels themselves (no
+    // device -> host copy); anything else goes through the staging buffer and one copy.
+    void* direct = nullptr;
+    cudaPointerAttributes pa;
+    if (obytes <= kDirectOutputBytes && cudaPointerGetAttributes(&pa, out_host) == cudaSuccess &&
+        pa.type == cudaMemoryTypeHost && pa.devicePointer && aligned16(pa.devicePointer))
+        direct = pa.devicePointer;
+    cudaGetLastError();                 // a pointer the runtime does not know is not an error here
+    moe_status st = moe_forward(L, L->x_stage[i], T, direct ? direct : L->out_stage, stream);
     if (st != MOE_OK) return st;
-    return from_cuda(cudaMemcpyAsync(out_host, L->out_stage, obytes, cudaMemcpyDeviceToHost, s));
+    e = cudaEventRecord(L->x_read[i], s);
+    if (e == cudaSuccess && !direct) e = cudaMemcpyAsync(out_host, L->out_stage, obytes, cudaMemcpyDeviceToHost, s);
+    return from_cuda(e);
 }
 
 moe_status moe_forward_host(moe_layer* L, const uint16_t* x_host, int32_t T, void* out_host, moe_stream stream) {
@@ -454,6 +506,8 @@ void moe_layer_destroy(moe_layer* L) {
     if (!L) return;
     if (L->last_stream) cudaStreamSynchronize(L->last_stream);
     else cudaDeviceSynchronize();
+    if (L->copy_s) cudaStreamSynchronize(L->copy_s);
+    destroy_streams(L);
     cudaFree(L->ws_base);
     qe::prefill_plan_destroy(L->plan);
     delete L;

@@ -336,6 +336,12 @@ def test_forward_host_matches_device():
     assert np.array_equal(outs[0].numpy(), dev_out)
     assert np.array_equal(outs[2].numpy(), dev_out)
     assert np.array_equal(outs[1].numpy(), run_forward(layer, x[::-1].copy()))
+    # an output in ordinary (pageable) host memory goes through the staging buffer and a copy;
+    # a pinned one is written in place by the kernels: the same values either way
+    op = torch.empty((cfg.T, cfg.d), dtype=torch.float32)
+    assert not op.is_pinned()
+    layer.forward_host(xh, op)
+    assert np.array_equal(op.numpy(), dev_out)
     layer.close()
 
 
