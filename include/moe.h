@@ -250,9 +250,10 @@ void moe_layer_destroy(moe_layer *layer);
  *                               row is read once for both tokens; mode 1 or 0 sends T = 2 to the
  *                               batch kernels.  Such a launch does not write MOE_DEBUG_ULIST.
  */
-/*   MOE_OPT_PROGRAMMATIC_LAUNCH  1 (default): chained kernels of the single-token path start
- *                               early with programmatic dependent launch and wait on the device
- *                               for their inputs; 0: ordinary stream order.  Same results.
+/*   MOE_OPT_PROGRAMMATIC_LAUNCH  1 (default): chained kernels (the single-token kernels, and the
+ *                               batch expert kernels and combine after the router) start early
+ *                               with programmatic dependent launch and wait on the device for
+ *                               their inputs; 0: ordinary stream order.  Same results.
  */
 /*   MOE_OPT_WAIT_LIMIT_US        time limit, in microseconds (100 .. 10,000,000; default 2,000,000), of
  *                               every bounded device-side wait of the grouped-GEMM kernels.  When a

@@ -23,6 +23,7 @@
 // MOE_ERR_RANGE).  Down writes y per slot; the combine adds the chosen experts in ascending
 // expert index, then the shared expert.
 #include "internal.cuh"
+#include "decode_common.cuh"
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -91,6 +92,10 @@ gateup_kernel(const uint8_t* __restrict__ gate_up, const float* __restrict__ gu_
               int f_sh, int S, const int32_t* __restrict__ ulist, const int32_t* __restrict__ n_unique_p,
               const int32_t* __restrict__ cnt, const int32_t* __restrict__ off, const int32_t* __restrict__ perm,
               uint16_t* __restrict__ h, int fmax, int* status, const void* const* __restrict__ etab, int E) {
+    // Launched with programmatic dependent launch after the previous kernel of the layer: wait
+    // for its results before reading anything, then let the next kernel launch.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     constexpr int R = kGateUpRows;
     constexpr int COLS = Kind<WK>::COLS;                          // columns per 16-byte chunk
     constexpr int XV = COLS / 8;                                  // 16-byte x vectors per chunk
@@ -276,6 +281,10 @@ down_kernel(const uint8_t* __restrict__ down, const float* __restrict__ dn_scale
             const int32_t* __restrict__ ulist, const int32_t* __restrict__ n_unique_p,
             const int32_t* __restrict__ cnt, const int32_t* __restrict__ off, const int32_t* __restrict__ perm,
             float* __restrict__ Y, const void* const* __restrict__ etab, int E) {
+    // Launched with programmatic dependent launch after the previous kernel of the layer: wait
+    // for its results before reading anything, then let the next kernel launch.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     constexpr int R = kDownRows;
     constexpr int COLS = Kind<WK>::COLS;
     constexpr int HV = COLS / 8;      // 16-byte h vectors per chunk
@@ -440,6 +449,10 @@ __global__ void __launch_bounds__(kThreads)
 combine_kernel(const float* __restrict__ Y, const float* __restrict__ wts, const int32_t* __restrict__ asc,
                const int32_t* __restrict__ slot_of, int T, int k, int d, int S, void* __restrict__ out,
                int out_bf16) {
+    // Launched with programmatic dependent launch after the previous kernel of the layer: wait
+    // for its results before reading anything, then let the next kernel launch.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int t = blockIdx.y;
     const int j4 = blockIdx.x * blockDim.x + threadIdx.x;
     if (j4 * 4 >= d) return;
@@ -478,16 +491,19 @@ cudaError_t launch_experts_t(const LayerDims& L, const moe_weights& W, const uin
                              const Workspace& ws, int num_sms, const Launch& ctx) {
     const int fmax = L.S && L.f_shared > L.f ? L.f_shared : L.f;
     const unsigned grid = (unsigned)num_sms * 2;
+    const bool pdl = L.pdl != 0;
     QE_LAUNCH(ctx, MOE_KERNEL_GATEUP,
-              (gateup_kernel<WK, TG><<<grid, kThreads, 0, ctx.s>>>(
+              (dec::launch_pdl(pdl, gateup_kernel<WK, TG>, dim3(grid), dim3(kThreads), 0, ctx.s,
                   (const uint8_t*)W.gate_up, W.gate_up_scale, (const uint8_t*)W.shared_gate_up, W.shared_gate_up_scale,
-                  x, ws.xsum, T, L.k, L.d, L.f, L.f_shared, L.S, ws.ulist, ws.n_unique, ws.cnt, ws.off, ws.perm, ws.h,
-                  fmax, ws.status, ws.etab, L.E)));
+                  x, (const double*)ws.xsum, T, L.k, L.d, L.f, L.f_shared, L.S, (const int32_t*)ws.ulist,
+                  (const int32_t*)ws.n_unique, (const int32_t*)ws.cnt, (const int32_t*)ws.off, (const int32_t*)ws.perm,
+                  ws.h, fmax, ws.status, (const void* const*)ws.etab, L.E)));
     QE_LAUNCH(ctx, MOE_KERNEL_DOWN,
-              (down_kernel<WK, TG><<<grid, kThreads, 0, ctx.s>>>(
-                  (const uint8_t*)W.down, W.down_scale, (const uint8_t*)W.shared_down, W.shared_down_scale, ws.h, fmax,
-                  T, L.k, L.d, L.f, L.f_shared, L.S, ws.ulist, ws.n_unique, ws.cnt, ws.off, ws.perm, ws.Y, ws.etab,
-                  L.E)));
+              (dec::launch_pdl(pdl, down_kernel<WK, TG>, dim3(grid), dim3(kThreads), 0, ctx.s,
+                  (const uint8_t*)W.down, W.down_scale, (const uint8_t*)W.shared_down, W.shared_down_scale,
+                  (const uint16_t*)ws.h, fmax, T, L.k, L.d, L.f, L.f_shared, L.S, (const int32_t*)ws.ulist,
+                  (const int32_t*)ws.n_unique, (const int32_t*)ws.cnt, (const int32_t*)ws.off, (const int32_t*)ws.perm,
+                  ws.Y, (const void* const*)ws.etab, L.E)));
     return cudaSuccess;
 }
 
@@ -518,8 +534,9 @@ cudaError_t launch_combine(const LayerDims& L, int T, const Workspace& ws, void*
     if (T == 0) return cudaSuccess;
     dim3 grid((unsigned)((L.d / 4 + kThreads - 1) / kThreads), (unsigned)T);
     QE_LAUNCH(ctx, MOE_KERNEL_COMBINE,
-              (combine_kernel<<<grid, kThreads, 0, ctx.s>>>(ws.Y, ws.wts, ws.asc, ws.slot_of, T, L.k, L.d, L.S, out,
-                                                             L.out_bf16)));
+              (dec::launch_pdl(L.pdl != 0, combine_kernel, grid, dim3(kThreads), 0, ctx.s, (const float*)ws.Y,
+                               (const float*)ws.wts, (const int32_t*)ws.asc, (const int32_t*)ws.slot_of, T, L.k, L.d,
+                               L.S, out, L.out_bf16)));
     return cudaSuccess;
 }
 

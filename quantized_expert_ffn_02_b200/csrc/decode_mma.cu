@@ -133,6 +133,10 @@ struct Unit {
 
 template <bool GU>
 __global__ void __launch_bounds__(kUMaxWarps * kWarp, 1) union_mma_kernel(const UArgs a) {
+    // Launched with programmatic dependent launch after the previous kernel of the layer: wait
+    // for its results before reading anything, then let the next kernel launch.
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bars[kUMaxWarps][kUStages];
     __shared__ __align__(8) uint64_t vbar;                 // a unit's v rows landed
@@ -535,7 +539,7 @@ cudaError_t launch_decode_mma(const LayerDims& L, const moe_weights& W, const ui
         const int warps = union_warps(vb, u_stage<true>());
         const size_t smem = vb + (size_t)warps * kUStages * u_stage<true>();
         QE_LAUNCH(ctx, MOE_KERNEL_GATEUP,
-                  (union_mma_kernel<true><<<num_sms, warps * kWarp, smem, ctx.s>>>(g)));
+                  (launch_pdl(L.pdl != 0, union_mma_kernel<true>, dim3(num_sms), dim3(warps * kWarp), smem, ctx.s, g)));
     }
     // down: v = h, out y
     {
@@ -550,7 +554,7 @@ cudaError_t launch_decode_mma(const LayerDims& L, const moe_weights& W, const ui
         const int warps = union_warps(vb, u_stage<false>());
         const size_t smem = vb + (size_t)warps * kUStages * u_stage<false>();
         QE_LAUNCH(ctx, MOE_KERNEL_DOWN,
-                  (union_mma_kernel<false><<<num_sms, warps * kWarp, smem, ctx.s>>>(dn)));
+                  (launch_pdl(L.pdl != 0, union_mma_kernel<false>, dim3(num_sms), dim3(warps * kWarp), smem, ctx.s, dn)));
     }
     return cudaSuccess;
 }
