@@ -424,31 +424,50 @@ __global__ void __launch_bounds__(kSmallThreads, 1) route_small_kernel(const Sma
         warp_select<MAXPER>(a.logits + (size_t)t * E, a.keys + (size_t)t * E, E, k, a.router, a.scaling, lane,
                             a.idx + (size_t)t * k, a.wts + (size_t)t * k, a.asc + (size_t)t * k, a.opts,
                             s_idx + t * k);
+    // Bucketing.  s_cnt[e] becomes the set of tokens that chose expert e (a bit per token:
+    // T <= 32); its population is the count, and an entry's slot is its expert's offset plus
+    // the number of earlier tokens in that set (stable, in token order).
     for (int i = tid; i < E; i += kSmallThreads) s_cnt[i] = 0;
     __syncthreads();
     stamp(6);
-    __threadfence_block();
     for (int i = tid; i < T * k; i += kSmallThreads)
-        if (s_idx[i] >= 0) atomicAdd(&s_cnt[s_idx[i]], 1);         // -1: dropped by adaptive top-p
+        if (s_idx[i] >= 0) atomicOr(reinterpret_cast<unsigned*>(&s_cnt[s_idx[i]]), 1u << (i / k));  // -1: dropped
     __syncthreads();
     stamp(7);
-    // exclusive scan of the counts (each thread owns a run of experts) and of the used flags
+    // exclusive scan of (count, used) over the experts: each thread a run of experts, then a
+    // warp scan and a scan of the warp totals
     const int per = (E + kSmallThreads - 1) / kSmallThreads;
     const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
     int sum = 0, used = 0;
-    for (int i = e0; i < e1; ++i) { sum += s_cnt[i]; used += s_cnt[i] > 0; }
-    s_scan[tid] = sum | (used << 16);       // T*k <= 1024 < 2^16 and E <= 1024 < 2^16
-    __syncthreads();
-    for (int o = 1; o < kSmallThreads; o <<= 1) {
-        const int add = tid >= o ? s_scan[tid - o] : 0;
-        __syncthreads();
-        s_scan[tid] += add;
-        __syncthreads();
+    for (int i = e0; i < e1; ++i) {
+        const int c = __popc((unsigned)s_cnt[i]);
+        sum += c;
+        used += c > 0;
     }
-    const int base = tid ? s_scan[tid - 1] : 0;
+    const int mine = sum | (used << 16);     // T*k <= 1024 < 2^16 and E <= 1024 < 2^16
+    int v = mine;
+#pragma unroll
+    for (int o = 1; o < kWarp; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += y;
+    }
+    if (lane == kWarp - 1) s_scan[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < kSmallWarps ? s_scan[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < kWarp; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        if (lane < kSmallWarps) s_scan[kSmallWarps + lane] = w;
+    }
+    __syncthreads();
+    const int incl = v + (warp ? s_scan[kSmallWarps + warp - 1] : 0);
+    const int base = incl - mine;
     int run = base & 0xffff, urun = base >> 16;
     for (int i = e0; i < e1; ++i) {
-        const int c = s_cnt[i];
+        const int c = __popc((unsigned)s_cnt[i]);
         s_off[i] = run;
         a.cnt[i] = c;
         a.off[i] = run;
@@ -456,25 +475,19 @@ __global__ void __launch_bounds__(kSmallThreads, 1) route_small_kernel(const Sma
         run += c;
     }
     if (tid == kSmallThreads - 1) {
-        a.off[E] = s_scan[tid] & 0xffff;
-        *a.n_unique = s_scan[tid] >> 16;
+        a.off[E] = incl & 0xffff;
+        *a.n_unique = incl >> 16;
     }
     __syncthreads();
     stamp(8);
-    // stable placement in token order (the k experts of a token are distinct)
-    if (warp == 0) {
-        for (int t = 0; t < T; ++t) {
-            if (lane < k) {
-                const int ex = s_idx[t * k + lane];
-                int p = -1;                                // -1: dropped by adaptive top-p
-                if (ex >= 0) {
-                    p = s_off[ex]++;                       // a token's kept experts are distinct
-                    a.perm[p] = t * k + lane;
-                }
-                a.slot_of[(size_t)t * k + lane] = p;
-            }
-            __syncwarp();
+    for (int i = tid; i < T * k; i += kSmallThreads) {
+        const int ex = s_idx[i], t = i / k;
+        int p = -1;                                        // -1: dropped by adaptive top-p
+        if (ex >= 0) {
+            p = s_off[ex] + __popc((unsigned)s_cnt[ex] & ((1u << t) - 1u));
+            a.perm[p] = i;
         }
+        a.slot_of[i] = p;
     }
     if (tid == 0) *a.counter = 0u;
     stamp(9);
