@@ -225,7 +225,7 @@ constexpr int kSmallThreads = 512;
 constexpr int kSmallWarps = kSmallThreads / kWarp;      // experts per block
 constexpr int kSmallMaxT = 32;
 constexpr int kSmallMaxE = 1024;
-constexpr int kSmallMaxSteps = 16;                      // 64-column steps per slice (32 floats per lane)
+constexpr int kSmallMaxSteps = 12;                      // 64-column steps per slice (the fp64 tiles fit)
 constexpr int kSmallMaxSlices = 16;
 
 struct SmallArgs {
@@ -312,14 +312,24 @@ __global__ void __launch_bounds__(kSmallThreads, 1) route_small_kernel(const Sma
     // A kernel launched after this one with programmatic dependent launch may start now: it
     // waits (griddepcontrol.wait) before it reads anything written here.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    // ---- the router-row slice (lane: column pairs 64 i + 2 lane) and x's slice for every token
-    float w0[kSmallMaxSteps], w1[kSmallMaxSteps];
-#pragma unroll
-    for (int i = 0; i < kSmallMaxSteps; ++i) {
-        float2 v = make_float2(0.0f, 0.0f);
-        if (i < ns && e < E) v = __ldg(reinterpret_cast<const float2*>(a.wr + (size_t)e * d + c0 + 64 * i) + lane);
-        w0[i] = v.x;
-        w1[i] = v.y;
+    // ---- shared memory: x's slice for every token (bf16), then fp64 tiles: the group's 16
+    //      router-row slices [16][kc + 4] and one pass's 8 token slices [8][kc + 4] (rows padded
+    //      by 4 doubles so that each half-warp's fragment loads meet 32 distinct banks), then the
+    //      warps' partial products [16][64]
+    const int kc = 64 * ns, pitch = kc + 4;        // columns of the slice, row pitch (doubles)
+    double* const wd = reinterpret_cast<double*>(xsm + (size_t)T * 32 * ns);
+    double* const xd = wd + (size_t)kSmallWarps * pitch;
+    double* const red = xd + (size_t)8 * pitch;
+    for (int i = tid; i < kSmallWarps * (kc / 4); i += kSmallThreads) {     // the router slices, in fp64
+        const int r = i / (kc / 4), c = i - r * (kc / 4);
+        const int ee = g * kSmallWarps + r;
+        const float4 v = ee < E ? __ldg(reinterpret_cast<const float4*>(a.wr + (size_t)ee * d + c0) + c)
+                                : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        double* const dst = wd + (size_t)r * pitch + 4 * c;
+        dst[0] = v.x;
+        dst[1] = v.y;
+        dst[2] = v.z;
+        dst[3] = v.w;
     }
     const int row16 = 8 * ns;                      // 16-byte groups of a token's slice
     for (int i = tid; i < T * row16; i += kSmallThreads) {
@@ -340,39 +350,45 @@ __global__ void __launch_bounds__(kSmallThreads, 1) route_small_kernel(const Sma
             if (lane == 0) xpart[(size_t)z * T + t] = s;
         }
     }
-    // ---- partial logits, 8 tokens per pass.  The pass's x slices are converted to fp64 once per
-    //      block, into shared memory after the bf16 rows ([8][32 ns] pairs): converting per use
-    //      (every warp, every element) measured four times slower than the products themselves.
-    double2* const xd = reinterpret_cast<double2*>(xsm + (size_t)T * 32 * ns);
+    // ---- partial logits on the fp64 tensor cores (mma.sync m8n8k4), 8 tokens per pass: the
+    //      block's 16 experts are two 8-expert tiles, and each tile's K slice is dealt to 8 warps
+    //      (kc / 8 columns each); the 8 partial tiles are then added in warp order.
+    const int tile = warp >> 3, kp = warp & 7, fg = lane >> 2, fq = lane & 3;
+    const int kw = kc / 8;                         // columns per warp
     for (int t0 = 0; t0 < T; t0 += 8) {
         const int nt = min(8, T - t0);
-        __syncthreads();                                   // the previous pass is done with xd
-        for (int i = tid; i < nt * 32 * ns; i += kSmallThreads) {
-            const int j = i / (32 * ns), p = i - j * 32 * ns;
-            const uint32_t v = xsm[(size_t)(t0 + j) * 32 * ns + p];
-            xd[i] = make_double2((double)__uint_as_float(v << 16), (double)__uint_as_float(v & 0xffff0000u));
+        __syncthreads();                                   // the previous pass is done with xd, red
+        for (int i = tid; i < 8 * (kc / 2); i += kSmallThreads) {      // x pairs of the pass, fp64
+            const int j = i / (kc / 2), pr = i - j * (kc / 2);
+            uint32_t v = 0u;                                // tokens past T: zeros (unused)
+            if (j < nt) v = xsm[(size_t)(t0 + j) * 32 * ns + pr];
+            double* const dst = xd + (size_t)j * pitch + 2 * pr;
+            dst[0] = (double)__uint_as_float(v << 16);
+            dst[1] = (double)__uint_as_float(v & 0xffff0000u);
         }
         __syncthreads();
-        double acc[8];
+        // A (8 x 4): lane (fg, fq) holds x[token fg][k + fq]; B (4 x 8): w[expert fg][k + fq];
+        // C: tokens fg, experts 2 fq and 2 fq + 1 of the tile
+        double c0v = 0.0, c1v = 0.0;
+        const double* const xa = xd + (size_t)fg * pitch + kp * kw + fq;
+        const double* const wb = wd + (size_t)(8 * tile + fg) * pitch + kp * kw + fq;
+#pragma unroll 4
+        for (int kk = 0; kk < kw; kk += 4)
+            asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+                         : "+d"(c0v), "+d"(c1v)
+                         : "d"(xa[kk]), "d"(wb[kk]));
+        red[(size_t)warp * 64 + 2 * lane] = c0v;
+        red[(size_t)warp * 64 + 2 * lane + 1] = c1v;
+        __syncthreads();
+        if (tid < 128) {                                   // (tile, token, expert of the tile)
+            const int tl = tid >> 6, o = tid & 63;         // o: the C element (lane o / 2, o % 2)
+            double sum = 0.0;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = 0.0;
-#pragma unroll
-        for (int i = 0; i < kSmallMaxSteps; ++i) {
-            if (i < ns) {
-                const double wa = w0[i], wb = w1[i];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (j < nt) {
-                        const double2 v = xd[(size_t)j * 32 * ns + 32 * i + lane];
-                        acc[j] = fma(v.x, wa, acc[j]);
-                        acc[j] = fma(v.y, wb, acc[j]);
-                    }
-                }
-            }
+            for (int p = 0; p < 8; ++p) sum += red[(size_t)(8 * tl + p) * 64 + o];
+            const int tok = o >> 3, ex = 8 * tl + 2 * ((o >> 1) & 3) + (o & 1);
+            const int t = t0 + tok, ee = g * kSmallWarps + ex;
+            if (ee < E && t < T) a.part[((size_t)z * T + t) * E + ee] = sum;
         }
-        const double s = warp_sum8_scatter(acc, lane);
-        const int t = t0 + 4 * ((lane >> 4) & 1) + 2 * ((lane >> 3) & 1) + ((lane >> 2) & 1);
-        if (e < E && (lane & 3) == 0 && t < T) a.part[((size_t)z * T + t) * E + e] = s;
     }
     // ---- the last block of the group: logits and keys of its experts, slices added in order
     stamp(2);
@@ -554,7 +570,8 @@ cudaError_t launch_route_small(const LayerDims& L, const float* router_w, const 
     a.opts = L.ropts;
     a.trace = L.phase_trace ? ws.trace : nullptr;
     const dim3 grid((unsigned)route_small_groups(L.E), (unsigned)(L.d / 64 / ns));
-    const size_t smem = (size_t)T * 128 * ns + (size_t)8 * 512 * ns;   // bf16 slices, one pass in fp64
+    // bf16 slices of every token, the fp64 router slices and one pass's fp64 x, the partial tiles
+    const size_t smem = (size_t)T * 128 * ns + (size_t)(kSmallWarps + 8) * (64 * ns + 4) * 8 + 16 * 64 * 8;
 #define QE_ROUTE_SMALL(MAXPER)                                                          \
     QE_LAUNCH(ctx, MOE_KERNEL_ROUTER_LOGITS,                                            \
               (route_small_kernel<MAXPER><<<grid, kSmallThreads, smem, ctx.s>>>(a)))
@@ -572,7 +589,7 @@ cudaError_t prepare_router(const LayerDims& L) {
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(router_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     // the small-batch router's x slices: at most 32 tokens x 16 steps x 128 bytes
-    const int small = kSmallMaxT * kSmallMaxSteps * 128 + 8 * kSmallMaxSteps * 512;
+    const int small = kSmallMaxT * kSmallMaxSteps * 128 + (kSmallWarps + 8) * (64 * kSmallMaxSteps + 4) * 8 + 16 * 64 * 8;
     if (e == cudaSuccess) e = cudaFuncSetAttribute(route_small_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, small);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(route_small_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, small);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(route_small_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, small);
