@@ -321,7 +321,12 @@ moe_status moe_layer_get_option(const moe_layer *layer, int32_t option, int64_t 
  *                    barrier, 3 x rearranged and the shared rows done, 4 first grid barrier passed,
  *                    5 router pieces gathered, 12 candidates, 13 ranks and pointers, 14 and 15
  *                    around a proxy fence, 6 experts selected, 7 routed gate/up done, 8 h
- *                    complete, 9 down done, 10 output stored
+ *                    complete, 9 down done, 10 output stored.  A call that runs the
+ *                    small-batch router (2 <= T <= 32, or T = 1 off the single launch) writes
+ *                    one row per router block instead (block z * groups + g): 0 start, 1 x and
+ *                    the router slice staged, 2 partial logits stored, 3 past the group's
+ *                    counter, 4 the group's logits stored, 5 past the last counter, then in
+ *                    the last block 6 selection done, 7 counted, 8 offsets, 9 slots placed
  */
 enum { MOE_DEBUG_H = 0, MOE_DEBUG_Y = 1, MOE_DEBUG_IDX = 2, MOE_DEBUG_W = 3, MOE_DEBUG_ASC = 4,
        MOE_DEBUG_ULIST = 5, MOE_DEBUG_CNT = 6, MOE_DEBUG_XSUM = 7, MOE_DEBUG_TRACE = 8 };
