@@ -118,21 +118,17 @@ struct FusedArgs {
     float scaling;
 };
 
-__device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long* p) {
-    unsigned long long v;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p));
-    return v;
-}
 __device__ __forceinline__ unsigned long long ld_acquire(const unsigned long long* p) {
     unsigned long long v;
     asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
-// Arrive: this CTA's earlier writes (ordered before by __syncthreads) become visible first.  The
-// add returns nothing, so the arriving thread goes straight on to its wait.  One thread calls it.
-__device__ __forceinline__ void arrive(unsigned long long* count) {
+// Arrive: this CTA's earlier writes (ordered before by __syncthreads) become visible first.
+// Returns the count before the arrival.  One thread calls it.  (A fire-and-forget add in its
+// place measured slower: the other CTAs saw the last arrival about 1 us later.)
+__device__ __forceinline__ unsigned long long arrive(unsigned long long* count) {
     __threadfence();
-    asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(count), "l"(1ull) : "memory");
+    return atomicAdd(count, 1ull);
 }
 // Bounded wait until the arrival count reaches `target`.  One thread calls it.
 __device__ bool wait_arrivals(const unsigned long long* count, unsigned long long target) {
@@ -507,16 +503,6 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
         bar_expect_tx(saddr(&s_xbar), 2u * d * NT);
         bulk_g2s(xraw_s, a.x, 2u * d * NT, saddr(&s_xbar));
     }
-    // Arrivals before this launch: a multiple of 2G.  Until this CTA arrives, at most G - 1
-    // arrivals of this launch (all at barrier 0) can have landed, so the count read here rounds
-    // down to that base (thread 0 uses it at its arrival).
-    const unsigned long long bar_v0 = tid == 0 ? ld_relaxed(a.bar) : 0ull;
-    // the layer's expert pointer table is read during the selection: bring it into L2 now
-    if (tid == 2 * kWarp) prefetch_l2(a.etab, 32u * (uint32_t)E);
-    // selection: the CTA's halves take one token each (NT = 2); thread ltid of half tt holds
-    // expert ltid of token tt (its bias is loaded now, used after barrier 0)
-    const int nwh = nwc / NT, tt = warp / nwh, lw = warp - tt * nwh, ltid = tid - tt * nwh * kWarp;
-    const float my_bias = a.bias && ltid < E ? __ldg(a.bias + ltid) : 0.0f;
 
     // ---- the ring: use q of this warp goes to stage q % nst
     //      q < my_tasks: gate/up row pair (task q); q >= my_tasks: down stage (lane 0's cursor)
@@ -692,10 +678,14 @@ __global__ void __launch_bounds__(kFzMaxThreads, 1) decode_fused_kernel(const Fu
         xoffs[tk] = 8.0f * (float)xs[tk] * exp2i(-sig[tk]);
         xunscale[tk] = exp2i(-sig[tk]) * 16777216.0f;
     }
+    // selection: the CTA's halves take one token each (NT = 2); thread ltid of half tt holds
+    // expert ltid of token tt
+    const int nwh = nwc / NT, tt = warp / nwh, lw = warp - tt * nwh, ltid = tid - tt * nwh * kWarp;
+    const float my_bias = a.bias && ltid < E ? a.bias[ltid] : 0.0f;
     __syncthreads();                                       // the last stage (x) is free
     if (tid == 0) {                                        // barrier 0: every piece is stored
-        s_base = bar_v0 - bar_v0 % (2ull * G);
-        arrive(a.bar);
+        const unsigned long long old = arrive(a.bar);
+        s_base = old - old % (2ull * G);
     }
     stamp(2);
 
